@@ -1,0 +1,329 @@
+// api.cu -- the C ABI of libmoe_b200.so (declared in include/moe.h): argument
+// checks, the workspace carve-up and the launch sequence of each entry point.
+#include "kernels.h"
+#include "../../include/moe.h"
+
+#include <stdint.h>
+#include <string.h>
+
+namespace {
+
+using namespace moe;
+
+constexpr size_t ALIGN = 256;
+
+inline size_t up(size_t v) { return (v + ALIGN - 1) & ~(ALIGN - 1); }
+
+// Workspace regions.  The status block sits at offset 0 so moe_get_status can
+// find it without the shape.  The routing part depends on (T, E, k) only and is
+// all moe_route / moe_permute need; the plan part adds the band tables; the
+// last part holds the permuted activations and the expert intermediates.
+struct Layout {
+  size_t status, sync, blk_hist, blk_base, counts, offsets, topk_idx, topk_gate, perm, row_of, arrive;
+  size_t routing_end;
+  size_t sorted_e, band_start, tile_start1, bands, band_done1, band_done2;
+  size_t plan_end;
+  size_t x_perm, h, y;
+  size_t total;
+};
+
+Layout layout(int T, int d, int f, int E, int k) {
+  Layout L;
+  const size_t R = (size_t)T * k;
+  const size_t nblk = (size_t)route_blocks(T);
+  const size_t mb = (size_t)max_bands((int)R, E);
+  size_t o = 0;
+  L.status = o; o = up(o + sizeof(Status));
+  L.sync = o; o = up(o + sizeof(Sync));
+  L.blk_hist = o; o = up(o + nblk * E * 4);
+  L.blk_base = o; o = up(o + nblk * E * 4);
+  L.counts = o; o = up(o + (size_t)E * 4);
+  L.offsets = o; o = up(o + (size_t)(E + 1) * 4);
+  L.topk_idx = o; o = up(o + R * 4);
+  L.topk_gate = o; o = up(o + R * 4);
+  L.perm = o; o = up(o + R * 4);
+  L.row_of = o; o = up(o + R * 4);
+  L.arrive = o; o = up(o + (size_t)T * 4);
+  L.routing_end = o;
+  L.sorted_e = o; o = up(o + (size_t)E * 4);
+  L.band_start = o; o = up(o + (size_t)(E + 1) * 4);
+  L.tile_start1 = o; o = up(o + (size_t)(E + 1) * 4);
+  L.bands = o; o = up(o + mb * sizeof(Band));
+  L.band_done1 = o; o = up(o + mb * 4);
+  L.band_done2 = o; o = up(o + mb * 4);
+  L.plan_end = o;
+  L.x_perm = o; o = up(o + R * d * 2);
+  L.h = o; o = up(o + R * f * 2);
+  L.y = o; o = up(o + R * d * 2);
+  L.total = o;
+  return L;
+}
+
+template <class T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+Work work_from(void* ws, const Layout& L, bool plan, bool acts) {
+  Work w;
+  memset(&w, 0, sizeof(w));
+  w.status = at<Status>(ws, L.status);
+  w.sync = at<Sync>(ws, L.sync);
+  w.blk_hist = at<int32_t>(ws, L.blk_hist);
+  w.blk_base = at<int32_t>(ws, L.blk_base);
+  w.counts = at<int32_t>(ws, L.counts);
+  w.offsets = at<int32_t>(ws, L.offsets);
+  w.topk_idx = at<int32_t>(ws, L.topk_idx);
+  w.topk_gate = at<float>(ws, L.topk_gate);
+  w.perm = at<int32_t>(ws, L.perm);
+  w.row_of = at<int32_t>(ws, L.row_of);
+  w.arrive = at<uint32_t>(ws, L.arrive);
+  if (plan) {
+    w.sorted_e = at<int32_t>(ws, L.sorted_e);
+    w.band_start = at<int32_t>(ws, L.band_start);
+    w.tile_start1 = at<int32_t>(ws, L.tile_start1);
+    w.bands = at<Band>(ws, L.bands);
+    w.band_done1 = at<uint32_t>(ws, L.band_done1);
+    w.band_done2 = at<uint32_t>(ws, L.band_done2);
+  }
+  if (acts) {
+    w.x_perm = at<__nv_bfloat16>(ws, L.x_perm);
+    w.h = at<__nv_bfloat16>(ws, L.h);
+    w.y = at<__nv_bfloat16>(ws, L.y);
+  }
+  return w;
+}
+
+// Shape checks: MOE_ERR_INVALID for meaningless shapes, MOE_ERR_UNSUPPORTED for
+// valid MoE shapes outside what the kernels tile.
+moe_status check_route_shape(int T, int E, int k) {
+  if (T < 1 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID;
+  if (E > MAX_E || k > MAX_K) return MOE_ERR_UNSUPPORTED;
+  if ((long long)T * k > (1LL << 30)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_shape(int T, int d, int f, int E, int k) {
+  moe_status s = check_route_shape(T, E, k);
+  if (s != MOE_OK) return s;
+  if (d < 1 || f < 1) return MOE_ERR_INVALID;
+  if (d % BN2 != 0 || f % BN1 != 0) return MOE_ERR_UNSUPPORTED;
+  if ((long long)T * k * (d > f ? d : f) >= (1LL << 40)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+inline bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+
+int sms_cache[64] = {0};
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64 && sms_cache[dev] > 0) return sms_cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) sms_cache[dev] = n;
+  return n;
+}
+
+// Per-SM throughputs for the split cost model, from B200 measurements: a
+// producer SM sustains about 1/148 of ~1.0 PFLOP/s of bf16 MMA inside this
+// kernel, one consumer SM moves about 40 GB/s of combine traffic, HBM ~6.5 TB/s.
+CostModel default_cost_model() {
+  CostModel cm;
+  cm.mma_flops_per_sm = 1.0e15f / 148.0f;
+  cm.copy_bytes_per_sm = 40.0e9f;
+  cm.hbm_bytes = 6.5e12f;
+  cm.max_consumers = 32;
+  return cm;
+}
+
+inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                                   \
+  do {                                                  \
+    cudaError_t e_ = (expr);                            \
+    if (e_ != cudaSuccess) return MOE_ERR_CUDA;         \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(int T, int d, int f, int E, int k) {
+  if (check_shape(T, d, f, E, k) != MOE_OK) return 0;
+  return layout(T, d, f, E, k).total;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int moe_num_sms(void) { return device_sms(); }
+
+moe_status moe_route(const float* logits, int T, int E, int k, int32_t* topk_idx,
+                     float* topk_gate, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = check_route_shape(T, E, k);
+  if (s != MOE_OK) return s;
+  if (!ok_ptr(logits) || !ok_ptr(topk_idx) || !ok_ptr(topk_gate) || !ok_opt(counts))
+    return MOE_ERR_INVALID;
+  // any shape's full workspace covers the routing part; d/f do not matter here
+  const Layout L = layout(T, BN2, BN1, E, k);
+  if (!ws || !aligned16(ws) || ws_bytes < L.routing_end) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Work w = work_from(ws, L, false, false);
+  MOE_TRY(launch_route(logits, T, E, k, topk_idx, topk_gate, w.blk_hist, nullptr, st));
+  if (counts) MOE_TRY(launch_colsum(w.blk_hist, route_blocks(T), E, counts, st));
+  return MOE_OK;
+}
+
+moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t* topk_idx,
+                       int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* row_of,
+                       void* x_perm, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = check_route_shape(T, E, k);
+  if (s != MOE_OK) return s;
+  if (d < 1) return MOE_ERR_INVALID;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!ok_ptr(x) || !ok_ptr(topk_idx) || !ok_ptr(offsets) || !ok_ptr(perm) || !ok_ptr(row_of) ||
+      !ok_ptr(x_perm) || !ok_opt(counts))
+    return MOE_ERR_INVALID;
+  const Layout L = layout(T, BN2, BN1, E, k);
+  if (!ws || !aligned16(ws) || ws_bytes < L.routing_end) return MOE_ERR_WORKSPACE;
+  const int nsm = device_sms();
+  if (nsm <= 0) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Work w = work_from(ws, L, false, false);
+  if (counts) w.counts = counts;
+  w.offsets = offsets;
+  w.perm = perm;
+  w.row_of = row_of;
+  const int nblk = route_blocks(T);
+  MOE_TRY(launch_hist(topk_idx, T, E, k, w.blk_hist, st));
+  MOE_TRY(launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, default_cost_model(), st));
+  MOE_TRY(launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, st));
+  MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(x), perm, T * k, d, k,
+                        static_cast<__nv_bfloat16*>(x_perm), nsm, st));
+  return MOE_OK;
+}
+
+moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, int d, int f, int E,
+                           int k, const void* W1, const void* W3, const void* W2, void* h, void* y,
+                           void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = check_shape(T, d, f, E, k);
+  if (s != MOE_OK) return s;
+  if (!ok_ptr(x_perm) || !ok_ptr(offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
+      !ok_ptr(y) || !ok_opt(h))
+    return MOE_ERR_INVALID;
+  const Layout L = layout(T, d, f, E, k);
+  if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const int nsm = device_sms();
+  if (nsm <= 1) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Work w = work_from(ws, L, true, true);
+  MOE_TRY(launch_plan(w, 0, offsets, T, d, f, E, k, nsm, 1, 1, default_cost_model(), st));
+  FfnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.w = w;
+  a.x_perm = static_cast<const __nv_bfloat16*>(x_perm);
+  a.h = h ? static_cast<__nv_bfloat16*>(h) : w.h;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.W1 = W1; a.W3 = W3; a.W2 = W2;
+  a.R = T * k; a.T = T; a.d = d; a.f = f; a.E = E; a.k = k;
+  a.phase = PH_G1 | PH_G2;
+  a.join = 0;
+  a.mgb = 1;
+  a.timeout_ns = 2000000000ull;
+  MOE_TRY(launch_ffn(a, nsm, st));
+  return MOE_OK;
+}
+
+moe_status moe_combine(const void* y, const int32_t* row_of, const float* topk_gate, int T, int d,
+                       int k, void* out, void* stream) {
+  if (T < 1 || d < 1 || k < 1) return MOE_ERR_INVALID;
+  if (k > MAX_K || d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!ok_ptr(y) || !ok_ptr(row_of) || !ok_ptr(topk_gate) || !ok_ptr(out)) return MOE_ERR_INVALID;
+  const int nsm = device_sms();
+  if (nsm <= 0) return MOE_ERR_CUDA;
+  return cuda_status(launch_combine(static_cast<const __nv_bfloat16*>(y), row_of, topk_gate, T, d, k,
+                                    static_cast<__nv_bfloat16*>(out), nsm,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (!args) return MOE_ERR_INVALID;
+  const moe_layer_args& A = *args;
+  moe_status s = check_shape(A.T, A.d, A.f, A.E, A.k);
+  if (s != MOE_OK) return s;
+  if (mode != MOE_MODE_SEQUENTIAL && mode != MOE_MODE_OVERLAPPED) return MOE_ERR_INVALID;
+  if (!ok_ptr(A.x) || !ok_ptr(A.logits) || !ok_ptr(A.W1) || !ok_ptr(A.W3) || !ok_ptr(A.W2) ||
+      !ok_ptr(A.out) || !ok_opt(A.topk_idx) || !ok_opt(A.topk_gate) || !ok_opt(A.counts) ||
+      !ok_opt(A.offsets) || !ok_opt(A.perm))
+    return MOE_ERR_INVALID;
+  if (A.consumer_sms < 0 || A.mgb < 0 || A.timeout_us < 0) return MOE_ERR_INVALID;
+  const Layout L = layout(A.T, A.d, A.f, A.E, A.k);
+  if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const int nsm = device_sms();
+  if (nsm <= 1) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Work w = work_from(ws, L, true, true);
+  if (A.topk_idx) w.topk_idx = A.topk_idx;
+  if (A.topk_gate) w.topk_gate = A.topk_gate;
+  if (A.counts) w.counts = A.counts;
+  if (A.offsets) w.offsets = A.offsets;
+  if (A.perm) w.perm = A.perm;
+  const int T = A.T, d = A.d, f = A.f, E = A.E, k = A.k, R = T * k;
+  const int mgb = A.mgb > 0 ? A.mgb : 1;
+  const int nblk = route_blocks(T);
+  MOE_TRY(launch_route(A.logits, T, E, k, w.topk_idx, w.topk_gate, w.blk_hist, w.arrive, st));
+  MOE_TRY(launch_plan(w, nblk, nullptr, T, d, f, E, k, nsm, A.consumer_sms, mgb, default_cost_model(), st));
+  MOE_TRY(launch_scatter(w.topk_idx, T, E, k, w.blk_base, w.perm, w.row_of, st));
+  MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(A.x), w.perm, R, d, k, w.x_perm, nsm, st));
+  FfnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.w = w;
+  a.x_perm = w.x_perm;
+  a.h = w.h;
+  a.y = w.y;
+  a.W1 = A.W1; a.W3 = A.W3; a.W2 = A.W2;
+  a.gate = w.topk_gate;
+  a.out = static_cast<__nv_bfloat16*>(A.out);
+  a.R = R; a.T = T; a.d = d; a.f = f; a.E = E; a.k = k;
+  a.mgb = mgb;
+  a.flags = A.flags;
+  a.timeout_ns = (A.timeout_us > 0 ? (uint64_t)A.timeout_us : 2000000ull) * 1000ull;
+  if (mode == MOE_MODE_OVERLAPPED) {
+    a.phase = PH_G1 | PH_G2 | PH_CONS;
+    a.join = (A.flags & MOE_SCHED_NO_JOIN) ? 0 : 1;
+    MOE_TRY(launch_ffn(a, nsm, st));
+  } else {
+    a.phase = PH_G1;
+    MOE_TRY(launch_ffn(a, nsm, st));
+    a.phase = PH_G2;
+    MOE_TRY(launch_ffn(a, nsm, st));
+    MOE_TRY(launch_combine(w.y, w.row_of, w.topk_gate, T, d, k, a.out, nsm, st));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_get_status(void* ws, void* stream, int* consumer_sms, int* n_bands) {
+  if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  Status h;
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (consumer_sms) *consumer_sms = h.consumer_sms;
+  if (n_bands) *n_bands = h.n_bands;
+  if (h.code == ST_TIMEOUT) return MOE_ERR_TIMEOUT;
+  return h.code == ST_OK ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// kernels.h -- internal launch functions of libmoe_b200.so (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include "common.cuh"
+
+namespace moe {
+
+// route.cu
+cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx,
+                         float* topk_gate, int32_t* blk_hist, uint32_t* arrive_or_null,
+                         cudaStream_t s);
+cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int32_t* blk_hist,
+                        cudaStream_t s);
+cudaError_t launch_colsum(const int32_t* blk_hist, int nblk, int E, int32_t* counts,
+                          cudaStream_t s);
+// Plan: counts/offsets (from blk_hist when nblk > 0, else from `offsets_in`),
+// per-block scatter bases, expert priority order, band table, tile counts,
+// zeroed sync counters and the producer/consumer split.
+cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
+                        int E, int k, int num_sms, int consumer_hint, int mgb,
+                        const CostModel& cm, cudaStream_t s);
+cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const int32_t* blk_base,
+                           int32_t* perm, int32_t* row_of, cudaStream_t s);
+cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, int R, int d, int k,
+                          __nv_bfloat16* x_perm, int num_sms, cudaStream_t s);
+
+// combine.cu
+cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* row_of, const float* gate,
+                           int T, int d, int k, __nv_bfloat16* out, int num_sms, cudaStream_t s);
+
+// ffn.cu
+enum : int { PH_G1 = 1, PH_G2 = 2, PH_CONS = 4 };
+
+struct FfnArgs {
+  Work w;
+  const __nv_bfloat16* x_perm;   // A operand of GEMM1
+  __nv_bfloat16* h;              // GEMM1 output / GEMM2 A operand
+  __nv_bfloat16* y;              // GEMM2 output
+  const void* W1; const void* W3; const void* W2;
+  const float* gate;             // [T][k] (consumer role)
+  __nv_bfloat16* out;            // [T][d] (consumer role)
+  int R, T, d, f, E, k;
+  int phase;                     // PH_* bits
+  int join;                      // producers join the combine when the tile queue drains
+  int mgb;
+  uint32_t flags;
+  uint64_t timeout_ns;
+};
+
+size_t ffn_smem_bytes();
+cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,334 @@
+// route.cu -- steps (a) routing and (b) expert-contiguous permutation, plus the
+// per-call plan (band table, tile counts, producer/consumer split).
+//
+// Routing follows "Fine-grained Computation-Communication Overlap via
+// Tile-level Signaling and Scheduling for Mixture-of-Experts", Section 2.1
+// (top-k experts per token, gate weights); the permutation is that paper's
+// Section 3.2.1 row layout on one GPU (rows grouped by expert, no pad rows), and
+// the tile order is its Section 3.2.2 schedule rule (ii): experts with more rows
+// first, each expert's tiles contiguous.  The split follows "Weave" (arXiv
+// 2609.21483), Abstract: once routing is known, a cost model sizes the
+// communication (here: combine) and computation worker groups.
+#include "kernels.h"
+
+#include <float.h>
+
+namespace moe {
+
+// ------------------------------------------------------------------ route ---
+// One warp per token.  Lane l holds logits of experts l, l+32, ... (E <= 256).
+// k rounds of a warp arg-max under the order (logit desc, id asc).  Lane 0 then
+// forms the gates in double (exp of l_j - l_0, summed in slot order) and adds the
+// token's experts to the block's histogram (blk_hist[b][e], no global atomics:
+// the plan kernel scans the per-block counts, so ranks come out deterministic).
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E,
+                                                    int k, int32_t* __restrict__ topk_idx,
+                                                    float* __restrict__ topk_gate,
+                                                    int32_t* __restrict__ blk_hist,
+                                                    uint32_t* __restrict__ arrive) {
+  __shared__ int hist[MAX_E];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * ROUTE_TOK;
+  const int t1 = min(T, t0 + ROUTE_TOK);
+  const int nv = (E + 31) >> 5;
+  for (int t = t0 + warp; t < t1; t += 8) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = (i < nv && e < E) ? __ldg(logits + (size_t)t * E + e) : -FLT_MAX;
+    }
+    uint32_t used = 0;
+    for (int i = 0; i < 8; ++i)
+      if (!(i < nv && lane + 32 * i < E)) used |= 1u << i;
+    int sel_e[MAX_K];
+    float sel_v[MAX_K];
+    for (int j = 0; j < k; ++j) {
+      float bv = -FLT_MAX;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (!(used & (1u << i)) && (v[i] > bv || (v[i] == bv && e < be))) { bv = v[i]; be = e; }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+      }
+      if ((be & 31) == lane) used |= 1u << (be >> 5);
+      sel_e[j] = be;
+      sel_v[j] = bv;
+    }
+    if (lane == 0) {
+      double w[MAX_K];
+      double s = 0.0;
+      const double m = (double)sel_v[0];
+      for (int j = 0; j < k; ++j) {
+        w[j] = exp((double)sel_v[j] - m);
+        s += w[j];
+      }
+      for (int j = 0; j < k; ++j) {
+        topk_idx[(size_t)t * k + j] = sel_e[j];
+        topk_gate[(size_t)t * k + j] = (float)(w[j] / s);
+        atomicAdd(&hist[sel_e[j]], 1);
+      }
+      if (arrive) arrive[t] = 0u;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) blk_hist[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx,
+                         float* topk_gate, int32_t* blk_hist, uint32_t* arrive, cudaStream_t s) {
+  route_kernel<<<route_blocks(T), 256, 0, s>>>(logits, T, E, k, topk_idx, topk_gate, blk_hist, arrive);
+  return cudaGetLastError();
+}
+
+__global__ void colsum_kernel(const int32_t* __restrict__ blk_hist, int nblk, int E,
+                              int32_t* __restrict__ counts) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  int s = 0;
+  for (int b = 0; b < nblk; ++b) s += blk_hist[(size_t)b * E + e];
+  counts[e] = s;
+}
+
+cudaError_t launch_colsum(const int32_t* blk_hist, int nblk, int E, int32_t* counts, cudaStream_t s) {
+  colsum_kernel<<<cdiv(E, 256), 256, 0, s>>>(blk_hist, nblk, E, counts);
+  return cudaGetLastError();
+}
+
+// Per-block expert histogram of given top-k ids (moe_permute's entry, where the
+// routing came from the caller rather than route_kernel).
+__global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ topk_idx, int T,
+                                                   int E, int k, int32_t* __restrict__ blk_hist) {
+  __shared__ int hist[MAX_E];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const long p0 = (long)blockIdx.x * ROUTE_TOK * k;
+  const long p1 = (long)min(T, (int)(blockIdx.x + 1) * ROUTE_TOK) * k;
+  for (long p = p0 + threadIdx.x; p < p1; p += blockDim.x) atomicAdd(&hist[topk_idx[p]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) blk_hist[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int32_t* blk_hist,
+                        cudaStream_t s) {
+  hist_kernel<<<route_blocks(T), 256, 0, s>>>(topk_idx, T, E, k, blk_hist);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------- plan ---
+// Producer/consumer split (the Weave-style spatial scheduler): choose the
+// consumer SM count C minimising
+//   max( F2 / ((S - C) * phi),  Bc / min(C * beta, beta_hbm) ) + tail(C)
+// where F2 = GEMM2 FLOPs (the part the combine overlaps), Bc = combine bytes
+// (read every y row, write every output row), tail = one row band's combine on
+// C SMs after the last tile.  Deterministic: the same counts give the same C.
+__device__ int choose_consumers(int S, long long R, int T, int d, int f, const CostModel& cm) {
+  const double F2 = 2.0 * (double)R * f * d;
+  const double Bc = 2.0 * (double)R * d + 2.0 * (double)T * d;
+  const double band_bytes = 2.0 * BM * d * 2.0;
+  int best = 1;
+  double best_t = 1e300;
+  const int cmax = min(cm.max_consumers, S - 1);
+  for (int C = 1; C <= cmax; ++C) {
+    const double tp = F2 / ((double)(S - C) * cm.mma_flops_per_sm);
+    const double bw = fmin((double)C * cm.copy_bytes_per_sm, (double)cm.hbm_bytes);
+    const double tc = Bc / bw;
+    const double t = fmax(tp, tc) + band_bytes / ((double)C * cm.copy_bytes_per_sm);
+    if (t < best_t) { best_t = t; best = C; }
+  }
+  return best;
+}
+
+__host__ __device__ inline int n_items_for(int nb, int mgb) {
+  if (mgb <= 1 || nb <= 2) return nb;
+  return 2 + cdiv(nb - 2, mgb);
+}
+
+__global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int32_t* offsets_in,
+                                                    int T, int d, int f, int E, int k, int num_sms,
+                                                    int consumer_hint, int mgb, CostModel cm) {
+  __shared__ int cnt[MAX_E];
+  __shared__ int offs[MAX_E + 1];
+  __shared__ int sorted[MAX_E];
+  __shared__ int bstart[MAX_E + 1];
+  __shared__ int nbands_s;
+  const int tid = threadIdx.x;
+  // counts and per-block bases (exclusive scan down each expert's column)
+  if (nblk > 0) {
+    for (int e = tid; e < E; e += blockDim.x) {
+      int run = 0;
+      for (int b = 0; b < nblk; ++b) {
+        const int hcount = w.blk_hist[(size_t)b * E + e];
+        w.blk_base[(size_t)b * E + e] = run;
+        run += hcount;
+      }
+      cnt[e] = run;
+    }
+  } else {
+    for (int e = tid; e < E; e += blockDim.x) cnt[e] = offsets_in[e + 1] - offsets_in[e];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) { offs[e] = run; run += cnt[e]; }
+    offs[E] = run;
+  }
+  __syncthreads();
+  for (int e = tid; e <= E; e += blockDim.x) {
+    if (e < E) w.counts[e] = cnt[e];
+    w.offsets[e] = offs[e];
+  }
+  if (nblk > 0) {
+    for (int i = tid; i < nblk * E; i += blockDim.x) w.blk_base[i] += offs[i % E];
+  }
+  // expert priority: rows descending, id ascending (rank by comparison count)
+  for (int e = tid; e < E; e += blockDim.x) {
+    int r = 0;
+    for (int o = 0; o < E; ++o) r += (cnt[o] > cnt[e]) || (cnt[o] == cnt[e] && o < e);
+    sorted[r] = e;
+  }
+  __syncthreads();
+  const int NT1 = f / BN1, NT2 = d / BN2;
+  if (tid == 0) {
+    int nb = 0, nt1 = 0;
+    for (int s = 0; s < E; ++s) {
+      const int e = sorted[s];
+      bstart[s] = nb;
+      if (w.bands) {
+        w.band_start[s] = nb;
+        w.tile_start1[s] = nt1;
+      }
+      const int bands = cdiv(cnt[e], BM);
+      nb += bands;
+      nt1 += bands * NT1;
+    }
+    bstart[E] = nb;
+    if (w.bands) {
+      w.band_start[E] = nb;
+      w.tile_start1[E] = nt1;
+    }
+    nbands_s = nb;
+    const long long R = offs[E];
+    const int C = consumer_hint > 0 ? min(consumer_hint, num_sms - 1)
+                                    : choose_consumers(num_sms, R, T, d, f, cm);
+    Status st;
+    st.code = ST_OK;
+    st.consumer_sms = C;
+    st.n_bands = nb;
+    st.n_tiles1 = nt1;
+    st.n_tiles2 = nb * NT2;
+    st.where = W_NONE;
+    st.n_items = n_items_for(nb, mgb);
+    st.pad = 0;
+    *w.status = st;
+    w.sync->q1 = 0; w.sync->q2 = 0; w.sync->qc = 0; w.sync->pad = 0;
+  }
+  if (w.bands == nullptr) return;   // permutation only: no tile plan wanted
+  for (int s = tid; s < E; s += blockDim.x) w.sorted_e[s] = sorted[s];
+  __syncthreads();
+  for (int s = tid; s < E; s += blockDim.x) {
+    const int e = sorted[s];
+    const int b0 = bstart[s], nbe = bstart[s + 1] - b0;
+    for (int i = 0; i < nbe; ++i) {
+      Band bd;
+      bd.expert = e;
+      bd.row0 = offs[e] + i * BM;
+      bd.rows = min(BM, cnt[e] - i * BM);
+      bd.pad = 0;
+      w.bands[b0 + i] = bd;
+    }
+  }
+  for (int i = tid; i < nbands_s; i += blockDim.x) { w.band_done1[i] = 0u; w.band_done2[i] = 0u; }
+}
+
+cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
+                        int E, int k, int num_sms, int consumer_hint, int mgb, const CostModel& cm,
+                        cudaStream_t s) {
+  plan_kernel<<<1, 1024, 0, s>>>(w, nblk, offsets_in, T, d, f, E, k, num_sms, consumer_hint, mgb, cm);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- scatter ---
+// Block b owns the slots of route block b (tokens [b*128, b*128+128)) and walks
+// them in ascending order, 256 at a time.  Within a warp, __match_any_sync gives
+// each slot's rank among earlier lanes with the same expert; per-warp counts in
+// shared memory give the rank among earlier warps; a running count per expert
+// carries across chunks.  row = (expert's offset + earlier blocks' count, from
+// the plan) + rank inside the block -- a stable counting sort.
+__global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ topk_idx, int T,
+                                                      int E, int k, const int32_t* __restrict__ blk_base,
+                                                      int32_t* __restrict__ perm,
+                                                      int32_t* __restrict__ row_of) {
+  __shared__ int running[MAX_E];
+  __shared__ int wcnt[8][MAX_E];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < E; e += 256) running[e] = 0;
+  for (int i = threadIdx.x; i < 8 * MAX_E; i += 256) (&wcnt[0][0])[i] = 0;
+  __syncthreads();
+  const long p0 = (long)blockIdx.x * ROUTE_TOK * k;
+  const long p1 = (long)min(T, (int)(blockIdx.x + 1) * ROUTE_TOK) * k;
+  const int* base = blk_base + (size_t)blockIdx.x * E;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (long c = p0; c < p1; c += 256) {
+    const long p = c + threadIdx.x;
+    const bool valid = p < p1;
+    const int e = valid ? topk_idx[p] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank_w = __popc(peers & lt);
+    if (valid && rank_w == 0) wcnt[warp][e] = __popc(peers);
+    __syncthreads();
+    if (valid) {
+      int pre = running[e];
+      for (int w2 = 0; w2 < warp; ++w2) pre += wcnt[w2][e];
+      const int r = base[e] + pre + rank_w;
+      perm[r] = (int32_t)p;
+      row_of[p] = r;
+    }
+    __syncthreads();
+    for (int e2 = threadIdx.x; e2 < E; e2 += 256) {
+      int add = 0;
+      for (int w2 = 0; w2 < 8; ++w2) { add += wcnt[w2][e2]; wcnt[w2][e2] = 0; }
+      running[e2] += add;
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const int32_t* blk_base,
+                           int32_t* perm, int32_t* row_of, cudaStream_t s) {
+  scatter_kernel<<<route_blocks(T), 256, 0, s>>>(topk_idx, T, E, k, blk_base, perm, row_of);
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------- gather ---
+// x_perm[r] = x[perm[r] / k]: one warp per row, 16-byte vector loads and stores.
+__global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x,
+                                                     const int32_t* __restrict__ perm, int R,
+                                                     int dv, int k, uint4* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb) {
+    const size_t t = (size_t)(perm[r] / k);
+    const uint4* src = x + t * dv;
+    uint4* dst = x_perm + (size_t)r * dv;
+    for (int v = lane; v < dv; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, int R, int d, int k,
+                          __nv_bfloat16* x_perm, int num_sms, cudaStream_t s) {
+  const int grid = max(1, min(cdiv(R, 8), num_sms * 8));
+  gather_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(x), perm, R, d / 8, k,
+                                     reinterpret_cast<uint4*>(x_perm));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

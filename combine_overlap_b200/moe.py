@@ -1,0 +1,232 @@
+"""Thin ctypes binding over libmoe_b200.so (the C ABI in include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (PyTorch provides device memory and
+streams); calls are issued on the current torch stream.  If the library is not
+built this module raises at import -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run combine_overlap_b200.build.build() "
+                      "(nvcc, sm_100a) first")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+MOE_OK, MOE_ERR_INVALID, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_WORKSPACE = range(6)
+MODE_SEQUENTIAL, MODE_OVERLAPPED = 0, 1
+DBG_SKIP_FLAG_BAND = 0x1
+SCHED_NO_JOIN = 0x2
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} (code {code})")
+
+
+class LayerArgs(ctypes.Structure):
+    _fields_ = [
+        ("T", ctypes.c_int), ("d", ctypes.c_int), ("f", ctypes.c_int), ("E", ctypes.c_int),
+        ("k", ctypes.c_int),
+        ("x", ctypes.c_void_p), ("logits", ctypes.c_void_p),
+        ("W1", ctypes.c_void_p), ("W3", ctypes.c_void_p), ("W2", ctypes.c_void_p),
+        ("out", ctypes.c_void_p),
+        ("topk_idx", ctypes.c_void_p), ("topk_gate", ctypes.c_void_p),
+        ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p), ("perm", ctypes.c_void_p),
+        ("consumer_sms", ctypes.c_int), ("mgb", ctypes.c_int), ("flags", ctypes.c_uint),
+        ("timeout_us", ctypes.c_int),
+    ]
+
+
+_P, _I, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_lib.moe_workspace_size.argtypes = [_I, _I, _I, _I, _I]
+_lib.moe_workspace_size.restype = _S
+_lib.moe_route.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _S, _P]
+_lib.moe_permute.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _S, _P]
+_lib.moe_grouped_ffn.argtypes = [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P]
+_lib.moe_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
+_lib.moe_layer_forward.argtypes = [ctypes.POINTER(LayerArgs), _I, _P, _S, _P]
+_lib.moe_get_status.argtypes = [_P, _P, ctypes.POINTER(_I), ctypes.POINTER(_I)]
+_lib.moe_status_string.argtypes = [_I]
+_lib.moe_status_string.restype = ctypes.c_char_p
+_lib.moe_num_sms.restype = _I
+for _fn in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_layer_forward",
+            "moe_get_status"):
+    getattr(_lib, _fn).restype = _I
+
+
+def declared_symbols() -> list[str]:
+    """Function names declared in include/moe.h."""
+    with open(HEADER) as fh:
+        text = fh.read()
+    return sorted(set(re.findall(r"^\s*(?:[\w\*]+\s+)+\**(moe_\w+)\s*\(", text, re.M)))
+
+
+def status_string(code: int) -> str:
+    return _lib.moe_status_string(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code != MOE_OK:
+        raise MoEError(code, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(T: int, d: int, f: int, E: int, k: int) -> int:
+    return int(_lib.moe_workspace_size(T, d, f, E, k))
+
+
+def num_sms() -> int:
+    return int(_lib.moe_num_sms())
+
+
+def alloc_workspace(T, d, f, E, k, device="cuda") -> torch.Tensor:
+    n = workspace_size(T, d, f, E, k)
+    if n == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED, "moe_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def route(logits: torch.Tensor, k: int, ws: torch.Tensor, counts: bool = False):
+    _need(logits, torch.float32, "logits")
+    T, E = logits.shape
+    idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    gate = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    cnt = torch.empty(E, dtype=torch.int32, device=logits.device) if counts else None
+    _check(_lib.moe_route(_ptr(logits), T, E, k, _ptr(idx), _ptr(gate), _ptr(cnt), _ptr(ws),
+                          ws.numel(), _stream()), "moe_route")
+    return (idx, gate, cnt) if counts else (idx, gate)
+
+
+def permute(x: torch.Tensor, topk_idx: torch.Tensor, E: int, ws: torch.Tensor):
+    _need(x, torch.bfloat16, "x")
+    _need(topk_idx, torch.int32, "topk_idx")
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    dev = x.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    row_of = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty((T * k, d), dtype=torch.bfloat16, device=dev)
+    _check(_lib.moe_permute(_ptr(x), T, d, E, k, _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                            _ptr(perm), _ptr(row_of), _ptr(x_perm), _ptr(ws), ws.numel(),
+                            _stream()), "moe_permute")
+    return counts, offsets, perm, row_of, x_perm
+
+
+def grouped_ffn(x_perm: torch.Tensor, offsets: torch.Tensor, W1, W3, W2, T: int, k: int,
+                ws: torch.Tensor, want_h: bool = True):
+    """x_perm: [T*k][d] bf16 (rows past offsets[E] unused)."""
+    _need(x_perm, torch.bfloat16, "x_perm")
+    _need(offsets, torch.int32, "offsets")
+    for n, w in (("W1", W1), ("W3", W3), ("W2", W2)):
+        _need(w, torch.bfloat16, n)
+    E, d, f = W1.shape
+    dev = x_perm.device
+    y = torch.empty((T * k, d), dtype=torch.bfloat16, device=dev)
+    h = torch.empty((T * k, f), dtype=torch.bfloat16, device=dev) if want_h else None
+    _check(_lib.moe_grouped_ffn(_ptr(x_perm), _ptr(offsets), T, d, f, E, k, _ptr(W1), _ptr(W3),
+                                _ptr(W2), _ptr(h), _ptr(y), _ptr(ws), ws.numel(), _stream()),
+           "moe_grouped_ffn")
+    return h, y
+
+
+def combine(y: torch.Tensor, row_of: torch.Tensor, topk_gate: torch.Tensor, out=None):
+    _need(y, torch.bfloat16, "y")
+    _need(row_of, torch.int32, "row_of")
+    _need(topk_gate, torch.float32, "topk_gate")
+    T, k = topk_gate.shape
+    d = y.shape[1]
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=y.device)
+    _check(_lib.moe_combine(_ptr(y), _ptr(row_of), _ptr(topk_gate), T, d, k, _ptr(out), _stream()),
+           "moe_combine")
+    return out
+
+
+def make_args(x, logits, W1, W3, W2, k, out, topk_idx=None, topk_gate=None, counts=None,
+              offsets=None, perm=None, consumer_sms=0, mgb=1, flags=0, timeout_us=0) -> LayerArgs:
+    T, d = x.shape
+    E, _, f = W1.shape
+    return LayerArgs(T, d, f, E, k, x.data_ptr(), logits.data_ptr(), W1.data_ptr(), W3.data_ptr(),
+                     W2.data_ptr(), out.data_ptr(),
+                     *(0 if t is None else t.data_ptr() for t in (topk_idx, topk_gate, counts, offsets, perm)),
+                     consumer_sms, mgb, flags, timeout_us)
+
+
+def layer_forward(x, logits, W1, W3, W2, k, ws, mode=MODE_OVERLAPPED, out=None, outputs=False,
+                  consumer_sms=0, mgb=1, flags=0, timeout_us=0, stream=None):
+    """One MoE layer.  Returns out, or (out, dict of routing outputs) if outputs."""
+    _need(x, torch.bfloat16, "x")
+    _need(logits, torch.float32, "logits")
+    for n, w in (("W1", W1), ("W3", W3), ("W2", W2)):
+        _need(w, torch.bfloat16, n)
+    T, d = x.shape
+    E = logits.shape[1]
+    dev = x.device
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    extra = {}
+    if outputs:
+        extra = dict(topk_idx=torch.empty((T, k), dtype=torch.int32, device=dev),
+                     topk_gate=torch.empty((T, k), dtype=torch.float32, device=dev),
+                     counts=torch.empty(E, dtype=torch.int32, device=dev),
+                     offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                     perm=torch.empty(T * k, dtype=torch.int32, device=dev))
+    args = make_args(x, logits, W1, W3, W2, k, out, consumer_sms=consumer_sms, mgb=mgb,
+                     flags=flags, timeout_us=timeout_us, **extra)
+    _check(_lib.moe_layer_forward(ctypes.byref(args), int(mode), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "moe_layer_forward")
+    return (out, extra) if outputs else out
+
+
+def get_status(ws: torch.Tensor, stream=None):
+    """(status code, consumer SMs used, row bands) of the last call on ws; syncs."""
+    c = ctypes.c_int(0)
+    nb = ctypes.c_int(0)
+    code = _lib.moe_get_status(_ptr(ws), _stream(stream), ctypes.byref(c), ctypes.byref(nb))
+    return int(code), int(c.value), int(nb.value)
+
+
+class MoELayer:
+    """Holds the weights and a workspace; forward() runs the layer."""
+
+    def __init__(self, W1, W3, W2, k: int, max_tokens: int):
+        self.W1, self.W3, self.W2, self.k = W1, W3, W2, k
+        self.E, self.d, self.f = W1.shape
+        self.max_tokens = max_tokens
+        self.ws = alloc_workspace(max_tokens, self.d, self.f, self.E, k, W1.device)
+
+    def forward(self, x, logits, mode=MODE_OVERLAPPED, **kw):
+        if x.shape[0] > self.max_tokens:
+            raise ValueError("more tokens than the workspace was sized for")
+        return layer_forward(x, logits, self.W1, self.W3, self.W2, self.k, self.ws, mode, **kw)

@@ -1,0 +1,153 @@
+/*
+ * moe.h -- C ABI of libmoe_b200.so: one Mixture-of-Experts layer on a B200
+ * (sm_100a), with the gate-weighted combine overlapped with the expert GEMM at
+ * tile granularity.
+ *
+ * The method is the one of "Fine-grained Computation-Communication Overlap via
+ * Tile-level Signaling and Scheduling for Mixture-of-Experts" (arXiv 2607.19539)
+ * on a single GPU: a persistent rank-wide expert GEMM (the producer, Section
+ * 3.3.1) publishes a ready signal per output tile from its epilogue; a small
+ * partition of SMs (the consumer, Sections 3.3.2-3.3.3) performs the return step
+ * -- here the gate-weighted unpermute/combine back to token order, standing in
+ * for the return all-to-all -- as tiles become ready.  The producer/consumer SM
+ * split is chosen per call from the routing counts by a small cost model, as in
+ * "Weave: Fine-Grained Dynamic SM Scheduling in an MoE Megakernel for
+ * Compute-Communication Overlap" (arXiv 2609.21483), Abstract.
+ *
+ * Conventions for every entry point:
+ *  - Pointers are DEVICE pointers unless stated otherwise; the caller allocates
+ *    and owns every buffer, including the workspace.  The library allocates no
+ *    device memory.
+ *  - bf16 = bfloat16 bit patterns (2 bytes); matrices are dense row-major.
+ *    Every device pointer must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void*.  Calls are asynchronous on it
+ *    and never synchronise the host, except moe_get_status.
+ *  - Argument errors return at once, before any launch, with MOE_ERR_INVALID or
+ *    MOE_ERR_UNSUPPORTED; a launch failure returns MOE_ERR_CUDA.  Errors found on
+ *    the device (a bounded wait that ran out) are written to the status block in
+ *    the workspace and read back by moe_get_status.  Kernels never trap and
+ *    every wait inside them is bounded.
+ *  - Preconditions: 1 <= T; 1 <= k <= min(E, 8); E <= 256; d % 256 == 0;
+ *    f % 128 == 0; logits finite.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,      /* bad argument (null pointer, bad size, misaligned)    */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid MoE shape this build does not handle          */
+  MOE_ERR_CUDA = 3,         /* a CUDA call failed                                  */
+  MOE_ERR_TIMEOUT = 4,      /* a bounded device wait ran out (see moe_get_status)  */
+  MOE_ERR_WORKSPACE = 5     /* workspace missing or smaller than moe_workspace_size */
+} moe_status;
+
+typedef enum {
+  /* route -> permute -> GEMM1 (all SMs) -> GEMM2 (all SMs) -> combine, each a
+   * separate launch: the conventional non-overlapped path (paper Section 4.1.3,
+   * the baseline that runs expert compute and the return step one after the
+   * other). */
+  MOE_MODE_SEQUENTIAL = 0,
+  /* route -> permute -> one persistent launch in which producer CTAs run the
+   * GEMM tiles and consumer CTAs combine each row band as soon as its tiles are
+   * flagged ready (paper Sections 3.3.1-3.3.3). */
+  MOE_MODE_OVERLAPPED = 1
+} moe_mode;
+
+/* Debug flags (moe_layer_args.flags). */
+#define MOE_DBG_SKIP_FLAG_BAND 0x1u  /* the producer never flags the first row band of
+                                        GEMM2, so the consumer's bounded wait runs out:
+                                        exercises MOE_ERR_TIMEOUT without a GPU fault */
+#define MOE_SCHED_NO_JOIN      0x2u  /* producer CTAs do not join the combine after the
+                                        GEMM tile queue drains (dedicated consumers only) */
+
+typedef struct {
+  int T, d, f, E, k;        /* tokens, d_model, d_ff, experts, top-k                */
+  const void* x;            /* [T][d] bf16 tokens                                   */
+  const float* logits;      /* [T][E] fp32 gate logits                              */
+  const void* W1;           /* [E][d][f] bf16 gate projection                       */
+  const void* W3;           /* [E][d][f] bf16 up projection                         */
+  const void* W2;           /* [E][f][d] bf16 down projection                       */
+  void* out;                /* [T][d] bf16 layer output                             */
+  /* Optional outputs (NULL = kept only in the workspace): */
+  int32_t* topk_idx;        /* [T][k] selected experts, by logit desc then id asc   */
+  float* topk_gate;         /* [T][k] softmax over the selected logits              */
+  int32_t* counts;          /* [E] routed rows per expert                           */
+  int32_t* offsets;         /* [E+1] exclusive prefix sum of counts                 */
+  int32_t* perm;            /* [T*k] routed row r -> source slot p = t*k + j        */
+  int consumer_sms;         /* overlapped mode: 0 = cost model; > 0 = this many     */
+  int mgb;                  /* row bands per consumer item (paper's x), >= 1; 0 = 1 */
+  unsigned flags;           /* MOE_DBG_* / MOE_SCHED_* bits                         */
+  int timeout_us;           /* bound on each device wait; 0 = default (2 s)         */
+} moe_layer_args;
+
+/* Bytes of device workspace moe_layer_forward, moe_route, moe_permute and
+ * moe_grouped_ffn need for this shape (one buffer serves all of them).  0 on
+ * an invalid shape. */
+size_t moe_workspace_size(int T, int d, int f, int E, int k);
+
+/* Step (a), routing (paper Section 2.1, "Routing"): per token the k largest
+ * logits, ordered by logit descending then expert id ascending (ties to the
+ * lower id); gates g_j = softmax over the k selected logits.
+ * logits [T][E] fp32 -> topk_idx [T][k] int32, topk_gate [T][k] fp32.
+ * counts [E] int32 (optional, NULL to skip): routed rows per expert. */
+moe_status moe_route(const float* logits, int T, int E, int k,
+                     int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Step (b), permutation into expert-contiguous order (paper Section 3.2.1,
+ * remote-owner-aligned row layout, one owner per expert on one GPU, no pad
+ * rows): counts, offsets (exclusive scan), and a stable order -- the rows of
+ * expert e are its slots p = t*k + j in ascending p.
+ * perm [T*k]: row r -> slot p; row_of [T*k]: slot p -> row r;
+ * x_perm [T*k][d] bf16: x_perm[r] = x[perm[r] / k].
+ * counts [E] and offsets [E+1] are outputs (offsets required, counts optional). */
+moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t* topk_idx,
+                       int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* row_of,
+                       void* x_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* Steps (c1)+(c2) alone, the grouped SwiGLU expert FFN on permuted rows (paper
+ * Section 3.3.1, one persistent kernel covering all experts): for expert e and
+ * rows r in [offsets[e], offsets[e+1]):
+ *   h[r] = bf16(silu(x_perm[r] W1_e) * (x_perm[r] W3_e)),  y[r] = bf16(h[r] W2_e)
+ * (fp32 accumulation).  x_perm [R][d], y [R][d] bf16, R = offsets[E] <= T*k;
+ * h [R][f] bf16 is written to the caller's buffer if non-NULL, else kept in the
+ * workspace. */
+moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, int d, int f,
+                           int E, int k, const void* W1, const void* W3, const void* W2,
+                           void* h, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Step (d) alone, the weighted reduction (paper Section 2.1, "Weighted reduction
+ * (scale)"): out[t] = bf16( sum_{j<k} g[t][j] * y[row_of[t*k+j]] ), fp32 in slot
+ * order.  y [T*k][d] bf16, row_of [T*k], topk_gate [T][k] -> out [T][d] bf16. */
+moe_status moe_combine(const void* y, const int32_t* row_of, const float* topk_gate,
+                       int T, int d, int k, void* out, void* stream);
+
+/* The whole layer, steps (a)-(e).  Both modes give bit-identical outputs. */
+moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reads the status block the last call left in `ws`.
+ * Returns MOE_OK or the device-side error (MOE_ERR_TIMEOUT).  Host outputs may be
+ * NULL: consumer_sms = the consumer SM count used (cost model or hint),
+ * n_bands = row bands (tiles of 128 rows) over all experts. */
+moe_status moe_get_status(void* ws, void* stream, int* consumer_sms, int* n_bands);
+
+/* Static English description of a status code. */
+const char* moe_status_string(moe_status s);
+
+/* The number of SMs the persistent kernels use on the current device (a host
+ * query, cached per device). */
+int moe_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,74 @@
+"""The C-ABI library loads on a CPU-only host, exports every function that
+include/moe.h declares, and rejects bad arguments on the host before any CUDA
+call (no compute is launched here)."""
+import ctypes
+
+import pytest
+
+moe = pytest.importorskip("combine_overlap_b200.moe")
+
+
+def test_exports_every_declared_symbol():
+    names = moe.declared_symbols()
+    assert {"moe_route", "moe_permute", "moe_layer_forward", "moe_grouped_ffn", "moe_combine",
+            "moe_workspace_size", "moe_get_status", "moe_status_string", "moe_num_sms"} <= set(names)
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_workspace_size_rules():
+    ws = moe.workspace_size
+    assert ws(256, 512, 1024, 8, 2) > 0
+    assert ws(0, 512, 1024, 8, 2) == 0          # no tokens
+    assert ws(256, 512, 1024, 8, 9) == 0        # k > E
+    assert ws(256, 500, 1024, 8, 2) == 0        # d not a multiple of 256
+    assert ws(256, 512, 1000, 8, 2) == 0        # f not a multiple of 128
+    assert ws(256, 512, 1024, 300, 2) == 0      # E > 256
+    assert ws(256, 512, 1024, 16, 9) == 0       # k > 8
+    # grows with every dimension; the intermediates dominate
+    base = ws(256, 512, 1024, 8, 2)
+    for args in ((512, 512, 1024, 8, 2), (256, 1024, 1024, 8, 2), (256, 512, 2048, 8, 2),
+                 (256, 512, 1024, 8, 4)):
+        assert ws(*args) > base
+    R = 4096 * 2
+    assert ws(4096, 4096, 14336, 8, 2) >= R * 4096 * 2 * 2 + R * 14336 * 2
+
+
+def test_status_strings():
+    for c in range(6):
+        assert moe.status_string(c)
+    assert moe.status_string(4).startswith("a bounded device wait")
+
+
+def _call_forward(args, mode=1, ws=0x1000, ws_bytes=1 << 40):
+    return moe._lib.moe_layer_forward(ctypes.byref(args), mode, ctypes.c_void_p(ws), ws_bytes, None)
+
+
+def _args(**kw):
+    a = moe.LayerArgs(256, 512, 1024, 8, 2, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000,
+                      0, 0, 0, 0, 0, 0, 1, 0, 0)
+    for k_, v in kw.items():
+        setattr(a, k_, v)
+    return a
+
+
+def test_host_side_argument_errors():
+    # every one of these returns before the library touches the GPU
+    assert _call_forward(_args(k=9)) == moe.MOE_ERR_INVALID
+    assert _call_forward(_args(T=0)) == moe.MOE_ERR_INVALID
+    assert _call_forward(_args(d=320)) == moe.MOE_ERR_UNSUPPORTED
+    assert _call_forward(_args(x=0)) == moe.MOE_ERR_INVALID
+    assert _call_forward(_args(out=0x6008)) == moe.MOE_ERR_INVALID      # misaligned
+    assert _call_forward(_args(consumer_sms=-1)) == moe.MOE_ERR_INVALID
+    assert _call_forward(_args(), mode=7) == moe.MOE_ERR_INVALID
+    assert _call_forward(_args(), ws=0) == moe.MOE_ERR_WORKSPACE
+    assert _call_forward(_args(), ws_bytes=1024) == moe.MOE_ERR_WORKSPACE
+    assert moe._lib.moe_layer_forward(None, 1, None, 0, None) == moe.MOE_ERR_INVALID
+    P = ctypes.c_void_p
+    assert moe._lib.moe_route(P(0x1000), 16, 8, 0, P(0x2000), P(0x3000), None, P(0x4000), 1 << 30,
+                              None) == moe.MOE_ERR_INVALID
+    assert moe._lib.moe_route(P(0x1000), 16, 8, 2, P(0x2000), P(0x3000), None, None, 1 << 30,
+                              None) == moe.MOE_ERR_WORKSPACE
+    assert moe._lib.moe_combine(P(0x1000), P(0x2000), P(0x3000), 16, 512, 9, P(0x4000),
+                                None) == moe.MOE_ERR_UNSUPPORTED

@@ -1,0 +1,101 @@
+"""The whole layer, steps (a)-(e), on the GPU.
+
+* Small layers, every element: GPU vs the oracle within 2e-2 * max|ref|; routing
+  outputs bit-exact; the overlapped mode bit-identical to the sequential mode
+  for every consumer-SM count tried (cost model, 1, 2, 4, 8, 32), segment size
+  mgb in {1, 2, 3} and with or without producers joining the combine.
+* Every benchmark workload at full size, in the configuration the benchmark
+  times: routing outputs in full, and a seeded sample of tokens through the
+  oracle's token-by-token definition path; overlapped == sequential in full."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from combine_overlap_b200 import synth
+import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+moe = pytest.importorskip("combine_overlap_b200.moe")
+
+SMALL = [
+    synth.WORKLOADS["tiny"],
+    synth.small("ragged_T", 333, 256, 256, 5, 2, "zipf"),
+    synth.small("k3_multi_band", 600, 512, 384, 4, 3),
+    synth.small("hot_expert", 500, 256, 128, 16, 4, "hot"),
+    synth.small("one_token", 1, 256, 128, 8, 2),
+]
+
+
+def _forward(inp, wl, ws, mode, **kw):
+    out, extra = moe.layer_forward(inp["x"], inp["logits"], inp["W1"], inp["W3"], inp["W2"], wl.k,
+                                   ws, mode, outputs=True, **kw)
+    code, c, nb = moe.get_status(ws)
+    assert code == moe.MOE_OK, moe.status_string(code)
+    return out, extra, c
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_layer_small(orc, wl):
+    inp = gu.inputs(wl)
+    ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
+    ref = orc.forward(gu.host(inp["x"]), gu.host(inp["logits"]), gu.host(inp["W1"]),
+                      gu.host(inp["W3"]), gu.host(inp["W2"]), wl.k)
+    seq, extra, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL)
+    assert np.array_equal(gu.host(extra["topk_idx"]), ref["topk_idx"])
+    gu.assert_gates(gu.host(extra["topk_gate"]), ref["topk_gate"])
+    assert np.array_equal(gu.host(extra["counts"]), ref["counts"])
+    assert np.array_equal(gu.host(extra["offsets"]), ref["offsets"])
+    assert np.array_equal(gu.host(extra["perm"]), ref["perm"])
+    gu.assert_close(gu.host(seq), ref["out"], what=f"sequential ({wl.name})")
+    seq_bits = gu.host(seq)
+    for kw in (dict(), dict(consumer_sms=1), dict(consumer_sms=2), dict(consumer_sms=4),
+               dict(consumer_sms=8), dict(consumer_sms=32), dict(mgb=2), dict(mgb=3, consumer_sms=3),
+               dict(flags=moe.SCHED_NO_JOIN, consumer_sms=2)):
+        ovl, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, **kw)
+        assert c >= 1
+        assert np.array_equal(gu.host(ovl), seq_bits), f"overlapped {kw} differs from sequential"
+
+
+def test_layer_repeat_bitwise():
+    wl = synth.small("repeat", 700, 512, 256, 8, 2, "zipf")
+    inp = gu.inputs(wl)
+    ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
+    first = moe.layer_forward(inp["x"], inp["logits"], inp["W1"], inp["W3"], inp["W2"], wl.k, ws)
+    first = first.clone()
+    for _ in range(20):
+        again = moe.layer_forward(inp["x"], inp["logits"], inp["W1"], inp["W3"], inp["W2"], wl.k, ws)
+        assert torch.equal(again, first)
+
+
+FULL = ["mixtral", "fine_grained", "imbalanced", "sweep_T512_hot", "sweep_T2048_uniform",
+        "sweep_T8192_zipf", "sweep_T32768_uniform"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_layer_full_size_sampled(orc, name):
+    wl = synth.WORKLOADS[name]
+    orc.set_threads(os.cpu_count() or 1)
+    inp = gu.inputs(wl)
+    ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
+    ovl, extra, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED)
+    ovl_bits = gu.host(ovl)
+    seq, _, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL)
+    assert np.array_equal(gu.host(seq), ovl_bits), "overlapped differs from sequential"
+    # routing in full
+    oidx, ogate = orc.route(gu.host(inp["logits"]), wl.k)
+    assert np.array_equal(gu.host(extra["topk_idx"]), oidx)
+    gu.assert_gates(gu.host(extra["topk_gate"]), ogate)
+    oc, oo, op, _ = orc.permute(oidx, wl.E)
+    assert np.array_equal(gu.host(extra["counts"]), oc)
+    assert np.array_equal(gu.host(extra["offsets"]), oo)
+    assert np.array_equal(gu.host(extra["perm"]), op)
+    # sampled tokens through the definition path (always including the first and last)
+    n = 48 if wl.d * wl.f * wl.k > 4096 * 4096 * 4 else 96
+    rng = np.random.default_rng(wl.seed)
+    toks = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(wl.T, size=n, replace=False)])).astype(np.int32)
+    ref = orc.tokens(gu.host(inp["x"]), oidx, ogate, gu.host(inp["W1"]), gu.host(inp["W3"]),
+                     gu.host(inp["W2"]), toks)
+    gu.assert_close(ovl_bits[toks], ref, what=f"{name} sampled tokens")
