@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""MoE-layer throughput on B200: tokens/s and TFLOP/s against the roofline,
+overlapped vs sequential.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole layer (route, permute, grouped SwiGLU FFN,
+combine) over one batch of synthetic tokens through moe_layer_forward.  The
+default workload is the Mixtral-8x7B-shaped layer (T=4096, d=4096, E=8, top-2,
+d_ff=14336).  Under torchrun with N > 1 every rank runs an independent replica
+on its own GPU and token shard (the layer has no cross-token exchange), and the
+job value is N*T tokens over the slowest rank's time (weak scaling).
+
+--impl reference times the CPU oracle (plain C++) on the host cores, a bounded
+token sample per step; it is a deliberately slow baseline, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from combine_overlap_b200 import synth  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the persistent FFN kernel, keyed by workload, valid only for the kernel sources
+# whose hash is recorded with it (see profiles/).
+TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha1()
+    for rel in ("combine_overlap_b200/csrc/ffn.cu", "combine_overlap_b200/csrc/common.cuh",
+                "combine_overlap_b200/csrc/combine.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixtral", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--consumer-sms", type=int, default=0, help="0 = cost model")
+    ap.add_argument("--mgb", type=int, default=1)
+    ap.add_argument("--no-join", action="store_true", help="producers do not join the combine")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- clocks ---
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int, enabled: bool = True):
+        self.proc = None
+        self.path = None
+        if not enabled:
+            return
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", sel], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, RuntimeError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------ distributed ---
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}: launch N>1 under torchrun")
+    return world, rank, local
+
+
+def flops_and_bytes(wl: synth.Workload, counts):
+    """Algorithmic FLOPs (6 R d f, no masked rows) and minimum HBM bytes (active
+    experts' weights + x + logits + out + routing indices) of one layer."""
+    F = 6 * wl.R * wl.d * wl.f
+    active = sum(1 for c in counts if c > 0)
+    B = active * 3 * wl.d * wl.f * 2 + wl.T * wl.d * 2 * 2 + wl.T * wl.E * 4 + 16 * wl.R
+    return F, B
+
+
+# --------------------------------------------------------------- our arm ---
+def run_ours(args):
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    from combine_overlap_b200 import moe
+
+    wl = synth.WORKLOADS[args.workload]
+    # each rank its own token shard; the same expert weights on every rank
+    shard = wl if rank == 0 else synth.Workload(wl.name, wl.T, wl.d, wl.f, wl.E, wl.k, wl.router,
+                                                 wl.seed + 1000 * rank)
+    x = synth.make_x(shard, dev)
+    logits = synth.make_logits(shard, dev)
+    W1, W3, W2 = synth.make_weights(wl, dev)
+    ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k, dev)
+    out = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device=dev)
+    kw = dict(consumer_sms=args.consumer_sms, mgb=args.mgb,
+              flags=moe.SCHED_NO_JOIN if args.no_join else 0)
+
+    def step(mode, evb=None, eve=None):
+        moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, mode, out=out, ev_begin=evb, ev_end=eve, **kw)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step(moe.MODE_OVERLAPPED)
+        step(moe.MODE_SEQUENTIAL)
+    torch.cuda.synchronize()
+    code, consumer_sms, n_bands = moe.get_status(ws)
+    if code != moe.MOE_OK:
+        raise RuntimeError(f"warm-up: {moe.status_string(code)}")
+    counts = moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, moe.MODE_OVERLAPPED, outputs=True,
+                               **kw)[1]["counts"].cpu().tolist()
+
+    def timed(mode, clocks=False):
+        K = args.steps
+        evb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        eve = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        clk = Clocks(local, clocks and not args.no_clocks) if clocks else None
+        e0.record(stream)
+        for i in range(K):
+            step(mode, evb[i], eve[i])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        c = clk.stop() if clk else None
+        total = e0.elapsed_time(e1) / K
+        ffn = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / K
+        return total, ffn, c
+
+    t_ovl, ffn_ovl, clocks = timed(moe.MODE_OVERLAPPED, clocks=True)
+    t_seq, ffn_seq, _ = timed(moe.MODE_SEQUENTIAL)
+
+    # end to end through the public call: H2D of the step's inputs from pinned
+    # host memory, the layer, D2H of its output, every step
+    x_h = x.cpu().pin_memory()
+    l_h = logits.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    x_d, l_d = torch.empty_like(x), torch.empty_like(logits)
+    for _ in range(max(1, args.warmup)):
+        x_d.copy_(x_h, non_blocking=True)
+        l_d.copy_(l_h, non_blocking=True)
+        moe.layer_forward(x_d, l_d, W1, W3, W2, wl.k, ws, moe.MODE_OVERLAPPED, out=out, **kw)
+        out_h.copy_(out, non_blocking=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_d.copy_(x_h, non_blocking=True)
+        l_d.copy_(l_h, non_blocking=True)
+        moe.layer_forward(x_d, l_d, W1, W3, W2, wl.k, ws, moe.MODE_OVERLAPPED, out=out, **kw)
+        out_h.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_e2e = e0.elapsed_time(e1) / args.steps
+    code, _, _ = moe.get_status(ws)
+    if code != moe.MOE_OK:
+        raise RuntimeError(f"timed runs: {moe.status_string(code)}")
+
+    times = torch.tensor([t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e = times.tolist()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, x, logits, W1, W3, W2, args.cpu_seconds)
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        F, B = flops_and_bytes(wl, counts)
+        peak_tf = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+        hbm = peaks["hbm_gbs"]
+        t_roof_ms = max(F / (peak_tf * 1e12), B / (hbm * 1e9)) * 1e3
+        ach = F / (ffn_ovl * 1e-3) / 1e12
+        h = kernel_source_hash()
+        tr = TRAFFIC.get(wl.name)
+        traffic = tr["bytes"] if tr and tr.get("kernel_hash") == h else None
+        T_all = wl.T * world
+        res = {
+            "metric": "MoE-layer tokens/s",
+            "value": T_all / (t_ovl * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": t_ovl,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic: seeded counter-based N(0,1) tokens and gate logits, random-init N(0,0.02) bf16 expert weights",
+            "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "d_ff": wl.f, "E": wl.E,
+                       "top_k": wl.k, "router": wl.router, "mode": "overlapped",
+                       "parallelism": f"replicas x{world} (token shards, no collective)",
+                       "l2": "inputs larger than L2: active expert weights %.2f GB per step" % (B / 1e9)},
+            "tflops": world * F / (t_ovl * 1e-3) / 1e12,
+            "roofline_frac_layer": t_roof_ms / t_ovl,
+            "roofline_layer": {"bound": "tensor" if F / (peak_tf * 1e12) >= B / (hbm * 1e9) else "hbm",
+                               "time_ms": t_roof_ms, "flops": F, "min_bytes": B,
+                               "peak_tflops": peak_tf, "peak_hbm_gbs": hbm, "peaks": src},
+            "sequential": {"value": T_all / (t_seq * 1e-3), "ms_per_step": t_seq,
+                           "ffn_ms": ffn_seq, "tflops": world * F / (t_seq * 1e-3) / 1e12},
+            "speedup_vs_sequential": t_seq / t_ovl,
+            "consumer_sms": consumer_sms,
+            "n_bands": n_bands,
+            "masked_row_waste": (n_bands * 128 - wl.R) / (n_bands * 128),
+            "roofline": {"kernel": "ffn_kernel (persistent GEMM1+GEMM2+combine)", "bound": "tensor",
+                         "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
+                         "traffic": traffic, "launch_ms": ffn_ovl,
+                         "peak_kind": f"{src} sustained bf16 (cuBLAS 8192^3 under the power cap)"},
+            "e2e": {"value": T_all / (t_e2e * 1e-3), "unit": "tokens/s", "ms_per_step": t_e2e,
+                    "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
+                    "d2h_bytes_per_step": out.numel() * 2},
+            "gpu_launches": 5 * args.steps,
+            "clocks": clocks,
+            "kernel_hash": h,
+        }
+        if cpu is not None:
+            res["cpu_baseline"] = cpu
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+# ------------------------------------------------------------ CPU oracle ---
+def _oracle_tokens_per_s(o, xh, idx, gate, W, n, T, seed):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    toks = rng.choice(T, size=min(n, T), replace=False).astype(np.int32)
+    t0 = time.perf_counter()
+    o.tokens(xh, idx, gate, W[0], W[1], W[2], toks)
+    return len(toks), time.perf_counter() - t0
+
+
+def _host_inputs(wl, x, logits, W1, W3, W2):
+    import oracle
+    o = oracle.get()
+    threads = o.set_threads(os.cpu_count() or 1)
+    xh = synth.bf16_bits(x)
+    lh = logits.detach().cpu().numpy()
+    W = [synth.bf16_bits(w) for w in (W1, W3, W2)]
+    idx, gate = o.route(lh, wl.k)
+    return o, threads, xh, idx, gate, W
+
+
+def cpu_baseline(wl, x, logits, W1, W3, W2, seconds):
+    """The oracle, as it stands, on a bounded token sample of the same workload."""
+    o, threads, xh, idx, gate, W = _host_inputs(wl, x, logits, W1, W3, W2)
+    n0 = max(threads, 4)
+    n, dt = _oracle_tokens_per_s(o, xh, idx, gate, W, n0, wl.T, 1)
+    n = int(min(wl.T, max(n0, n * seconds / max(dt, 1e-6))))
+    n, dt = _oracle_tokens_per_s(o, xh, idx, gate, W, n, wl.T, 2)
+    return {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {wl.T} tokens (routing in full), token-by-token oracle path, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = synth.make_inputs(wl, dev)
+    o, threads, xh, idx, gate, W = _host_inputs(wl, inp["x"], inp["logits"], inp["W1"], inp["W3"], inp["W2"])
+    del inp
+    if dev == "cuda":
+        torch.cuda.empty_cache()
+    # size each step to ~3 s of oracle work
+    n, dt = _oracle_tokens_per_s(o, xh, idx, gate, W, max(threads, 4), wl.T, 0)
+    n = int(min(wl.T, max(threads, n * 3.0 / max(dt, 1e-6))))
+    for i in range(args.warmup):
+        _oracle_tokens_per_s(o, xh, idx, gate, W, max(threads, 4), wl.T, 100 + i)
+    tot_n, tot_t = 0, 0.0
+    for i in range(args.steps):
+        m, t = _oracle_tokens_per_s(o, xh, idx, gate, W, n, wl.T, 1000 + i)
+        tot_n += m
+        tot_t += t
+    v = tot_n / tot_t
+    sample = f"{n} of {wl.T} tokens per step, token-by-token oracle path, {threads} threads"
+    res = {
+        "impl": "reference",
+        "metric": "MoE-layer tokens/s", "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.T / v * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic: seeded counter-based inputs, random-init weights",
+        "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "d_ff": wl.f, "E": wl.E,
+                   "top_k": wl.k, "router": wl.router, "mode": "cpu oracle",
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    args = parse()
+    if args.steps < 1 or args.warmup < 0:
+        raise SystemExit("--steps must be >= 1 and --warmup >= 0")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

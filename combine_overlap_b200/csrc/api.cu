@@ -300,6 +300,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   a.mgb = mgb;
   a.flags = A.flags;
   a.timeout_ns = (A.timeout_us > 0 ? (uint64_t)A.timeout_us : 2000000ull) * 1000ull;
+  if (A.ev_ffn_begin) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_begin), st));
   if (mode == MOE_MODE_OVERLAPPED) {
     a.phase = PH_G1 | PH_G2 | PH_CONS;
     a.join = (A.flags & MOE_SCHED_NO_JOIN) ? 0 : 1;
@@ -311,6 +312,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
     MOE_TRY(launch_ffn(a, nsm, st));
     MOE_TRY(launch_combine(w.y, w.row_of, w.topk_gate, T, d, k, a.out, nsm, st));
   }
+  if (A.ev_ffn_end) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_end), st));
   return MOE_OK;
 }
 

@@ -46,6 +46,7 @@ class LayerArgs(ctypes.Structure):
         ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p), ("perm", ctypes.c_void_p),
         ("consumer_sms", ctypes.c_int), ("mgb", ctypes.c_int), ("flags", ctypes.c_uint),
         ("timeout_us", ctypes.c_int),
+        ("ev_ffn_begin", ctypes.c_void_p), ("ev_ffn_end", ctypes.c_void_p),
     ]
 
 
@@ -174,17 +175,21 @@ def combine(y: torch.Tensor, row_of: torch.Tensor, topk_gate: torch.Tensor, out=
 
 
 def make_args(x, logits, W1, W3, W2, k, out, topk_idx=None, topk_gate=None, counts=None,
-              offsets=None, perm=None, consumer_sms=0, mgb=1, flags=0, timeout_us=0) -> LayerArgs:
+              offsets=None, perm=None, consumer_sms=0, mgb=1, flags=0, timeout_us=0,
+              ev_begin=None, ev_end=None) -> LayerArgs:
     T, d = x.shape
     E, _, f = W1.shape
     return LayerArgs(T, d, f, E, k, x.data_ptr(), logits.data_ptr(), W1.data_ptr(), W3.data_ptr(),
                      W2.data_ptr(), out.data_ptr(),
                      *(0 if t is None else t.data_ptr() for t in (topk_idx, topk_gate, counts, offsets, perm)),
-                     consumer_sms, mgb, flags, timeout_us)
+                     consumer_sms, mgb, flags, timeout_us,
+                     None if ev_begin is None else ev_begin.cuda_event,
+                     None if ev_end is None else ev_end.cuda_event)
 
 
 def layer_forward(x, logits, W1, W3, W2, k, ws, mode=MODE_OVERLAPPED, out=None, outputs=False,
-                  consumer_sms=0, mgb=1, flags=0, timeout_us=0, stream=None):
+                  consumer_sms=0, mgb=1, flags=0, timeout_us=0, stream=None, ev_begin=None,
+                  ev_end=None):
     """One MoE layer.  Returns out, or (out, dict of routing outputs) if outputs."""
     _need(x, torch.bfloat16, "x")
     _need(logits, torch.float32, "logits")
@@ -202,8 +207,16 @@ def layer_forward(x, logits, W1, W3, W2, k, ws, mode=MODE_OVERLAPPED, out=None, 
                      counts=torch.empty(E, dtype=torch.int32, device=dev),
                      offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
                      perm=torch.empty(T * k, dtype=torch.int32, device=dev))
+    # torch creates an event lazily and only times events it has seen recorded:
+    # record them here first (this also creates them); the library records them
+    # again at the FFN boundaries, and the last record is the one timed.
+    s = stream if stream is not None else torch.cuda.current_stream()
+    for ev in (ev_begin, ev_end):
+        if ev is not None:
+            ev.record(s)
     args = make_args(x, logits, W1, W3, W2, k, out, consumer_sms=consumer_sms, mgb=mgb,
-                     flags=flags, timeout_us=timeout_us, **extra)
+                     flags=flags, timeout_us=timeout_us, ev_begin=ev_begin, ev_end=ev_end, **extra)
+
     _check(_lib.moe_layer_forward(ctypes.byref(args), int(mode), _ptr(ws), ws.numel(),
                                   _stream(stream)), "moe_layer_forward")
     return (out, extra) if outputs else out

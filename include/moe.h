@@ -86,6 +86,12 @@ typedef struct {
   int mgb;                  /* row bands per consumer item (paper's x), >= 1; 0 = 1 */
   unsigned flags;           /* MOE_DBG_* / MOE_SCHED_* bits                         */
   int timeout_us;           /* bound on each device wait; 0 = default (2 s)         */
+  /* Optional timing hooks (cudaEvent_t as void*, NULL = none): recorded on the
+   * stream just before the first and just after the last expert-FFN launch
+   * (overlapped: the one persistent kernel, which also runs the combine;
+   * sequential: GEMM1, GEMM2 and the combine kernel). */
+  void* ev_ffn_begin;
+  void* ev_ffn_end;
 } moe_layer_args;
 
 /* Bytes of device workspace moe_layer_forward, moe_route, moe_permute and

@@ -47,7 +47,7 @@ def _call_forward(args, mode=1, ws=0x1000, ws_bytes=1 << 40):
 
 def _args(**kw):
     a = moe.LayerArgs(256, 512, 1024, 8, 2, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000,
-                      0, 0, 0, 0, 0, 0, 1, 0, 0)
+                      0, 0, 0, 0, 0, 0, 1, 0, 0, None, None)
     for k_, v in kw.items():
         setattr(a, k_, v)
     return a
