@@ -62,6 +62,9 @@ _lib.moe_get_status.argtypes = [_P, _P, ctypes.POINTER(_I), ctypes.POINTER(_I)]
 _lib.moe_status_string.argtypes = [_I]
 _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_num_sms.restype = _I
+_lib.moe_permute_noalloc.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
+_lib.moe_permute_noalloc.restype = _I
+_lib.moe_permute_noalloc_scratch_bytes.restype = _S
 for _fn in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_layer_forward",
             "moe_get_status"):
     getattr(_lib, _fn).restype = _I
@@ -141,6 +144,25 @@ def permute(x: torch.Tensor, topk_idx: torch.Tensor, E: int, ws: torch.Tensor):
     _check(_lib.moe_permute(_ptr(x), T, d, E, k, _ptr(topk_idx), _ptr(counts), _ptr(offsets),
                             _ptr(perm), _ptr(row_of), _ptr(x_perm), _ptr(ws), ws.numel(),
                             _stream()), "moe_permute")
+    return counts, offsets, perm, row_of, x_perm
+
+
+def permute_noalloc(x: torch.Tensor, topk_idx: torch.Tensor, E: int):
+    """moe_permute without a workspace: the library's fixed scratch array is used
+    instead (for callers that cannot allocate device memory; T <= 65536)."""
+    _need(x, torch.bfloat16, "x")
+    _need(topk_idx, torch.int32, "topk_idx")
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    dev = x.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    row_of = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty((T * k, d), dtype=torch.bfloat16, device=dev)
+    _check(_lib.moe_permute_noalloc(_ptr(x), T, d, E, k, _ptr(topk_idx), _ptr(counts),
+                                    _ptr(offsets), _ptr(perm), _ptr(row_of), _ptr(x_perm),
+                                    _stream()), "moe_permute_noalloc")
     return counts, offsets, perm, row_of, x_perm
 
 

@@ -136,6 +136,30 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
 moe_status moe_combine(const void* y, const int32_t* row_of, const float* topk_gate,
                        int T, int d, int k, void* out, void* stream);
 
+/* moe_permute for callers that cannot allocate device memory.  The paper has no
+ * counterpart to this entry point; it exists for callers such as a runtime that
+ * has already handed all device memory to its own pool, a plug-in host that owns
+ * every allocation, or code that must not call cudaMalloc where it permutes.
+ * Same arguments, outputs and results as moe_permute, minus the workspace: the
+ * per-block histograms and scan bases live in one fixed array inside the library
+ * (moe_permute_noalloc_scratch_bytes() bytes, a little over 1 MiB), which every
+ * GPU that loads the library holds until the process exits.  This call allocates
+ * nothing and calls no allocating routine.
+ *  - Limits: T <= 65536 (MOE_ERR_UNSUPPORTED above that), E <= 256, k <= 8,
+ *    d % 8 == 0; counts may be NULL.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any stream
+ *    capture.
+ *  - Every call on a device shares the one array and leaves its contents behind;
+ *    nothing in it needs to start at zero.  Calls whose work overlaps on the GPU
+ *    (e.g. on two streams at once) race on the array: order them on one stream. */
+moe_status moe_permute_noalloc(const void* x, int T, int d, int E, int k,
+                               const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                               int32_t* perm, int32_t* row_of, void* x_perm, void* stream);
+
+/* Size in bytes of the fixed scratch array moe_permute_noalloc uses. */
+size_t moe_permute_noalloc_scratch_bytes(void);
+
 /* The whole layer, steps (a)-(e).  Both modes give bit-identical outputs. */
 moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode,
                              void* ws, size_t ws_bytes, void* stream);
