@@ -45,29 +45,39 @@ __device__ __forceinline__ void combine_token_warp(const __nv_bfloat16* __restri
   const int dv = d >> 3;
   const uint4* yv = reinterpret_cast<const uint4*>(y);
   uint4* ov = reinterpret_cast<uint4*>(out) + (size_t)t * dv;
-  for (int v = lane; v < dv; v += 32) {
-    uint4 in[MAX_K];
-#pragma unroll
-    for (int j = 0; j < MAX_K; ++j)
-      if (j < k) in[j] = __ldcg(yv + (size_t)rows[j] * dv + v);
-    float acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  // two 16-byte vectors per lane per pass: 2k loads in flight per lane
+  for (int v0 = lane; v0 < dv; v0 += 64) {
+    const bool two = v0 + 32 < dv;
+    uint4 in[2][MAX_K];
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) {
       if (j < k) {
-        float f[8];
-        bf16x8_to_f32(in[j], f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(g[j], f[i], acc[i]);
+        in[0][j] = __ldcg(yv + (size_t)rows[j] * dv + v0);
+        if (two) in[1][j] = __ldcg(yv + (size_t)rows[j] * dv + v0 + 32);
       }
     }
-    uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]);
-    o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]);
-    o.w = pack_bf16x2(acc[6], acc[7]);
-    ov[v] = o;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u == 1 && !two) break;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < MAX_K; ++j) {
+        if (j < k) {
+          float f[8];
+          bf16x8_to_f32(in[u][j], f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(g[j], f[i], acc[i]);
+        }
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      ov[v0 + 32 * u] = o;
+    }
   }
 }
 

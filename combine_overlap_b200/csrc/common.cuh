@@ -34,7 +34,8 @@ enum : uint32_t { ST_OK = 0, ST_TIMEOUT = 4 };
 // where a wait ran out (Status::where)
 enum : uint32_t {
   W_NONE = 0, W_SCHED_EMPTY = 1, W_SCHED_FULL = 2, W_STAGE_EMPTY = 3, W_STAGE_FULL = 4,
-  W_TMEM_EMPTY = 5, W_TMEM_FULL = 6, W_BAND1 = 7, W_BAND2 = 8, W_DRAIN = 9
+  W_TMEM_EMPTY = 5, W_TMEM_FULL = 6, W_BAND1 = 7, W_BAND2 = 8, W_DRAIN = 9,
+  W_CONS_EMPTY = 10, W_CONS_FULL = 11
 };
 
 struct Status {
@@ -182,6 +183,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];"
       :: "r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
+
+// Untiled bulk copy global -> shared (no multicast): `bytes` (multiple of 16),
+// both addresses 16-byte aligned; completes `bytes` of transaction on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {

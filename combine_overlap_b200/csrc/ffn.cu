@@ -45,6 +45,8 @@ namespace moe {
 
 enum : int { K_END = 0, K_G1 = 1, K_G2 = 2 };
 
+constexpr int CONS_SLOTS = 16;   // at most this many tokens in flight per consumer CTA
+
 struct Item {
   int kind, band, nt, expert, row0, rows, pad0, pad1;
 };
@@ -58,11 +60,14 @@ struct SmemCtl {
   uint64_t sempty[SCHED_DEPTH];
   uint64_t epi_done[2];   // per accumulator: the four epilogue warps stored the tile
   uint64_t mma_done;
+  uint64_t cfull[CONS_SLOTS];    // consumer ring: a token's k expert rows landed in the slot
+  uint64_t cempty[CONS_SLOTS];   // consumer ring: the slot's token is reduced and stored
   Item ring[SCHED_DEPTH];
   uint32_t tmem_base;
   int item;
   int ok;
-  int pad;
+  int cn;                        // tokens completed by the current band
+  int ctok[BM];                  // ... and which
 };
 
 size_t ffn_smem_bytes() { return 1024 + (size_t)NSTAGE * STAGE_BYTES + sizeof(SmemCtl); }
@@ -352,16 +357,34 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
 }
 
 // ----------------------------------------------------------------- consumer ---
-// All warps of the CTA take combine items (row bands in priority order) from a
-// shared atomic counter.  For every row of a ready band, the token's arrival
-// counter is bumped with acq_rel; the warp that brings it to k holds every
-// one of the token's rows (published by earlier arrivals) and writes out[t].
-__device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, int nb, int n_items,
+// All CTAs that consume take combine items (row bands in priority order) from a
+// shared atomic counter.  For a ready band:
+//   1. every thread takes one row of the band and bumps its token's arrival
+//      counter (acq_rel); the thread that brings it to k records the token, whose
+//      k expert rows are now all stored (published by the earlier arrivals);
+//   2. thread 0 streams each recorded token's k rows of y into a ring of shared-
+//      memory slots with cp.async.bulk (the GEMM staging buffers are idle by
+//      now), so up to CONS_SLOTS tokens' rows are in flight per SM;
+//   3. warps 1-5 reduce a slot in fp32, slot order, and store out[t] with 16-byte
+//      stores -- the same arithmetic as combine_token_warp, so both modes agree
+//      bit for bit.  Each slot has one owning warp (see below).
+// If one token's rows do not fit the staging area, the warps fall back to
+// combine_token_warp straight from global memory.
+__device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int nb, int n_items,
                               const volatile uint32_t* abort) {
   const Work& w = a.w;
   const int NT2 = a.d / BN2;
+  const int k = a.k, d = a.d, dv = d >> 3;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NWARPS = FFN_THREADS / 32;
+  constexpr int NCW = NWARPS - 1;                         // reducing warps
+  const uint32_t row_bytes = (uint32_t)d * 2u;
+  const uint32_t tok_bytes = row_bytes * (uint32_t)k;
+  int S = (int)((size_t)NSTAGE * STAGE_BYTES / tok_bytes);
+  if (S > CONS_SLOTS) S = CONS_SLOTS;
+  if (S > NCW) S -= S % NCW;   // slots split evenly over the reducing warps
+  uint32_t base = 0;                                      // tokens this CTA reduced so far
+  uint32_t pend = 0, pend_par = 0;                        // issuer: slots with a copy issued
   while (true) {
     if (threadIdx.x == 0) ctl->item = *abort ? -1 : (int)atomicAdd(&w.sync->qc, 1u);
     __syncthreads();
@@ -375,26 +398,89 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, int nb, int n_item
         const bool ready = wait_count(&w.band_done2[b], (uint32_t)NT2, a.timeout_ns, abort);
         if (!ready) set_error(w.status, W_BAND2);
         ctl->ok = ready ? 1 : 0;
+        ctl->cn = 0;
       }
       __syncthreads();
       if (!ctl->ok) { ok = false; break; }
       const Band bd = w.bands[b];
-      for (int r = warp; r < bd.rows; r += NWARPS) {
-        int t = 0;
-        uint32_t old = 0;
-        if (lane == 0) {
-          t = w.perm[bd.row0 + r] / a.k;
-          old = atom_acq_rel_add(&w.arrive[t], 1u);
-        }
-        t = __shfl_sync(0xffffffffu, t, 0);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        if (old == (uint32_t)(a.k - 1)) combine_token_warp(a.y, w.row_of, a.gate, t, a.d, a.k, a.out, lane);
+      for (int r = threadIdx.x; r < bd.rows; r += FFN_THREADS) {
+        const int t = w.perm[bd.row0 + r] / k;
+        if (atom_acq_rel_add(&w.arrive[t], 1u) == (uint32_t)(k - 1)) ctl->ctok[atomicAdd(&ctl->cn, 1)] = t;
       }
+      __syncthreads();
+      const int n = ctl->cn;
+      if (S < 1) {
+        for (int i = warp; i < n; i += NWARPS)
+          combine_token_warp(a.y, w.row_of, a.gate, ctl->ctok[i], d, k, a.out, lane);
+      } else if (warp == 0) {
+        if (lane == 0) {
+          fence_proxy_async_global();   // y rows were stored by other SMs' generic stores
+          for (int i = 0; i < n; ++i) {
+            const uint32_t g = base + (uint32_t)i;
+            const int s = (int)(g % (uint32_t)S);
+            const uint32_t ph = (g / (uint32_t)S) & 1u;
+            if (!wait_bar(&ctl->cempty[s], ph ^ 1u, a.timeout_ns, abort)) { set_error(w.status, W_CONS_EMPTY); break; }
+            const int t = ctl->ctok[i];
+            uint8_t* dst = smem + (size_t)s * tok_bytes;
+            mbar_arrive_expect_tx(&ctl->cfull[s], tok_bytes);
+            for (int j = 0; j < k; ++j) {
+              const int r = w.row_of[(size_t)t * k + j];
+              bulk_load(dst + (size_t)j * row_bytes, a.y + (size_t)r * d, row_bytes, &ctl->cfull[s]);
+            }
+            pend |= 1u << s;
+            pend_par = (pend_par & ~(1u << s)) | (ph << s);
+          }
+        }
+      } else {
+        // Slot s belongs to warp 1 + s % NCW alone, which takes that slot's tokens in
+        // order, so it never waits on a slot's phase before the previous phase has
+        // completed (an mbarrier parity wait cannot tell phases two apart).
+        const int cw = warp - 1;
+        for (int i = 0; i < n; ++i) {
+          const uint32_t g = base + (uint32_t)i;
+          const int s = (int)(g % (uint32_t)S);
+          if (s % NCW != cw) continue;
+          const uint32_t ph = (g / (uint32_t)S) & 1u;
+          if (!__all_sync(0xffffffffu, wait_bar(&ctl->cfull[s], ph, a.timeout_ns, abort))) {
+            if (lane == 0) set_error(w.status, W_CONS_FULL);
+            break;
+          }
+          const int t = ctl->ctok[i];
+          float gt[MAX_K];
+#pragma unroll
+          for (int j = 0; j < MAX_K; ++j) gt[j] = j < k ? a.gate[(size_t)t * k + j] : 0.0f;
+          const uint4* src = reinterpret_cast<const uint4*>(smem + (size_t)s * tok_bytes);
+          uint4* ov = reinterpret_cast<uint4*>(a.out) + (size_t)t * dv;
+          for (int v = lane; v < dv; v += 32) {
+            float acc[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < MAX_K; ++j) {
+              if (j < k) {
+                float f[8];
+                bf16x8_to_f32(src[(size_t)j * dv + v], f);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] = fmaf(gt[j], f[q], acc[q]);
+              }
+            }
+            ov[v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                               pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl->cempty[s]);
+        }
+      }
+      base += (uint32_t)n;
       __syncthreads();
     }
     if (!ok) break;
     __syncthreads();
   }
+  // Never leave with a bulk copy still landing in shared memory.
+  if (threadIdx.x == 0)
+    for (int s = 0; s < S; ++s)
+      if (pend & (1u << s)) wait_bar(&ctl->cfull[s], (pend_par >> s) & 1u, a.timeout_ns, nullptr);
 }
 
 // ------------------------------------------------------------------- kernel ---
@@ -421,6 +507,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
     mbar_init(&ctl->epi_done[0], 4);
     mbar_init(&ctl->epi_done[1], 4);
     mbar_init(&ctl->mma_done, 1);
+    for (int i = 0; i < CONS_SLOTS; ++i) { mbar_init(&ctl->cfull[i], 1); mbar_init(&ctl->cempty[i], 1); }
     mbar_fence_init();
     fence_proxy_async_shared();
   }
@@ -447,7 +534,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
     __syncwarp();
   }
   __syncthreads();
-  if (do_consume) role_consumer(a, ctl, nb, n_items, abort);
+  if (do_consume) role_consumer(a, ctl, smem, nb, n_items, abort);
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

@@ -33,12 +33,22 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
   const int t0 = blockIdx.x * ROUTE_TOK;
   const int t1 = min(T, t0 + ROUTE_TOK);
   const int nv = (E + 31) >> 5;
+  // software pipeline: the next token's logits are loaded while this one is ranked
+  float vn[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = lane + 32 * i;
+    vn[i] = (t0 + warp < t1 && i < nv && e < E) ? __ldg(logits + (size_t)(t0 + warp) * E + e) : -FLT_MAX;
+  }
   for (int t = t0 + warp; t < t1; t += 8) {
     float v[8];
 #pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = vn[i];
+    const int tn = t + 8;
+#pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane + 32 * i;
-      v[i] = (i < nv && e < E) ? __ldg(logits + (size_t)t * E + e) : -FLT_MAX;
+      vn[i] = (tn < t1 && i < nv && e < E) ? __ldg(logits + (size_t)tn * E + e) : -FLT_MAX;
     }
     uint32_t used = 0;
     for (int i = 0; i < 8; ++i)
@@ -161,19 +171,39 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
   __shared__ int bstart[MAX_E + 1];
   __shared__ int nbands_s;
   const int tid = threadIdx.x;
-  // counts and per-block bases (exclusive scan down each expert's column)
+  // counts and per-block bases (exclusive scan down each expert's column): the
+  // blocks are split into P contiguous parts per expert, each thread sums its part,
+  // the part sums are scanned in shared memory, then each thread writes its bases.
+  __shared__ int part_sum[1024];
+  const int P = max(1, (int)blockDim.x / E);
+  const int e_me = tid % E, p_me = tid / E;
+  const bool scanner = nblk > 0 && p_me < P;
+  const int per = nblk > 0 ? cdiv(nblk, P) : 0;
+  const int bl0 = min(nblk, p_me * per), bl1 = min(nblk, bl0 + per);
+  if (scanner) {
+    int run = 0;
+#pragma unroll 8
+    for (int b = bl0; b < bl1; ++b) run += w.blk_hist[(size_t)b * E + e_me];
+    part_sum[p_me * E + e_me] = run;
+  }
+  __syncthreads();
   if (nblk > 0) {
     for (int e = tid; e < E; e += blockDim.x) {
       int run = 0;
-      for (int b = 0; b < nblk; ++b) {
-        const int hcount = w.blk_hist[(size_t)b * E + e];
-        w.blk_base[(size_t)b * E + e] = run;
-        run += hcount;
-      }
+      for (int q = 0; q < P; ++q) { const int v = part_sum[q * E + e]; part_sum[q * E + e] = run; run += v; }
       cnt[e] = run;
     }
   } else {
     for (int e = tid; e < E; e += blockDim.x) cnt[e] = offsets_in[e + 1] - offsets_in[e];
+  }
+  __syncthreads();
+  if (scanner) {
+    int run = part_sum[p_me * E + e_me];
+    for (int b = bl0; b < bl1; ++b) {
+      const int hcount = w.blk_hist[(size_t)b * E + e_me];
+      w.blk_base[(size_t)b * E + e_me] = run;
+      run += hcount;
+    }
   }
   __syncthreads();
   if (tid == 0) {

@@ -1,7 +1,8 @@
 """The whole layer, steps (a)-(e), on the GPU.
 
 * Small layers, every element: GPU vs the oracle within 2e-2 * max|ref|; routing
-  outputs bit-exact; the overlapped mode bit-identical to the sequential mode
+  outputs bit-exact (including layers whose tokens fill 3, 1 or none of the
+  consumer's staging slots); the overlapped mode bit-identical to the sequential mode
   for every consumer-SM count tried (cost model, 1, 2, 4, 8, 32), segment size
   mgb in {1, 2, 3} and with or without producers joining the combine.
 * Every benchmark workload at full size, in the configuration the benchmark
@@ -26,6 +27,10 @@ SMALL = [
     synth.small("k3_multi_band", 600, 512, 384, 4, 3),
     synth.small("hot_expert", 500, 256, 128, 16, 4, "hot"),
     synth.small("one_token", 1, 256, 128, 8, 2),
+    # consumer staging regimes: k*d*2 bytes per token against 192 KB of slots
+    synth.small("three_slots", 300, 4096, 128, 16, 8, "normal2"),    # 64 KB -> 3 slots < 5 warps
+    synth.small("one_slot", 200, 12288, 128, 8, 8),                  # 192 KB -> 1 slot
+    synth.small("no_slot", 160, 12544, 128, 8, 8),                   # 196 KB -> register fallback
 ]
 
 
