@@ -70,6 +70,7 @@ def parse():
     ap.add_argument("--consumer-sms", type=int, default=0, help="0 = cost model")
     ap.add_argument("--mgb", type=int, default=1)
     ap.add_argument("--no-join", action="store_true", help="producers do not join the combine")
+    ap.add_argument("--one-cta", action="store_true", help="128-row tiles on single CTAs instead of CTA pairs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -172,7 +173,7 @@ def run_ours(args):
     ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k, dev)
     out = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device=dev)
     kw = dict(consumer_sms=args.consumer_sms, mgb=args.mgb,
-              flags=moe.SCHED_NO_JOIN if args.no_join else 0)
+              flags=(moe.SCHED_NO_JOIN if args.no_join else 0) | (moe.SCHED_ONE_CTA if args.one_cta else 0))
 
     def step(mode, evb=None, eve=None):
         moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, mode, out=out, ev_begin=evb, ev_end=eve, **kw)
@@ -213,17 +214,29 @@ def run_ours(args):
 
     # the contract's timed region: K overlapped steps (clocks sampled meanwhile)
     t_ovl, ffn_ovl, clocks = timed(moe.MODE_OVERLAPPED, clocks=True)
-    # overlapped vs sequential: alternating rounds of K steps, medians, so that
-    # clock and power drift hits both modes alike
-    rounds = {"seq": [], "ovl": [], "seq_ffn": [], "ovl_ffn": []}
-    for _ in range(3):
-        ts, fs, _ = timed(moe.MODE_SEQUENTIAL)
-        to, fo, _ = timed(moe.MODE_OVERLAPPED)
-        rounds["seq"].append(ts); rounds["seq_ffn"].append(fs)
-        rounds["ovl"].append(to); rounds["ovl_ffn"].append(fo)
-    t_seq = statistics.median(rounds["seq"])
-    ffn_seq = statistics.median(rounds["seq_ffn"])
-    t_ovl_med = statistics.median(rounds["ovl"])
+    # overlapped vs sequential: the two modes alternate step by step (paired
+    # samples under the same clock and power state), each step timed with events
+    # on the stream; medians per mode
+    K = args.steps
+    ev = {m: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)] for m in ("seq", "ovl")}
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        for m, mode in (("seq", moe.MODE_SEQUENTIAL), ("ovl", moe.MODE_OVERLAPPED)):
+            e0, e1, fb, fe = ev[m][i]
+            e0.record(stream)
+            step(mode, fb, fe)
+            e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    step_ms = {m: [e0.elapsed_time(e1) for e0, e1, _, _ in ev[m]] for m in ev}
+    ffn_ms = {m: [fb.elapsed_time(fe) for _, _, fb, fe in ev[m]] for m in ev}
+    t_seq = statistics.median(step_ms["seq"])
+    ffn_seq = statistics.median(ffn_ms["seq"])
+    t_ovl_med = statistics.median(step_ms["ovl"])
+    ffn_ovl_med = statistics.median(ffn_ms["ovl"])
 
     # end to end through the public call: H2D of the step's inputs from pinned
     # host memory, the layer, D2H of its output, every step
@@ -253,10 +266,11 @@ def run_ours(args):
     if code != moe.MOE_OK:
         raise RuntimeError(f"timed runs: {moe.status_string(code)}")
 
-    times = torch.tensor([t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med], dtype=torch.float64, device=dev)
+    times = torch.tensor([t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med],
+                         dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med = times.tolist()
+    t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med = times.tolist()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -288,6 +302,7 @@ def run_ours(args):
             "data": "synthetic: seeded counter-based N(0,1) tokens and gate logits, random-init N(0,0.02) bf16 expert weights",
             "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "d_ff": wl.f, "E": wl.E,
                        "top_k": wl.k, "router": wl.router, "mode": "overlapped",
+                       "mma_tile": "128x256 per CTA" if args.one_cta else "256x256 per CTA pair (cta_group::2)",
                        "parallelism": f"replicas x{world} (token shards, no collective)",
                        "l2": "inputs larger than L2: active expert weights %.2f GB per step" % (B / 1e9)},
             "tflops": world * F / (t_ovl * 1e-3) / 1e12,
@@ -297,8 +312,8 @@ def run_ours(args):
                                "peak_tflops": peak_tf, "peak_hbm_gbs": hbm, "peaks": src},
             "sequential": {"value": T_all / (t_seq * 1e-3), "ms_per_step": t_seq,
                            "ffn_ms": ffn_seq, "tflops": world * F / (t_seq * 1e-3) / 1e12,
-                           "overlapped_ms_per_step": t_ovl_med,
-                           "method": "median of 3 alternating rounds of K steps per mode"},
+                           "overlapped_ms_per_step": t_ovl_med, "overlapped_ffn_ms": ffn_ovl_med,
+                           "method": "K steps of each mode, alternating step by step; medians"},
             "speedup_vs_sequential": t_seq / t_ovl_med,
             "consumer_sms": consumer_sms,
             "n_bands": n_bands,

@@ -19,9 +19,9 @@ inline size_t up(size_t v) { return (v + ALIGN - 1) & ~(ALIGN - 1); }
 // all moe_route / moe_permute need; the plan part adds the band tables; the
 // last part holds the permuted activations and the expert intermediates.
 struct Layout {
-  size_t status, sync, blk_hist, blk_base, counts, offsets, topk_idx, topk_gate, perm, row_of, arrive;
+  size_t status, sync, stamps, blk_hist, blk_base, counts, offsets, topk_idx, topk_gate, perm, row_of, arrive, ready_q;
   size_t routing_end;
-  size_t sorted_e, band_start, tile_start1, bands, band_done1, band_done2;
+  size_t sorted_e, band_start, tile_start1, bands, band_done1, band_done2, groups, group_start;
   size_t plan_end;
   size_t x_perm, h, y;
   size_t total;
@@ -35,6 +35,7 @@ Layout layout(int T, int d, int f, int E, int k) {
   size_t o = 0;
   L.status = o; o = up(o + sizeof(Status));
   L.sync = o; o = up(o + sizeof(Sync));
+  L.stamps = o; o = up(o + ((size_t)STAMP_CTAS * NSTAMP + (size_t)STAMP_BANDS * 4) * 8);
   L.blk_hist = o; o = up(o + nblk * E * 4);
   L.blk_base = o; o = up(o + nblk * E * 4);
   L.counts = o; o = up(o + (size_t)E * 4);
@@ -44,6 +45,7 @@ Layout layout(int T, int d, int f, int E, int k) {
   L.perm = o; o = up(o + R * 4);
   L.row_of = o; o = up(o + R * 4);
   L.arrive = o; o = up(o + (size_t)T * 4);
+  L.ready_q = o; o = up(o + (size_t)T * 4);
   L.routing_end = o;
   L.sorted_e = o; o = up(o + (size_t)E * 4);
   L.band_start = o; o = up(o + (size_t)(E + 1) * 4);
@@ -51,6 +53,8 @@ Layout layout(int T, int d, int f, int E, int k) {
   L.bands = o; o = up(o + mb * sizeof(Band));
   L.band_done1 = o; o = up(o + mb * 4);
   L.band_done2 = o; o = up(o + mb * 4);
+  L.groups = o; o = up(o + mb * sizeof(Group));
+  L.group_start = o; o = up(o + (size_t)(E + 1) * 4);
   L.plan_end = o;
   L.x_perm = o; o = up(o + R * d * 2);
   L.h = o; o = up(o + R * f * 2);
@@ -67,6 +71,7 @@ Work work_from(void* ws, const Layout& L, bool plan, bool acts) {
   memset(&w, 0, sizeof(w));
   w.status = at<Status>(ws, L.status);
   w.sync = at<Sync>(ws, L.sync);
+  w.stamps = at<unsigned long long>(ws, L.stamps);
   w.blk_hist = at<int32_t>(ws, L.blk_hist);
   w.blk_base = at<int32_t>(ws, L.blk_base);
   w.counts = at<int32_t>(ws, L.counts);
@@ -76,6 +81,7 @@ Work work_from(void* ws, const Layout& L, bool plan, bool acts) {
   w.perm = at<int32_t>(ws, L.perm);
   w.row_of = at<int32_t>(ws, L.row_of);
   w.arrive = at<uint32_t>(ws, L.arrive);
+  w.ready_q = at<uint32_t>(ws, L.ready_q);
   if (plan) {
     w.sorted_e = at<int32_t>(ws, L.sorted_e);
     w.band_start = at<int32_t>(ws, L.band_start);
@@ -83,6 +89,8 @@ Work work_from(void* ws, const Layout& L, bool plan, bool acts) {
     w.bands = at<Band>(ws, L.bands);
     w.band_done1 = at<uint32_t>(ws, L.band_done1);
     w.band_done2 = at<uint32_t>(ws, L.band_done2);
+    w.groups = at<Group>(ws, L.groups);
+    w.group_start = at<int32_t>(ws, L.group_start);
   }
   if (acts) {
     w.x_perm = at<__nv_bfloat16>(ws, L.x_perm);
@@ -127,12 +135,13 @@ int device_sms() {
 }
 
 // Per-SM throughputs for the split cost model, from B200 measurements: a
-// producer SM sustains about 1/148 of ~1.0 PFLOP/s of bf16 MMA inside this
-// kernel, one consumer SM moves about 40 GB/s of combine traffic, HBM ~6.5 TB/s.
+// producer SM sustains about 1/148 of ~1.2 PFLOP/s of bf16 MMA inside this kernel
+// (power-capped), one consumer SM moves about 30 GB/s of combine traffic (bulk
+// reads of expert rows plus output stores), HBM ~6.5 TB/s.
 CostModel default_cost_model() {
   CostModel cm;
-  cm.mma_flops_per_sm = 1.0e15f / 148.0f;
-  cm.copy_bytes_per_sm = 40.0e9f;
+  cm.mma_flops_per_sm = 1.2e15f / 148.0f;
+  cm.copy_bytes_per_sm = 30.0e9f;
   cm.hbm_bytes = 6.5e12f;
   cm.max_consumers = 32;
   return cm;
@@ -180,7 +189,7 @@ moe_status moe_route(const float* logits, int T, int E, int k, int32_t* topk_idx
   if (!ws || !aligned16(ws) || ws_bytes < L.routing_end) return MOE_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Work w = work_from(ws, L, false, false);
-  MOE_TRY(launch_route(logits, T, E, k, topk_idx, topk_gate, w.blk_hist, nullptr, st));
+  MOE_TRY(launch_route(logits, T, E, k, topk_idx, topk_gate, w.blk_hist, nullptr, nullptr, st));
   if (counts) MOE_TRY(launch_colsum(w.blk_hist, route_blocks(T), E, counts, st));
   return MOE_OK;
 }
@@ -207,7 +216,7 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
   w.row_of = row_of;
   const int nblk = route_blocks(T);
   MOE_TRY(launch_hist(topk_idx, T, E, k, w.blk_hist, st));
-  MOE_TRY(launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, default_cost_model(), st));
+  MOE_TRY(launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, default_cost_model(), st));
   MOE_TRY(launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, st));
   MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(x), perm, T * k, d, k,
                         static_cast<__nv_bfloat16*>(x_perm), nsm, st));
@@ -224,11 +233,12 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
     return MOE_ERR_INVALID;
   const Layout L = layout(T, d, f, E, k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  const int nsm = device_sms();
-  if (nsm <= 1) return MOE_ERR_CUDA;
+  const int G = 2;
+  const int grid = ffn_grid(G);
+  if (grid <= G) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Work w = work_from(ws, L, true, true);
-  MOE_TRY(launch_plan(w, 0, offsets, T, d, f, E, k, nsm, 1, 1, default_cost_model(), st));
+  MOE_TRY(launch_plan(w, 0, offsets, T, d, f, E, k, grid, 1, 1, G, 1, default_cost_model(), st));
   FfnArgs a;
   memset(&a, 0, sizeof(a));
   a.w = w;
@@ -237,11 +247,12 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
   a.y = static_cast<__nv_bfloat16*>(y);
   a.W1 = W1; a.W3 = W3; a.W2 = W2;
   a.R = T * k; a.T = T; a.d = d; a.f = f; a.E = E; a.k = k;
+  a.G = G;
   a.phase = PH_G1 | PH_G2;
   a.join = 0;
   a.mgb = 1;
   a.timeout_ns = 2000000000ull;
-  MOE_TRY(launch_ffn(a, nsm, st));
+  MOE_TRY(launch_ffn(a, grid, st));
   return MOE_OK;
 }
 
@@ -272,7 +283,9 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   const Layout L = layout(A.T, A.d, A.f, A.E, A.k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   const int nsm = device_sms();
-  if (nsm <= 1) return MOE_ERR_CUDA;
+  const int G = (A.flags & MOE_SCHED_ONE_CTA) ? 1 : 2;
+  const int grid = ffn_grid(G);
+  if (nsm <= 1 || grid <= G) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Work w = work_from(ws, L, true, true);
   if (A.topk_idx) w.topk_idx = A.topk_idx;
@@ -283,8 +296,10 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   const int T = A.T, d = A.d, f = A.f, E = A.E, k = A.k, R = T * k;
   const int mgb = A.mgb > 0 ? A.mgb : 1;
   const int nblk = route_blocks(T);
-  MOE_TRY(launch_route(A.logits, T, E, k, w.topk_idx, w.topk_gate, w.blk_hist, w.arrive, st));
-  MOE_TRY(launch_plan(w, nblk, nullptr, T, d, f, E, k, nsm, A.consumer_sms, mgb, default_cost_model(), st));
+  MOE_TRY(launch_route(A.logits, T, E, k, w.topk_idx, w.topk_gate, w.blk_hist, w.arrive, w.ready_q, st));
+  const int join = (A.flags & MOE_SCHED_NO_JOIN) ? 0 : 1;
+  MOE_TRY(launch_plan(w, nblk, nullptr, T, d, f, E, k, grid, A.consumer_sms, mgb, G, join,
+                      default_cost_model(), st));
   MOE_TRY(launch_scatter(w.topk_idx, T, E, k, w.blk_base, w.perm, w.row_of, st));
   MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(A.x), w.perm, R, d, k, w.x_perm, nsm, st));
   FfnArgs a;
@@ -297,22 +312,51 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   a.gate = w.topk_gate;
   a.out = static_cast<__nv_bfloat16*>(A.out);
   a.R = R; a.T = T; a.d = d; a.f = f; a.E = E; a.k = k;
+  a.G = G;
   a.mgb = mgb;
   a.flags = A.flags;
   a.timeout_ns = (A.timeout_us > 0 ? (uint64_t)A.timeout_us : 2000000ull) * 1000ull;
   if (A.ev_ffn_begin) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_begin), st));
   if (mode == MOE_MODE_OVERLAPPED) {
     a.phase = PH_G1 | PH_G2 | PH_CONS;
-    a.join = (A.flags & MOE_SCHED_NO_JOIN) ? 0 : 1;
-    MOE_TRY(launch_ffn(a, nsm, st));
+    a.join = join;
+    MOE_TRY(launch_ffn(a, grid, st));
   } else {
     a.phase = PH_G1;
-    MOE_TRY(launch_ffn(a, nsm, st));
+    MOE_TRY(launch_ffn(a, grid, st));
     a.phase = PH_G2;
-    MOE_TRY(launch_ffn(a, nsm, st));
+    MOE_TRY(launch_ffn(a, grid, st));
     MOE_TRY(launch_combine(w.y, w.row_of, w.topk_gate, T, d, k, a.out, nsm, st));
   }
   if (A.ev_ffn_end) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_end), st));
+  return MOE_OK;
+}
+
+moe_status moe_debug_band_stamps(void* ws, void* stream, uint64_t* host_out, int max_bands) {
+  if (!ws || !aligned16(ws) || !host_out || max_bands < 1) return MOE_ERR_INVALID;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  const Layout L = layout(1, BN2, BN1, 1, 1);
+  const int n = max_bands < STAMP_BANDS ? max_bands : STAMP_BANDS;
+  if (cudaMemcpy(host_out, static_cast<char*>(ws) + L.stamps + (size_t)STAMP_CTAS * NSTAMP * 8,
+                 (size_t)n * 4 * 8, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_debug_stamps(void* ws, void* stream, uint64_t* host_out, int max_ctas, int* n_ctas) {
+  if (!ws || !aligned16(ws) || !host_out || max_ctas < 1) return MOE_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  const Layout L = layout(1, BN2, BN1, 1, 1);   // the stamps sit at a shape-independent offset
+  const int n = max_ctas < STAMP_CTAS ? max_ctas : STAMP_CTAS;
+  if (cudaMemcpy(host_out, static_cast<char*>(ws) + L.stamps, (size_t)n * NSTAMP * 8,
+                 cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (n_ctas) {
+    int g = 0;
+    for (int i = 0; i < n; ++i) g += host_out[(size_t)i * NSTAMP] != 0;
+    *n_ctas = g;
+  }
   return MOE_OK;
 }
 

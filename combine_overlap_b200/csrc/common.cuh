@@ -26,6 +26,9 @@ constexpr int FFN_THREADS = 192;                    // warp0 TMA, warp1 MMA, war
 constexpr int SCHED_DEPTH = 4;
 
 constexpr int ROUTE_TOK = 128;  // tokens per route / scatter block
+constexpr int STAMP_CTAS = 256; // debug timestamps: at most this many CTAs ...
+constexpr int NSTAMP = 8;       // ... times this many 64-bit words each
+constexpr int STAMP_BANDS = 2048;  // debug per-band stamps: at most this many bands x 4 words
 constexpr int MAX_E = 256;
 constexpr int MAX_K = 8;
 
@@ -35,7 +38,7 @@ enum : uint32_t { ST_OK = 0, ST_TIMEOUT = 4 };
 enum : uint32_t {
   W_NONE = 0, W_SCHED_EMPTY = 1, W_SCHED_FULL = 2, W_STAGE_EMPTY = 3, W_STAGE_FULL = 4,
   W_TMEM_EMPTY = 5, W_TMEM_FULL = 6, W_BAND1 = 7, W_BAND2 = 8, W_DRAIN = 9,
-  W_CONS_EMPTY = 10, W_CONS_FULL = 11
+  W_CONS_EMPTY = 10, W_CONS_FULL = 11, W_CONS_QUEUE = 12, W_CONS_IDLE = 13
 };
 
 struct Status {
@@ -46,15 +49,23 @@ struct Status {
   int32_t n_tiles2;
   uint32_t where;
   int32_t n_items;
-  uint32_t pad;
+  int32_t n_groups;    // producer tile rows: groups of G consecutive bands of one expert
 };
 
 struct Sync {          // zeroed by the plan kernel on every call
-  uint32_t q1, q2, qc, pad;
+  uint32_t q1, q2, qc;  // GEMM1 tiles, GEMM2 tiles, consumer band items taken
+  uint32_t rq_alloc;    // ready-token queue: entries allocated
+  uint32_t rq_head;     // ready-token queue: entries claimed for combining
+  uint32_t pad[3];
 };
 
 struct Band {          // one row band: up to BM rows of one expert
   int32_t expert, row0, rows, pad;
+};
+
+// A producer row group: G consecutive bands of one expert (G = CTAs per MMA).
+struct Group {
+  int32_t expert, band0, row0, rows;   // rows: valid rows over the whole group
 };
 
 // Cost-model constants for the producer/consumer split (per SM throughputs).
@@ -82,11 +93,16 @@ struct Work {
   int32_t* sorted_e;    // [E]   experts by rows desc, id asc
   int32_t* band_start;  // [E+1] first band of the s-th sorted expert
   int32_t* tile_start1; // [E+1] first GEMM1 tile of the s-th sorted expert
+  Group* groups;        // [max_bands] producer row groups in priority order
+  int32_t* group_start; // [E+1] first group of the s-th sorted expert
   uint32_t* band_done1; // [max_bands] GEMM1 tiles finished per band
   uint32_t* band_done2; // [max_bands] GEMM2 tiles finished per band
-  uint32_t* arrive;     // [T] rows of token t combined so far
+  uint32_t* arrive;     // [T] rows of token t that have arrived
+  uint32_t* ready_q;    // [T] tokens whose k rows all arrived (t + 1; 0 = entry not yet written)
   Sync* sync;
   Status* status;
+  unsigned long long* stamps;  // [STAMP_CTAS][NSTAMP] debug timestamps (MOE_DBG_TIMESTAMPS),
+                               // then [STAMP_BANDS][4] per consumed band
 };
 
 __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -107,6 +123,16 @@ __device__ __forceinline__ uint64_t globaltimer() {
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
@@ -246,6 +272,86 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Clusters (CTA pairs) ---------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `cta` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t cta) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(cta));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\t"
+               "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};"
+               :: "r"(cluster_addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// TMA load whose completion is counted on the pair leader's mbarrier (`bar_cluster`
+// is a shared::cluster address, possibly in the other CTA).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* tmap, uint32_t bar_cluster, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      :: "r"(smem_u32(dst)), "l"(tmap), "r"(bar_cluster), "r"(c0), "r"(c1) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const void* tmap, uint32_t bar_cluster,
+                                                 int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];"
+      :: "r"(smem_u32(dst)), "l"(tmap), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+               :: "r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A * B over a CTA pair (M = 256: 128 rows of A and half of B's N
+// from each CTA's shared memory, same offsets); issued by the pair's leader.
+__device__ __forceinline__ void tc_mma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile("{\n\t.reg .pred p;\n\t"
+               "setp.ne.b32 p, %4, 0;\n\t"
+               "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+               :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// Arrive once on `bar` (same offset) in every CTA of `mask` when this thread's
+// prior pair MMAs have completed.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               :: "r"(smem_u32(bar)), "h"(mask) : "memory");
 }
 
 // Shared-memory matrix descriptor (tcgen05 format, version 1), 128-byte swizzle.

@@ -24,11 +24,15 @@
 //     of a fixed stride;
 //   * per CTA: warp 0 = tile scheduler + TMA producer, warp 1 = TMEM allocator
 //     + single-thread tcgen05.mma issuer, warps 2-5 = epilogue (TMEM -> registers
-//     -> bf16 -> global), 4-stage smem ring, two 256-column TMEM accumulators so
-//     the epilogue of one tile overlaps the main loop of the next;
-//   * GEMM1 tile: 128 rows x 128 h-columns; one N=256 MMA accumulates x*W1 and
+//     -> bf16 -> global), a 192 KB smem operand ring, two 256-column TMEM
+//     accumulators so the epilogue of one tile overlaps the main loop of the next;
+//   * two variants, G = CTAs per MMA: G = 1, one CTA per 128-row tile; G = 2
+//     (default), a cluster pair per 256-row tile with tcgen05 cta_group::2 -- the
+//     leader issues the MMAs, each CTA loads its 128 rows of A and half of B (no
+//     multicast), and work items are mirrored into the peer over DSMEM;
+//   * GEMM1 tile: 128*G rows x 128 h-columns; one N=256 MMA accumulates x*W1 and
 //     x*W3 side by side (the B tile holds the W1 and W3 column blocks), and the
-//     epilogue applies silu(a)*b;  GEMM2 tile: 128 rows x 256 y-columns;
+//     epilogue applies silu(a)*b;  GEMM2 tile: 128*G rows x 256 y-columns;
 //   * A (x_perm or h) is K-major, W is stored [K][N] (N-major): both are read
 //     by TMA with 128-byte swizzle and fed to tcgen05 as K-major / MN-major
 //     operands, so the weights need no repacking;
@@ -40,25 +44,42 @@
 #include "../../include/moe.h"
 
 #include <cuda.h>
+#include <stddef.h>
 
 namespace moe {
 
 enum : int { K_END = 0, K_G1 = 1, K_G2 = 2 };
 
-constexpr int CONS_SLOTS = 16;   // at most this many tokens in flight per consumer CTA
+constexpr int CONS_SLOTS = 16;    // at most this many tokens in flight per consumer CTA
+constexpr int MAX_NST = 6;        // pipeline depth of the CTA-pair variant
+constexpr int STAGE_AREA = 196608;  // shared memory of the operand ring (and the consumer's slots)
 
-struct Item {
-  int kind, band, nt, expert, row0, rows, pad0, pad1;
+// Per-variant tiling.  G = CTAs per MMA: G = 1 computes a 128x256 tile per CTA
+// (A: 128 rows, B: all 256 columns); G = 2 computes a 256x256 tile per CTA pair
+// with tcgen05 cta_group::2 (each CTA: 128 rows of A and 128 columns of B), so a
+// CTA streams 32 KB per 64-deep k-block instead of 48 KB.
+template <int G>
+struct Cfg {
+  static constexpr int NBOX = G == 1 ? 4 : 2;                      // 64-column B boxes per CTA
+  static constexpr int STAGE = A_STAGE_BYTES + NBOX * B_BOX_BYTES;
+  static constexpr int NST = STAGE_AREA / STAGE;
+  static_assert(NST <= MAX_NST && NST * STAGE == STAGE_AREA, "stage ring must fill the area");
+};
+
+// 16-byte aligned: the pair leader copies items into its peer's ring with 16-byte
+// distributed-shared-memory stores.
+struct __align__(16) Item {
+  int kind, group, nt, expert, row0, rows, band0, pad;   // rows: valid rows of the whole group
 };
 
 struct SmemCtl {
-  uint64_t full[NSTAGE];
-  uint64_t empty[NSTAGE];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
-  uint64_t sfull[SCHED_DEPTH];
-  uint64_t sempty[SCHED_DEPTH];
-  uint64_t epi_done[2];   // per accumulator: the four epilogue warps stored the tile
+  uint64_t full[MAX_NST];        // operands of a stage landed (pair: counted on the leader)
+  uint64_t empty[MAX_NST];       // the MMAs reading a stage finished
+  uint64_t tfull[2];             // accumulator ready for the epilogue
+  uint64_t tempty[2];            // accumulator drained by every epilogue warp (pair: on the leader)
+  uint64_t sfull[SCHED_DEPTH];   // a work item is in the ring slot
+  uint64_t sempty[SCHED_DEPTH];  // every role read the slot (pair: on the leader)
+  uint64_t epi_done[2];          // per accumulator: this CTA's four epilogue warps stored the tile
   uint64_t mma_done;
   uint64_t cfull[CONS_SLOTS];    // consumer ring: a token's k expert rows landed in the slot
   uint64_t cempty[CONS_SLOTS];   // consumer ring: the slot's token is reduced and stored
@@ -67,10 +88,15 @@ struct SmemCtl {
   int item;
   int ok;
   int cn;                        // tokens completed by the current band
-  int ctok[BM];                  // ... and which
+  int ctok[BM];                  // ... and which,
+  int crow[BM][MAX_K];           // ... their k expert rows
+  float cgate[BM][MAX_K];        // ... and their k gates (staged once, read by every warp)
 };
 
-size_t ffn_smem_bytes() { return 1024 + (size_t)NSTAGE * STAGE_BYTES + sizeof(SmemCtl); }
+static_assert(offsetof(SmemCtl, ring) % 16 == 0, "ring items must be 16-byte aligned");
+static_assert(sizeof(Item) == 32, "an item is two 16-byte stores");
+
+size_t ffn_smem_bytes() { return 1024 + (size_t)STAGE_AREA + sizeof(SmemCtl); }
 
 __device__ __forceinline__ void set_error(Status* st, uint32_t where) {
   if (atomicCAS(&st->code, (uint32_t)ST_OK, (uint32_t)ST_TIMEOUT) == (uint32_t)ST_OK) {
@@ -78,14 +104,17 @@ __device__ __forceinline__ void set_error(Status* st, uint32_t where) {
   }
 }
 
-// Bounded mbarrier wait; `abort` (may be null) ends it early once any CTA has
-// recorded an error.
+// Bounded mbarrier wait (acquire at cluster scope when `cluster`, for phases that
+// the other CTA of a pair completes); `abort` (may be null) ends it early once
+// any CTA has recorded an error.
+template <bool cluster = false>
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
                                          const volatile uint32_t* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto test = [&]() { return cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (test()) return true;
   const uint64_t deadline = globaltimer() + timeout_ns;
   uint32_t n = 0;
-  while (!mbar_try_wait(bar, parity)) {
+  while (!test()) {
     if ((++n & 255u) == 0u) {
       if (globaltimer() > deadline) return false;
       if (abort && *abort) return false;
@@ -108,39 +137,40 @@ __device__ __forceinline__ bool wait_count(const uint32_t* p, uint32_t target, u
   return true;
 }
 
-__device__ __forceinline__ Item make_item(int kind, int band, int nt, const Band& bd) {
+__device__ __forceinline__ Item make_item(int kind, int group, int nt, const Group& gr) {
   Item it;
   it.kind = kind;
-  it.band = band;
+  it.group = group;
   it.nt = nt;
-  it.expert = bd.expert;
-  it.row0 = bd.row0;
-  it.rows = bd.rows;
-  it.pad0 = it.pad1 = 0;
+  it.expert = gr.expert;
+  it.row0 = gr.row0;
+  it.rows = gr.rows;
+  it.band0 = gr.band0;
+  it.pad = 0;
   return it;
 }
 
 // GEMM1 tile t: experts in priority order; inside an expert, column-block major
-// (all row bands of one 128-column block of W1/W3, then the next), so the
-// weights slice in use stays in L2 while every band of the expert reads it.
+// (every row group of one 128-column block of W1/W3, then the next), so the
+// weight slice in use stays in L2 while every group of the expert reads it.
 __device__ Item decode_g1(const Work& w, int t, int E) {
   int lo = 0, hi = E;  // tile_start1[lo] <= t < tile_start1[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (w.tile_start1[mid] <= t) lo = mid; else hi = mid;
   }
-  const int b0 = w.band_start[lo];
-  const int nbe = w.band_start[lo + 1] - b0;
+  const int g0 = w.group_start[lo];
+  const int nge = w.group_start[lo + 1] - g0;
   const int local = t - w.tile_start1[lo];
-  const int band = b0 + local % nbe;
-  return make_item(K_G1, band, local / nbe, w.bands[band]);
+  const int group = g0 + local % nge;
+  return make_item(K_G1, group, local / nge, w.groups[group]);
 }
 
-// GEMM2 tile t: band-major (all column blocks of a band, then the next band), so
-// bands complete -- and can be combined -- in priority order.
+// GEMM2 tile t: group-major (all column blocks of a row group, then the next), so
+// row bands complete -- and can be combined -- in priority order.
 __device__ Item decode_g2(const Work& w, int t, int NT2) {
-  const int band = t / NT2;
-  return make_item(K_G2, band, t % NT2, w.bands[band]);
+  const int group = t / NT2;
+  return make_item(K_G2, group, t % NT2, w.groups[group]);
 }
 
 __device__ __forceinline__ void item_range(int item, int nb, int mgb, int& b0, int& b1) {
@@ -155,81 +185,165 @@ __device__ __forceinline__ float silu_mul(float a, float b) {
   return __fdividef(a, 1.0f + __expf(-a)) * b;
 }
 
+// This CTA's rows of a row group (CTA `rank` of a G-CTA group owns band band0+rank).
+struct MyRows {
+  int row0, rows, band;
+};
+
+template <int G>
+__device__ __forceinline__ MyRows my_rows(const Item& it, uint32_t rank) {
+  MyRows m;
+  m.row0 = it.row0 + (int)rank * BM;
+  m.rows = min(BM, max(0, it.rows - (int)rank * BM));
+  m.band = it.band0 + (int)rank;
+  return m;
+}
+
+// Arrive on a barrier that lives in the pair leader (local when this CTA leads).
+template <int G>
+__device__ __forceinline__ void arrive_leader(uint64_t* bar, uint32_t rank) {
+  if (G == 1 || rank == 0) mbar_arrive(bar);
+  else mbar_arrive_remote(mapa_shared(smem_u32(bar), 0));
+}
+
 // ------------------------------------------------------------ TMA producer ---
+// G == 1, or the pair leader: takes work items from the atomic queues and puts
+// them in the ring (the leader also writes them into its peer's ring over
+// distributed shared memory).  The peer reads items from its own ring.  Each CTA
+// then loads its own 128 rows of A and its share of B for every k-block; in a
+// pair the loads count on the leader's `full` barrier.
+template <int G>
 __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
                          const CUtensorMap* tm_w3, const CUtensorMap* tm_a2,
                          const CUtensorMap* tm_w2, const FfnArgs& a, SmemCtl* ctl,
-                         uint8_t* smem, bool run_g1, bool run_g2, int n1, int n2,
+                         uint8_t* smem, uint32_t rank, bool run_g1, bool run_g2, int n1, int n2,
                          const volatile uint32_t* abort) {
+  using C = Cfg<G>;
   const Work& w = a.w;
   const int NT1 = a.f / BN1, NT2 = a.d / BN2;
   const uint64_t tmo = a.timeout_ns;
+  const bool leader = (G == 1) || rank == 0;
   int stage = 0, slot = 0;
   uint32_t ph = 0, sph = 0;
   uint32_t pending = 0, pend_par = 0;   // stages with an issued fill, and its parity
   bool g1 = run_g1, g2 = run_g2;
-  while (true) {
+  bool ok = true;
+  const bool stamp = (a.flags & MOE_DBG_TIMESTAMPS) && blockIdx.x < STAMP_CTAS;
+  unsigned long long* my_stamps = w.stamps + (size_t)blockIdx.x * NSTAMP;
+  unsigned long long n_g1 = 0, n_g2 = 0;
+  while (ok) {
     Item it;
-    it.kind = K_END;
-    if (*abort) g1 = g2 = false;
-    if (g1) {
-      const int t = (int)atomicAdd(&w.sync->q1, 1u);
-      if (t < n1) it = decode_g1(w, t, a.E); else g1 = false;
+    if (leader) {
+      it.kind = K_END;
+      if (*abort) g1 = g2 = false;
+      if (g1) {
+        const int t = (int)atomicAdd(&w.sync->q1, 1u);
+        if (t < n1) it = decode_g1(w, t, a.E);
+        else {
+          g1 = false;
+          if (stamp) my_stamps[1] = globaltimer();
+        }
+      }
+      if (it.kind == K_END && g2) {
+        const int t = (int)atomicAdd(&w.sync->q2, 1u);
+        if (t < n2) it = decode_g2(w, t, NT2); else g2 = false;
+      }
+      if (!wait_bar<G == 2>(&ctl->sempty[slot], sph ^ 1u, tmo, abort)) { set_error(w.status, W_SCHED_EMPTY); break; }
+      ctl->ring[slot] = it;
+      if (G == 2) {
+        const uint4* src = reinterpret_cast<const uint4*>(&it);
+        const uint32_t dst = mapa_shared(smem_u32(&ctl->ring[slot]), 1);
+        st_cluster_v4(dst, src[0]);
+        st_cluster_v4(dst + 16, src[1]);
+        mbar_arrive_remote(mapa_shared(smem_u32(&ctl->sfull[slot]), 1));
+      }
+      mbar_arrive(&ctl->sfull[slot]);
+    } else {
+      if (!wait_bar<true>(&ctl->sfull[slot], sph, tmo, abort)) { set_error(w.status, W_SCHED_FULL); break; }
+      it = ctl->ring[slot];
+      arrive_leader<G>(&ctl->sempty[slot], rank);
     }
-    if (it.kind == K_END && g2) {
-      const int t = (int)atomicAdd(&w.sync->q2, 1u);
-      if (t < n2) it = decode_g2(w, t, NT2); else g2 = false;
-    }
-    if (!wait_bar(&ctl->sempty[slot], sph ^ 1u, tmo, abort)) { set_error(w.status, W_SCHED_EMPTY); break; }
-    ctl->ring[slot] = it;
-    mbar_arrive(&ctl->sfull[slot]);
     if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
     if (it.kind == K_END) break;
     const bool is1 = it.kind == K_G1;
-    if (!is1) {
-      // GEMM2 reads h rows of this band: every GEMM1 column block must be stored.
-      if (!wait_count(&w.band_done1[it.band], (uint32_t)NT1, tmo, abort)) {
+    if (is1) ++n_g1; else ++n_g2;
+    const MyRows m = my_rows<G>(it, rank);
+    if (!is1 && m.rows > 0) {
+      // GEMM2 reads this CTA's h rows: every GEMM1 column block of its band must be stored.
+      if (!wait_count(&w.band_done1[m.band], (uint32_t)NT1, tmo, abort)) {
         set_error(w.status, W_BAND1);
         break;
       }
       fence_proxy_async_global();  // generic-proxy stores -> async-proxy (TMA) loads
     }
     const int nk = (is1 ? a.d : a.f) / BK;
-    bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
-      if (!wait_bar(&ctl->empty[stage], ph ^ 1u, tmo, abort)) { set_error(w.status, W_STAGE_EMPTY); ok = false; break; }
-      uint8_t* sa = smem + (size_t)stage * STAGE_BYTES;
+      if (!wait_bar<G == 2>(&ctl->empty[stage], ph ^ 1u, tmo, abort)) { set_error(w.status, W_STAGE_EMPTY); ok = false; break; }
+      uint8_t* sa = smem + (size_t)stage * C::STAGE;
       uint8_t* sb = sa + A_STAGE_BYTES;
       uint64_t* fb = &ctl->full[stage];
-      mbar_arrive_expect_tx(fb, STAGE_BYTES);
-      if (is1) {
-        tma_load_2d(sa, tm_a1, fb, kb * BK, it.row0);
-        tma_load_3d(sb, tm_w1, fb, it.nt * BN1, kb * BK, it.expert);
-        tma_load_3d(sb + B_BOX_BYTES, tm_w1, fb, it.nt * BN1 + 64, kb * BK, it.expert);
-        tma_load_3d(sb + 2 * B_BOX_BYTES, tm_w3, fb, it.nt * BN1, kb * BK, it.expert);
-        tma_load_3d(sb + 3 * B_BOX_BYTES, tm_w3, fb, it.nt * BN1 + 64, kb * BK, it.expert);
-      } else {
-        tma_load_2d(sa, tm_a2, fb, kb * BK, it.row0);
+      if (G == 1) {
+        mbar_arrive_expect_tx(fb, C::STAGE);
+        if (is1) {
+          tma_load_2d(sa, tm_a1, fb, kb * BK, m.row0);
+          tma_load_3d(sb, tm_w1, fb, it.nt * BN1, kb * BK, it.expert);
+          tma_load_3d(sb + B_BOX_BYTES, tm_w1, fb, it.nt * BN1 + 64, kb * BK, it.expert);
+          tma_load_3d(sb + 2 * B_BOX_BYTES, tm_w3, fb, it.nt * BN1, kb * BK, it.expert);
+          tma_load_3d(sb + 3 * B_BOX_BYTES, tm_w3, fb, it.nt * BN1 + 64, kb * BK, it.expert);
+        } else {
+          tma_load_2d(sa, tm_a2, fb, kb * BK, m.row0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          tma_load_3d(sb + q * B_BOX_BYTES, tm_w2, fb, it.nt * BN2 + q * 64, kb * BK, it.expert);
+          for (int q = 0; q < 4; ++q)
+            tma_load_3d(sb + q * B_BOX_BYTES, tm_w2, fb, it.nt * BN2 + q * 64, kb * BK, it.expert);
+        }
+      } else {
+        // the leader expects both CTAs' bytes; the peer's copies may land first
+        if (leader) mbar_arrive_expect_tx(fb, 2 * C::STAGE);
+        const uint32_t fbl = mapa_shared(smem_u32(fb), 0);
+        if (is1) {
+          // B columns [0,128) of the N=256 MMA come from the leader (W1), [128,256) from the peer (W3)
+          const CUtensorMap* tw = rank == 0 ? tm_w1 : tm_w3;
+          tma_load_2d_pair(sa, tm_a1, fbl, kb * BK, m.row0);
+          tma_load_3d_pair(sb, tw, fbl, it.nt * BN1, kb * BK, it.expert);
+          tma_load_3d_pair(sb + B_BOX_BYTES, tw, fbl, it.nt * BN1 + 64, kb * BK, it.expert);
+        } else {
+          tma_load_2d_pair(sa, tm_a2, fbl, kb * BK, m.row0);
+          const int n0 = it.nt * BN2 + (int)rank * 128;
+          tma_load_3d_pair(sb, tm_w2, fbl, n0, kb * BK, it.expert);
+          tma_load_3d_pair(sb + B_BOX_BYTES, tm_w2, fbl, n0 + 64, kb * BK, it.expert);
+        }
       }
       pending |= 1u << stage;
       pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
-      if (++stage == NSTAGE) { stage = 0; ph ^= 1u; }
+      if (++stage == C::NST) { stage = 0; ph ^= 1u; }
     }
-    if (!ok) break;
   }
-  // Never leave with a copy still landing in shared memory.
-  for (int s = 0; s < NSTAGE; ++s)
-    if (pending & (1u << s)) wait_bar(&ctl->full[s], (pend_par >> s) & 1u, tmo, nullptr);
+  // Never leave with a copy still landing in shared memory.  A CTA alone (and a
+  // pair leader) waits the last fill of each stage; a pair's peer, whose copies
+  // count on the leader, waits until the MMAs released each stage, and if that
+  // never comes (an aborted call), for a fixed 100 us.
+  bool drained = true;
+  for (int s = 0; s < C::NST; ++s) {
+    if (!(pending & (1u << s))) continue;
+    const uint32_t par = (pend_par >> s) & 1u;
+    if (leader) drained &= wait_bar<G == 2>(&ctl->full[s], par, tmo, nullptr);
+    else drained &= wait_bar<true>(&ctl->empty[s], par, tmo, abort);
+  }
+  if (!drained) {
+    const uint64_t until = globaltimer() + 100000ull;
+    while (globaltimer() < until) __nanosleep(1000);
+  }
+  if (stamp) { my_stamps[4] = n_g1; my_stamps[5] = n_g2; }
 }
 
 // --------------------------------------------------------------- MMA issuer ---
+// One thread (G == 1: each CTA; G == 2: the pair leader) issues every MMA.
+template <int G>
 __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t tmem_base,
                          const volatile uint32_t* abort) {
+  using C = Cfg<G>;
   const uint64_t tmo = a.timeout_ns;
-  constexpr uint32_t idesc = idesc_bf16_f32(BM, 256, true);
+  constexpr uint32_t idesc = idesc_bf16_f32(BM * G, 256, true);
   int stage = 0, slot = 0, acc = 0;
   uint32_t ph = 0, sph = 0, aph = 0;
   while (true) {
@@ -238,38 +352,49 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
     mbar_arrive(&ctl->sempty[slot]);
     if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
     if (it.kind == K_END) break;
-    if (!wait_bar(&ctl->tempty[acc], aph ^ 1u, tmo, abort)) { set_error(a.w.status, W_TMEM_EMPTY); break; }
+    if (!wait_bar<G == 2>(&ctl->tempty[acc], aph ^ 1u, tmo, abort)) { set_error(a.w.status, W_TMEM_EMPTY); break; }
     tc_fence_after();
     const uint32_t dt = tmem_base + (uint32_t)(acc * ACC_COLS);
     const int nk = (it.kind == K_G1 ? a.d : a.f) / BK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
-      if (!wait_bar(&ctl->full[stage], ph, tmo, abort)) { set_error(a.w.status, W_STAGE_FULL); ok = false; break; }
+      if (!wait_bar<G == 2>(&ctl->full[stage], ph, tmo, abort)) { set_error(a.w.status, W_STAGE_FULL); ok = false; break; }
       tc_fence_after();
-      const uint32_t sa = smem_u32(smem + (size_t)stage * STAGE_BYTES);
+      const uint32_t sa = smem_u32(smem + (size_t)stage * C::STAGE);
       const uint32_t sb = sa + A_STAGE_BYTES;
 #pragma unroll
       for (int ks = 0; ks < BK / 16; ++ks) {
         const uint64_t ad = smem_desc_sw128(sa + ks * 32, 16, 1024);
         const uint64_t bd = smem_desc_sw128(sb + ks * 2048, B_BOX_BYTES, 1024);
-        tc_mma_f16(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+        if (G == 1) tc_mma_f16(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+        else tc_mma_f16_pair(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
       }
-      tc_commit(&ctl->empty[stage]);  // frees the smem stage once these MMAs finish
-      if (++stage == NSTAGE) { stage = 0; ph ^= 1u; }
+      // frees the smem stage (in both CTAs of a pair) once these MMAs finish
+      if (G == 1) tc_commit(&ctl->empty[stage]);
+      else tc_commit_pair(&ctl->empty[stage], (uint16_t)0x3);
+      if (++stage == C::NST) { stage = 0; ph ^= 1u; }
     }
     if (!ok) break;
-    tc_commit(&ctl->tfull[acc]);      // accumulator ready for the epilogue
+    // accumulator ready for the epilogue (of both CTAs of a pair)
+    if (G == 1) tc_commit(&ctl->tfull[acc]);
+    else tc_commit_pair(&ctl->tfull[acc], (uint16_t)0x3);
     acc ^= 1;
     if (acc == 0) aph ^= 1u;
   }
   // Wait for every MMA this thread issued before TMEM can be released.
-  tc_commit(&ctl->mma_done);
+  if (G == 1) tc_commit(&ctl->mma_done);
+  else tc_commit_pair(&ctl->mma_done, (uint16_t)0x1);
   wait_bar(&ctl->mma_done, 0u, tmo, nullptr);
 }
 
 // ----------------------------------------------------------------- epilogue ---
-__device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base, int warp,
-                              int lane, const volatile uint32_t* abort) {
+// Four warps per CTA; warp q (= warp id mod 4) owns TMEM lanes [32q, 32q+32), i.e.
+// rows 32q.. of this CTA's 128 rows.  TMEM -> registers -> bf16 -> 16-byte global
+// stores, masked to the band's valid rows; then the tile is published on the
+// band's counter.
+template <int G>
+__device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base, uint32_t rank,
+                              int warp, int lane, const volatile uint32_t* abort) {
   const Work& w = a.w;
   const uint64_t tmo = a.timeout_ns;
   const int q = warp & 3;                 // TMEM lane quadrant this warp may read
@@ -279,20 +404,21 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
   while (true) {
     // Every lane waits; the warp proceeds only if all lanes saw the phase, so a
     // timeout never splits the warp before the .sync.aligned TMEM loads.
-    bool ok = __all_sync(0xffffffffu, wait_bar(&ctl->sfull[slot], sph, tmo, abort));
+    bool ok = __all_sync(0xffffffffu, wait_bar<G == 2>(&ctl->sfull[slot], sph, tmo, abort));
     if (!ok) { if (lane == 0) set_error(w.status, W_SCHED_FULL); break; }
     const Item it = ctl->ring[slot];
     __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->sempty[slot]);
+    if (lane == 0) arrive_leader<G>(&ctl->sempty[slot], rank);
     if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
     if (it.kind == K_END) break;
-    ok = __all_sync(0xffffffffu, wait_bar(&ctl->tfull[acc], aph, tmo, abort));
+    ok = __all_sync(0xffffffffu, wait_bar<G == 2>(&ctl->tfull[acc], aph, tmo, abort));
     if (!ok) { if (lane == 0) set_error(w.status, W_TMEM_FULL); break; }
     tc_fence_after();
+    const MyRows m = my_rows<G>(it, rank);
     const uint32_t tb = tmem_base + (uint32_t)(acc * ACC_COLS) + ((uint32_t)(q * 32) << 16);
-    const bool valid = row < it.rows;
+    const bool valid = row < m.rows;
     if (it.kind == K_G1) {
-      uint4* dst = reinterpret_cast<uint4*>(a.h + (size_t)(it.row0 + row) * a.f + it.nt * BN1);
+      uint4* dst = reinterpret_cast<uint4*>(a.h + (size_t)(m.row0 + row) * a.f + it.nt * BN1);
 #pragma unroll 1
       for (int c = 0; c < BN1 / 32; ++c) {
         uint32_t ra[32], rb[32];
@@ -312,7 +438,7 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
       }
       fence_proxy_async_global();   // h is read back by TMA in other CTAs
     } else {
-      uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)(it.row0 + row) * a.d + it.nt * BN2);
+      uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)(m.row0 + row) * a.d + it.nt * BN2);
 #pragma unroll 1
       for (int c = 0; c < BN2 / 32; ++c) {
         uint32_t r[32];
@@ -332,23 +458,23 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
     __syncwarp();
     const int my_acc = acc;
     if (lane == 0) {
-      mbar_arrive(&ctl->tempty[my_acc]);    // accumulator may be overwritten
-      mbar_arrive(&ctl->epi_done[my_acc]);  // this warp's rows of the tile are stored
+      arrive_leader<G>(&ctl->tempty[my_acc], rank);   // accumulator may be overwritten
+      mbar_arrive(&ctl->epi_done[my_acc]);             // this warp's rows of the tile are stored
     }
     acc ^= 1;
     if (acc == 0) aph ^= 1u;
-    // Publish the tile: one thread waits (bounded) for all four epilogue warps'
-    // stores of this tile, then fences and bumps the band's counter with release
-    // semantics.  A warp can run at most one tile ahead, and consecutive tiles
-    // use different accumulators, so each epi_done phase holds one tile's
+    // Publish the tile: one thread waits (bounded) for this CTA's four epilogue
+    // warps' stores of the tile, then fences and bumps its band's counter with
+    // release semantics.  A warp can run at most one tile ahead, and consecutive
+    // tiles use different accumulators, so each epi_done phase holds one tile's
     // arrivals only.
     if (warp == 2 && lane == 0) {
       const bool stored = wait_bar(&ctl->epi_done[my_acc], (eph >> my_acc) & 1u, tmo, abort);
-      const bool skip = (a.flags & MOE_DBG_SKIP_FLAG_BAND) && it.kind == K_G2 && it.band == 0;
+      const bool skip = (a.flags & MOE_DBG_SKIP_FLAG_BAND) && it.kind == K_G2 && m.band == 0;
       if (!stored) set_error(w.status, W_DRAIN);
-      else if (!skip) {
+      else if (m.rows > 0 && !skip) {
         __threadfence();
-        red_release_add(it.kind == K_G1 ? &w.band_done1[it.band] : &w.band_done2[it.band], 1u);
+        red_release_add(it.kind == K_G1 ? &w.band_done1[m.band] : &w.band_done2[m.band], 1u);
       }
     }
     eph ^= 1u << my_acc;
@@ -357,157 +483,252 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
 }
 
 // ----------------------------------------------------------------- consumer ---
-// All CTAs that consume take combine items (row bands in priority order) from a
-// shared atomic counter.  For a ready band:
-//   1. every thread takes one row of the band and bumps its token's arrival
-//      counter (acq_rel); the thread that brings it to k records the token, whose
-//      k expert rows are now all stored (published by the earlier arrivals);
-//   2. thread 0 streams each recorded token's k rows of y into a ring of shared-
-//      memory slots with cp.async.bulk (the GEMM staging buffers are idle by
-//      now), so up to CONS_SLOTS tokens' rows are in flight per SM;
-//   3. warps 1-5 reduce a slot in fp32, slot order, and store out[t] with 16-byte
-//      stores -- the same arithmetic as combine_token_warp, so both modes agree
-//      bit for bit.  Each slot has one owning warp (see below).
-// If one token's rows do not fit the staging area, the warps fall back to
+// The return step.  A consuming CTA repeatedly takes whichever work is ready:
+//  * BAND: the next combine item (row bands in priority order, [TLS] 3.3.2), once
+//    all its bands are flagged -- claimed only then, so nobody blocks on it.
+//    Every thread takes one row and bumps its token's arrival counter (acq_rel);
+//    the thread that brings it to k appends the token to the ready queue
+//    (st.release of t+1 into an allocated entry).
+//  * COMBINE: up to S ready tokens from the queue.  Their k expert rows are
+//    streamed into a shared-memory slot ring with cp.async.bulk by one thread,
+//    and warps 1-5 each reduce a column slice of every token in fp32, slot order
+//    (the arithmetic of combine_token_warp, so both modes agree bit for bit),
+//    storing out[t] with 16-byte stores.
+// Splitting arrival from reduction lets every consuming CTA share the tokens
+// that the last bands complete, instead of one CTA per band.
+// If one token's rows do not fit the staging area, warps fall back to
 // combine_token_warp straight from global memory.
+enum : int { C_IDLE = 0, C_BAND = 1, C_COMBINE = 2, C_DONE = 3, C_ERROR = 4 };
+
 __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int nb, int n_items,
                               const volatile uint32_t* abort) {
   const Work& w = a.w;
-  const int NT2 = a.d / BN2;
+  const uint32_t NT2 = (uint32_t)(a.d / BN2);
   const int k = a.k, d = a.d, dv = d >> 3;
+  const uint32_t T = (uint32_t)a.T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NWARPS = FFN_THREADS / 32;
   constexpr int NCW = NWARPS - 1;                         // reducing warps
   const uint32_t row_bytes = (uint32_t)d * 2u;
   const uint32_t tok_bytes = row_bytes * (uint32_t)k;
-  int S = (int)((size_t)NSTAGE * STAGE_BYTES / tok_bytes);
+  int S = (int)((size_t)STAGE_AREA / tok_bytes);
   if (S > CONS_SLOTS) S = CONS_SLOTS;
-  if (S > NCW) S -= S % NCW;   // slots split evenly over the reducing warps
+  const int chunk = S >= 1 ? S : NWARPS;                  // tokens per COMBINE
   uint32_t base = 0;                                      // tokens this CTA reduced so far
   uint32_t pend = 0, pend_par = 0;                        // issuer: slots with a copy issued
+  unsigned long long n_bands_done = 0;
+  const bool stamp_on = (a.flags & MOE_DBG_TIMESTAMPS) != 0;
+  uint64_t idle_since = 0;
+  int my_item = -1;                                       // thread 0: band ticket held, not yet processed
+  bool items_left = true;                                 // thread 0: band tickets may remain
   while (true) {
-    if (threadIdx.x == 0) ctl->item = *abort ? -1 : (int)atomicAdd(&w.sync->qc, 1u);
-    __syncthreads();
-    const int item = ctl->item;
-    if (item < 0 || item >= n_items) break;
-    int b0, b1;
-    item_range(item, nb, a.mgb, b0, b1);
-    bool ok = true;
-    for (int b = b0; b < b1; ++b) {
-      if (threadIdx.x == 0) {
-        const bool ready = wait_count(&w.band_done2[b], (uint32_t)NT2, a.timeout_ns, abort);
-        if (!ready) set_error(w.status, W_BAND2);
-        ctl->ok = ready ? 1 : 0;
-        ctl->cn = 0;
+    // ---- thread 0 decides what to do next.  Band items and queue entries are
+    // taken with fetch-and-add tickets (no CAS contention at the tail).  A CTA
+    // holding a band ticket waits for that band, combining already-queued
+    // tokens meanwhile; once every band ticket is taken, CTAs take queue tickets
+    // and wait for their entries -- every entry will be written, because every
+    // band still to come is held by a CTA that waits only on the producers.
+    if (threadIdx.x == 0) {
+      int act = C_IDLE, arg0 = 0, arg1 = 0;
+      if (*abort) act = C_ERROR;
+      if (act == C_IDLE && my_item < 0 && items_left) {
+        const int t = (int)atomicAdd(&w.sync->qc, 1u);
+        if (t < n_items) my_item = t; else items_left = false;
       }
-      __syncthreads();
-      if (!ctl->ok) { ok = false; break; }
-      const Band bd = w.bands[b];
-      for (int r = threadIdx.x; r < bd.rows; r += FFN_THREADS) {
-        const int t = w.perm[bd.row0 + r] / k;
-        if (atom_acq_rel_add(&w.arrive[t], 1u) == (uint32_t)(k - 1)) ctl->ctok[atomicAdd(&ctl->cn, 1)] = t;
-      }
-      __syncthreads();
-      const int n = ctl->cn;
-      if (S < 1) {
-        for (int i = warp; i < n; i += NWARPS)
-          combine_token_warp(a.y, w.row_of, a.gate, ctl->ctok[i], d, k, a.out, lane);
-      } else if (warp == 0) {
-        if (lane == 0) {
-          fence_proxy_async_global();   // y rows were stored by other SMs' generic stores
-          for (int i = 0; i < n; ++i) {
-            const uint32_t g = base + (uint32_t)i;
-            const int s = (int)(g % (uint32_t)S);
-            const uint32_t ph = (g / (uint32_t)S) & 1u;
-            if (!wait_bar(&ctl->cempty[s], ph ^ 1u, a.timeout_ns, abort)) { set_error(w.status, W_CONS_EMPTY); break; }
-            const int t = ctl->ctok[i];
-            uint8_t* dst = smem + (size_t)s * tok_bytes;
-            mbar_arrive_expect_tx(&ctl->cfull[s], tok_bytes);
-            for (int j = 0; j < k; ++j) {
-              const int r = w.row_of[(size_t)t * k + j];
-              bulk_load(dst + (size_t)j * row_bytes, a.y + (size_t)r * d, row_bytes, &ctl->cfull[s]);
-            }
-            pend |= 1u << s;
-            pend_par = (pend_par & ~(1u << s)) | (ph << s);
+      if (act == C_IDLE && my_item >= 0) {
+        int b0, b1;
+        item_range(my_item, nb, a.mgb, b0, b1);
+        bool ready = true;
+        for (int b = b0; b < b1 && ready; ++b) ready = ld_acquire(&w.band_done2[b]) >= NT2;
+        if (ready) {
+          act = C_BAND; arg0 = b0; arg1 = b1;
+          my_item = -1;
+        } else {
+          // meanwhile: tokens already in the queue (allocated entries only)
+          const uint32_t h = ld_relaxed(&w.sync->rq_head);
+          const uint32_t al = ld_relaxed(&w.sync->rq_alloc);
+          if (h < al) {
+            const uint32_t n = min(al - h, (uint32_t)chunk);
+            if (atomicCAS(&w.sync->rq_head, h, h + n) == h) { act = C_COMBINE; arg0 = (int)h; arg1 = (int)n; }
           }
         }
+      } else if (act == C_IDLE) {
+        const uint32_t h = atomicAdd(&w.sync->rq_head, (uint32_t)chunk);
+        if (h >= T) act = C_DONE;
+        else { act = C_COMBINE; arg0 = (int)h; arg1 = (int)min((uint32_t)chunk, T - h); }
+      }
+      if (act == C_IDLE) {
+        const uint64_t now = globaltimer();
+        if (idle_since == 0) idle_since = now;
+        else if (now - idle_since > a.timeout_ns) { set_error(w.status, W_CONS_IDLE); act = C_ERROR; }
       } else {
-        // Slot s belongs to warp 1 + s % NCW alone, which takes that slot's tokens in
-        // order, so it never waits on a slot's phase before the previous phase has
-        // completed (an mbarrier parity wait cannot tell phases two apart).
-        const int cw = warp - 1;
+        idle_since = 0;
+      }
+      ctl->item = act;
+      ctl->ok = arg0;
+      ctl->cn = arg1;
+    }
+    __syncthreads();
+    const int act = ctl->item, arg0 = ctl->ok, arg1 = ctl->cn;
+    __syncthreads();   // everyone has read the decision before thread 0 rewrites it
+    if (act == C_DONE || act == C_ERROR) break;
+    if (act == C_IDLE) {
+      if (threadIdx.x == 0) __nanosleep(200);
+      continue;
+    }
+    if (act == C_BAND) {
+      for (int b = arg0; b < arg1; ++b) {
+        const bool bstamp = stamp_on && b < STAMP_BANDS && threadIdx.x == 0;
+        unsigned long long* bs = w.stamps + (size_t)STAMP_CTAS * NSTAMP + (size_t)b * 4;
+        if (bstamp) { bs[0] = globaltimer(); bs[3] = blockIdx.x; }
+        const Band bd = w.bands[b];
+        unsigned long long completed = 0;
+        for (int r = threadIdx.x; r < bd.rows; r += FFN_THREADS) {
+          const int t = w.perm[bd.row0 + r] / k;
+          if (atom_acq_rel_add(&w.arrive[t], 1u) == (uint32_t)(k - 1)) {
+            const uint32_t e = atomicAdd(&w.sync->rq_alloc, 1u);
+            __threadfence();
+            st_release(&w.ready_q[e], (uint32_t)t + 1u);
+            ++completed;
+          }
+        }
+        ++n_bands_done;
+        if (bstamp) { bs[1] = globaltimer(); bs[2] = completed; }
+      }
+      __syncthreads();
+      continue;
+    }
+    // ---- C_COMBINE: queue entries [arg0, arg0 + arg1)
+    const int n = arg1;
+    bool got = true;
+    if (threadIdx.x < n) {
+      // the entry is (or will be) allocated and written by a band's arrivals: bounded spin
+      uint32_t* q = &w.ready_q[arg0 + threadIdx.x];
+      uint32_t v = ld_acquire(q);
+      const uint64_t deadline = globaltimer() + a.timeout_ns;
+      while (v == 0u && globaltimer() < deadline && !*abort) {
+        __nanosleep(64);
+        v = ld_acquire(q);
+      }
+      if (v == 0u) { set_error(w.status, W_CONS_QUEUE); got = false; }
+      else {
+        const int t = (int)v - 1;
+        ctl->ctok[threadIdx.x] = t;
+        for (int j = 0; j < k; ++j) {
+          ctl->crow[threadIdx.x][j] = w.row_of[(size_t)t * k + j];
+          ctl->cgate[threadIdx.x][j] = a.gate[(size_t)t * k + j];
+        }
+      }
+    }
+    if (!__syncthreads_and(got)) break;
+    if (S < 1) {
+      for (int i = warp; i < n; i += NWARPS)
+        combine_token_warp(a.y, w.row_of, a.gate, ctl->ctok[i], d, k, a.out, lane);
+    } else if (warp == 0) {
+      if (lane == 0) {
+        fence_proxy_async_global();   // y rows were stored by other SMs' generic stores
         for (int i = 0; i < n; ++i) {
           const uint32_t g = base + (uint32_t)i;
           const int s = (int)(g % (uint32_t)S);
-          if (s % NCW != cw) continue;
           const uint32_t ph = (g / (uint32_t)S) & 1u;
-          if (!__all_sync(0xffffffffu, wait_bar(&ctl->cfull[s], ph, a.timeout_ns, abort))) {
-            if (lane == 0) set_error(w.status, W_CONS_FULL);
-            break;
-          }
-          const int t = ctl->ctok[i];
-          float gt[MAX_K];
-#pragma unroll
-          for (int j = 0; j < MAX_K; ++j) gt[j] = j < k ? a.gate[(size_t)t * k + j] : 0.0f;
-          const uint4* src = reinterpret_cast<const uint4*>(smem + (size_t)s * tok_bytes);
-          uint4* ov = reinterpret_cast<uint4*>(a.out) + (size_t)t * dv;
-          for (int v = lane; v < dv; v += 32) {
-            float acc[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-#pragma unroll
-            for (int j = 0; j < MAX_K; ++j) {
-              if (j < k) {
-                float f[8];
-                bf16x8_to_f32(src[(size_t)j * dv + v], f);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) acc[q] = fmaf(gt[j], f[q], acc[q]);
-              }
-            }
-            ov[v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                               pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl->cempty[s]);
+          if (!wait_bar(&ctl->cempty[s], ph ^ 1u, a.timeout_ns, abort)) { set_error(w.status, W_CONS_EMPTY); break; }
+          uint8_t* dst = smem + (size_t)s * tok_bytes;
+          mbar_arrive_expect_tx(&ctl->cfull[s], tok_bytes);
+          for (int j = 0; j < k; ++j)
+            bulk_load(dst + (size_t)j * row_bytes, a.y + (size_t)ctl->crow[i][j] * d, row_bytes,
+                      &ctl->cfull[s]);
+          pend |= 1u << s;
+          pend_par = (pend_par & ~(1u << s)) | (ph << s);
         }
       }
-      base += (uint32_t)n;
-      __syncthreads();
+    } else {
+      // Every reducing warp takes every token in order (a slice of its columns),
+      // so each warp waits each slot's phases in order -- an mbarrier parity wait
+      // cannot tell two phases apart.
+      const int cw = warp - 1;
+      for (int i = 0; i < n; ++i) {
+        const uint32_t g = base + (uint32_t)i;
+        const int s = (int)(g % (uint32_t)S);
+        const uint32_t ph = (g / (uint32_t)S) & 1u;
+        if (!__all_sync(0xffffffffu, wait_bar(&ctl->cfull[s], ph, a.timeout_ns, abort))) {
+          if (lane == 0) set_error(w.status, W_CONS_FULL);
+          break;
+        }
+        const int t = ctl->ctok[i];
+        float gt[MAX_K];
+#pragma unroll
+        for (int j = 0; j < MAX_K; ++j) gt[j] = j < k ? ctl->cgate[i][j] : 0.0f;
+        const uint4* src = reinterpret_cast<const uint4*>(smem + (size_t)s * tok_bytes);
+        uint4* ov = reinterpret_cast<uint4*>(a.out) + (size_t)t * dv;
+        for (int v = cw * 32 + lane; v < dv; v += NCW * 32) {
+          float acc[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+#pragma unroll
+          for (int j = 0; j < MAX_K; ++j) {
+            if (j < k) {
+              float f[8];
+              bf16x8_to_f32(src[(size_t)j * dv + v], f);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) acc[q] = fmaf(gt[j], f[q], acc[q]);
+            }
+          }
+          ov[v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                             pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->cempty[s]);
+      }
     }
-    if (!ok) break;
+    base += (uint32_t)n;
     __syncthreads();
   }
   // Never leave with a bulk copy still landing in shared memory.
   if (threadIdx.x == 0)
     for (int s = 0; s < S; ++s)
       if (pend & (1u << s)) wait_bar(&ctl->cfull[s], (pend_par >> s) & 1u, a.timeout_ns, nullptr);
+  if (threadIdx.x == 0 && stamp_on && blockIdx.x < STAMP_CTAS)
+    w.stamps[(size_t)blockIdx.x * NSTAMP + 6] = n_bands_done;
 }
 
 // ------------------------------------------------------------------- kernel ---
+template <int G>
 __global__ void __launch_bounds__(FFN_THREADS, 1)
 ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_w1,
            const __grid_constant__ CUtensorMap tm_w3, const __grid_constant__ CUtensorMap tm_a2,
            const __grid_constant__ CUtensorMap tm_w2, const FfnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + (size_t)NSTAGE * STAGE_BYTES);
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + (size_t)STAGE_AREA);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = G == 2 ? cluster_ctarank() : 0u;
   Status* st = a.w.status;
   const volatile uint32_t* abort = &st->code;
   const int n1 = st->n_tiles1, n2 = st->n_tiles2, nb = st->n_bands, n_items = st->n_items;
+  // consumer CTAs come in whole groups (the plan rounds C to a multiple of G)
   const bool consumer_cta = (a.phase & PH_CONS) && (int)blockIdx.x < st->consumer_sms;
   const bool run_g1 = (a.phase & PH_G1) != 0;
   const bool run_g2 = (a.phase & PH_G2) && !consumer_cta;
   const bool do_consume = (a.phase & PH_CONS) && (consumer_cta || a.join);
+  const bool stamp = (a.flags & MOE_DBG_TIMESTAMPS) && blockIdx.x < STAMP_CTAS;
+  unsigned long long* my_stamps = a.w.stamps + (size_t)blockIdx.x * NSTAMP;
+  if (stamp && threadIdx.x == 0) {
+    my_stamps[0] = globaltimer();
+    for (int i = 1; i < NSTAMP; ++i) my_stamps[i] = 0;
+    my_stamps[7] = rank;
+  }
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NSTAGE; ++i) { mbar_init(&ctl->full[i], 1); mbar_init(&ctl->empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&ctl->tfull[i], 1); mbar_init(&ctl->tempty[i], 4); }
-    for (int i = 0; i < SCHED_DEPTH; ++i) { mbar_init(&ctl->sfull[i], 1); mbar_init(&ctl->sempty[i], 5); }
+    for (int i = 0; i < MAX_NST; ++i) { mbar_init(&ctl->full[i], 1); mbar_init(&ctl->empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&ctl->tfull[i], 1); mbar_init(&ctl->tempty[i], 4 * G); }
+    for (int i = 0; i < SCHED_DEPTH; ++i) {
+      mbar_init(&ctl->sfull[i], 1);
+      mbar_init(&ctl->sempty[i], G == 1 ? 5 : 10);   // pair: leader MMA + 4 epi, peer TMA + 4 epi
+    }
     mbar_init(&ctl->epi_done[0], 4);
     mbar_init(&ctl->epi_done[1], 4);
     mbar_init(&ctl->mma_done, 1);
-    for (int i = 0; i < CONS_SLOTS; ++i) { mbar_init(&ctl->cfull[i], 1); mbar_init(&ctl->cempty[i], 1); }
+    for (int i = 0; i < CONS_SLOTS; ++i) { mbar_init(&ctl->cfull[i], 1); mbar_init(&ctl->cempty[i], FFN_THREADS / 32 - 1); }
     mbar_fence_init();
     fence_proxy_async_shared();
   }
@@ -516,29 +737,39 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
     tma_prefetch_desc(&tm_a2); tma_prefetch_desc(&tm_w2);
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+    if (G == 1) tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+    else tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
     tc_fence_before();
   }
   __syncthreads();
+  if (G == 2) cluster_sync();   // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
 
   if (run_g1 || run_g2) {
     if (warp == 0) {
-      if (lane == 0) role_tma(&tm_a1, &tm_w1, &tm_w3, &tm_a2, &tm_w2, a, ctl, smem, run_g1, run_g2, n1, n2, abort);
+      if (lane == 0)
+        role_tma<G>(&tm_a1, &tm_w1, &tm_w3, &tm_a2, &tm_w2, a, ctl, smem, rank, run_g1, run_g2, n1, n2, abort);
     } else if (warp == 1) {
-      if (lane == 0) role_mma(a, ctl, smem, tmem_base, abort);
+      if (lane == 0 && rank == 0) role_mma<G>(a, ctl, smem, tmem_base, abort);
     } else {
-      role_epilogue(a, ctl, tmem_base, warp, lane, abort);
+      role_epilogue<G>(a, ctl, tmem_base, rank, warp, lane, abort);
     }
     __syncwarp();
   }
   __syncthreads();
+  if (stamp && threadIdx.x == 0) my_stamps[2] = globaltimer();
+  // A pair's peer may still be read by the leader's MMAs until the leader is
+  // done; nobody reuses the operand ring before both CTAs finished producing.
+  if (G == 2) cluster_sync();
   if (do_consume) role_consumer(a, ctl, smem, nb, n_items, abort);
   __syncthreads();
+  if (stamp && threadIdx.x == 0) my_stamps[3] = globaltimer();
+  if (G == 2) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (G == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+    else tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -572,16 +803,61 @@ static bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t*
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const size_t smem = ffn_smem_bytes();
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+namespace {
+constexpr int MAX_DEV = 64;
+int g_configured[2][MAX_DEV] = {{0}};
+int g_grid[2][MAX_DEV] = {{0}};
+
+template <int G>
+cudaError_t configure(int dev) {
+  if (dev < 0 || dev >= MAX_DEV) return cudaErrorInvalidDevice;
+  if (g_configured[G - 1][dev]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(ffn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)ffn_smem_bytes());
+  if (e != cudaSuccess) return e;
+  int nsm = 0;
+  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  int grid = nsm;
+  if (G == 2) {
+    // as many CTA pairs as can be resident at once (one CTA per SM)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(nsm & ~1));
+    cfg.blockDim = dim3(FFN_THREADS);
+    cfg.dynamicSmemBytes = ffn_smem_bytes();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, ffn_kernel<2>, &cfg);
     if (e != cudaSuccess) return e;
-    configured[dev] = 1;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    grid = 2 * min(clusters, nsm / 2);
   }
+  g_grid[G - 1][dev] = grid;
+  g_configured[G - 1][dev] = 1;
+  return cudaSuccess;
+}
+}  // namespace
+
+int ffn_grid(int G) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const cudaError_t e = G == 2 ? configure<2>(dev) : configure<1>(dev);
+  if (e != cudaSuccess) return 0;
+  return g_grid[G - 1][dev];
+}
+
+cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = a.G == 2 ? configure<2>(dev) : configure<1>(dev);
+  if (e != cudaSuccess) return e;
   CUtensorMap tm_a1, tm_w1, tm_w3, tm_a2, tm_w2;
   const cuuint64_t R = (cuuint64_t)a.R, d = (cuuint64_t)a.d, f = (cuuint64_t)a.f, E = (cuuint64_t)a.E;
   {
@@ -604,14 +880,22 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(FFN_THREADS);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = ffn_smem_bytes();
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  if (a.G == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ffn_kernel, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, a);
+  if (a.G == 2) return cudaLaunchKernelEx(&cfg, ffn_kernel<2>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, a);
+  return cudaLaunchKernelEx(&cfg, ffn_kernel<1>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, a);
 }
 
 }  // namespace moe

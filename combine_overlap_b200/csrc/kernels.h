@@ -8,9 +8,10 @@
 namespace moe {
 
 // route.cu
+// arrive / ready_q (optional): per-token counters the route kernel zeroes.
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx,
                          float* topk_gate, int32_t* blk_hist, uint32_t* arrive_or_null,
-                         cudaStream_t s);
+                         uint32_t* ready_q_or_null, cudaStream_t s);
 cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int32_t* blk_hist,
                         cudaStream_t s);
 cudaError_t launch_colsum(const int32_t* blk_hist, int nblk, int E, int32_t* counts,
@@ -18,8 +19,9 @@ cudaError_t launch_colsum(const int32_t* blk_hist, int nblk, int E, int32_t* cou
 // Plan: counts/offsets (from blk_hist when nblk > 0, else from `offsets_in`),
 // per-block scatter bases, expert priority order, band table, tile counts,
 // zeroed sync counters and the producer/consumer split.
+// G = CTAs per MMA tile (1: 128-row tiles, 2: CTA pairs with 256-row tiles).
 cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
-                        int E, int k, int num_sms, int consumer_hint, int mgb,
+                        int E, int k, int num_sms, int consumer_hint, int mgb, int G, int join,
                         const CostModel& cm, cudaStream_t s);
 cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const int32_t* blk_base,
                            int32_t* perm, int32_t* row_of, cudaStream_t s);
@@ -42,6 +44,7 @@ struct FfnArgs {
   const float* gate;             // [T][k] (consumer role)
   __nv_bfloat16* out;            // [T][d] (consumer role)
   int R, T, d, f, E, k;
+  int G;                         // CTAs per MMA tile: 1 or 2 (cluster pair, cta_group::2)
   int phase;                     // PH_* bits
   int join;                      // producers join the combine when the tile queue drains
   int mgb;
@@ -50,6 +53,9 @@ struct FfnArgs {
 };
 
 size_t ffn_smem_bytes();
+// CTAs the persistent kernel runs with for group size G (0 on error); also sets
+// the kernel's shared-memory attribute for the current device.
+int ffn_grid(int G);
 cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s);
 
 }  // namespace moe

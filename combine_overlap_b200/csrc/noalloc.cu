@@ -105,7 +105,7 @@ extern "C" moe_status moe_permute_noalloc(const void* x, int T, int d, int E, in
   cm.max_consumers = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (launch_hist(topk_idx, T, E, k, w.blk_hist, st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, cm, st) != cudaSuccess)
+  if (launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, cm, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, st) != cudaSuccess)
     return MOE_ERR_CUDA;

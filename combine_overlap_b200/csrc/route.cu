@@ -25,7 +25,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                                                     int k, int32_t* __restrict__ topk_idx,
                                                     float* __restrict__ topk_gate,
                                                     int32_t* __restrict__ blk_hist,
-                                                    uint32_t* __restrict__ arrive) {
+                                                    uint32_t* __restrict__ arrive,
+                                                    uint32_t* __restrict__ ready_q) {
   __shared__ int hist[MAX_E];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
@@ -87,6 +88,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
         atomicAdd(&hist[sel_e[j]], 1);
       }
       if (arrive) arrive[t] = 0u;
+      if (ready_q) ready_q[t] = 0u;
     }
   }
   __syncthreads();
@@ -94,8 +96,10 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 }
 
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx,
-                         float* topk_gate, int32_t* blk_hist, uint32_t* arrive, cudaStream_t s) {
-  route_kernel<<<route_blocks(T), 256, 0, s>>>(logits, T, E, k, topk_idx, topk_gate, blk_hist, arrive);
+                         float* topk_gate, int32_t* blk_hist, uint32_t* arrive, uint32_t* ready_q,
+                         cudaStream_t s) {
+  route_kernel<<<route_blocks(T), 256, 0, s>>>(logits, T, E, k, topk_idx, topk_gate, blk_hist, arrive,
+                                               ready_q);
   return cudaGetLastError();
 }
 
@@ -134,25 +138,28 @@ cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int32_t* b
 }
 
 // ------------------------------------------------------------------- plan ---
-// Producer/consumer split (the Weave-style spatial scheduler): choose the
-// consumer SM count C minimising
-//   max( F2 / ((S - C) * phi),  Bc / min(C * beta, beta_hbm) ) + tail(C)
-// where F2 = GEMM2 FLOPs (the part the combine overlaps), Bc = combine bytes
-// (read every y row, write every output row), tail = one row band's combine on
-// C SMs after the last tile.  Deterministic: the same counts give the same C.
-__device__ int choose_consumers(int S, long long R, int T, int d, int f, const CostModel& cm) {
+// Producer/consumer split (the Weave-style spatial scheduler): choose the number
+// C of CTAs (a multiple of G, from `cmin`) that consume from the start instead of
+// running GEMM2, minimising the modelled layer tail
+//   t(C) = t2 + max(0, Bc - C * beta * t2) / min(S * beta, beta_hbm),
+//   t2   = F2 / ((S - C) * phi)
+// F2 = GEMM2 FLOPs (the part the combine can overlap), Bc = combine bytes (every
+// routed row read once, every output row written once): C dedicated consumers
+// combine during GEMM2, and whatever is left is combined by all S CTAs once the
+// GEMM queue is empty (producers join).  Deterministic: same counts, same C.
+__device__ int choose_consumers(int S, int G, int cmin, long long R, int T, int d, int f,
+                                const CostModel& cm) {
   const double F2 = 2.0 * (double)R * f * d;
   const double Bc = 2.0 * (double)R * d + 2.0 * (double)T * d;
-  const double band_bytes = 2.0 * BM * d * 2.0;
-  int best = 1;
+  const double drain = fmin((double)S * cm.copy_bytes_per_sm, (double)cm.hbm_bytes);
+  int best = cmin;
   double best_t = 1e300;
-  const int cmax = min(cm.max_consumers, S - 1);
-  for (int C = 1; C <= cmax; ++C) {
-    const double tp = F2 / ((double)(S - C) * cm.mma_flops_per_sm);
-    const double bw = fmin((double)C * cm.copy_bytes_per_sm, (double)cm.hbm_bytes);
-    const double tc = Bc / bw;
-    const double t = fmax(tp, tc) + band_bytes / ((double)C * cm.copy_bytes_per_sm);
-    if (t < best_t) { best_t = t; best = C; }
+  const int cmax = min(cm.max_consumers, S - G);
+  for (int C = cmin; C <= cmax; C += G) {
+    const double t2 = F2 / ((double)(S - C) * cm.mma_flops_per_sm);
+    const double left = fmax(0.0, Bc - (double)C * cm.copy_bytes_per_sm * t2);
+    const double t = t2 + left / drain;
+    if (t < best_t * (1.0 - 1e-9)) { best_t = t; best = C; }
   }
   return best;
 }
@@ -164,11 +171,13 @@ __host__ __device__ inline int n_items_for(int nb, int mgb) {
 
 __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int32_t* offsets_in,
                                                     int T, int d, int f, int E, int k, int num_sms,
-                                                    int consumer_hint, int mgb, CostModel cm) {
+                                                    int consumer_hint, int mgb, int G, int join,
+                                                    CostModel cm) {
   __shared__ int cnt[MAX_E];
   __shared__ int offs[MAX_E + 1];
   __shared__ int sorted[MAX_E];
   __shared__ int bstart[MAX_E + 1];
+  __shared__ int gstart[MAX_E + 1];
   __shared__ int nbands_s;
   const int tid = threadIdx.x;
   // counts and per-block bases (exclusive scan down each expert's column): the
@@ -228,38 +237,50 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
   __syncthreads();
   const int NT1 = f / BN1, NT2 = d / BN2;
   if (tid == 0) {
-    int nb = 0, nt1 = 0;
+    int nb = 0, ng = 0, nt1 = 0;
     for (int s = 0; s < E; ++s) {
       const int e = sorted[s];
       bstart[s] = nb;
+      gstart[s] = ng;
       if (w.bands) {
         w.band_start[s] = nb;
+        w.group_start[s] = ng;
         w.tile_start1[s] = nt1;
       }
       const int bands = cdiv(cnt[e], BM);
+      const int groups = cdiv(bands, G);
       nb += bands;
-      nt1 += bands * NT1;
+      ng += groups;
+      nt1 += groups * NT1;
     }
     bstart[E] = nb;
+    gstart[E] = ng;
     if (w.bands) {
       w.band_start[E] = nb;
+      w.group_start[E] = ng;
       w.tile_start1[E] = nt1;
     }
     nbands_s = nb;
     const long long R = offs[E];
-    const int C = consumer_hint > 0 ? min(consumer_hint, num_sms - 1)
-                                    : choose_consumers(num_sms, R, T, d, f, cm);
+    // without producers joining, at least one CTA group must consume from the start
+    const int cmin = join ? 0 : G;
+    int C = consumer_hint > 0 ? consumer_hint : choose_consumers(num_sms, G, cmin, R, T, d, f, cm);
+    C = G * cdiv(C, G);                         // consumers come in whole CTA groups
+    C = max(cmin, min(C, num_sms - G));         // and leave at least one producer group
     Status st;
     st.code = ST_OK;
     st.consumer_sms = C;
     st.n_bands = nb;
     st.n_tiles1 = nt1;
-    st.n_tiles2 = nb * NT2;
+    st.n_tiles2 = ng * NT2;
     st.where = W_NONE;
     st.n_items = n_items_for(nb, mgb);
-    st.pad = 0;
+    st.n_groups = ng;
     *w.status = st;
-    w.sync->q1 = 0; w.sync->q2 = 0; w.sync->qc = 0; w.sync->pad = 0;
+    Sync z;
+    z.q1 = z.q2 = z.qc = z.rq_alloc = z.rq_head = 0;
+    z.pad[0] = z.pad[1] = z.pad[2] = 0;
+    *w.sync = z;
   }
   if (w.bands == nullptr) return;   // permutation only: no tile plan wanted
   for (int s = tid; s < E; s += blockDim.x) w.sorted_e[s] = sorted[s];
@@ -275,14 +296,24 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
       bd.pad = 0;
       w.bands[b0 + i] = bd;
     }
+    const int g0 = gstart[s], nge = gstart[s + 1] - g0;
+    for (int i = 0; i < nge; ++i) {
+      Group gr;
+      gr.expert = e;
+      gr.band0 = b0 + i * G;
+      gr.row0 = offs[e] + i * G * BM;
+      gr.rows = min(G * BM, cnt[e] - i * G * BM);
+      w.groups[g0 + i] = gr;
+    }
   }
   for (int i = tid; i < nbands_s; i += blockDim.x) { w.band_done1[i] = 0u; w.band_done2[i] = 0u; }
 }
 
 cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
-                        int E, int k, int num_sms, int consumer_hint, int mgb, const CostModel& cm,
-                        cudaStream_t s) {
-  plan_kernel<<<1, 1024, 0, s>>>(w, nblk, offsets_in, T, d, f, E, k, num_sms, consumer_hint, mgb, cm);
+                        int E, int k, int num_sms, int consumer_hint, int mgb, int G, int join,
+                        const CostModel& cm, cudaStream_t s) {
+  plan_kernel<<<1, 1024, 0, s>>>(w, nblk, offsets_in, T, d, f, E, k, num_sms, consumer_hint, mgb, G,
+                                 join, cm);
   return cudaGetLastError();
 }
 

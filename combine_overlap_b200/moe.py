@@ -27,6 +27,8 @@ MOE_OK, MOE_ERR_INVALID, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE
 MODE_SEQUENTIAL, MODE_OVERLAPPED = 0, 1
 DBG_SKIP_FLAG_BAND = 0x1
 SCHED_NO_JOIN = 0x2
+SCHED_ONE_CTA = 0x4
+DBG_TIMESTAMPS = 0x8
 
 
 class MoEError(RuntimeError):
@@ -62,6 +64,10 @@ _lib.moe_get_status.argtypes = [_P, _P, ctypes.POINTER(_I), ctypes.POINTER(_I)]
 _lib.moe_status_string.argtypes = [_I]
 _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_num_sms.restype = _I
+_lib.moe_debug_stamps.argtypes = [_P, _P, _P, _I, ctypes.POINTER(_I)]
+_lib.moe_debug_stamps.restype = _I
+_lib.moe_debug_band_stamps.argtypes = [_P, _P, _P, _I]
+_lib.moe_debug_band_stamps.restype = _I
 _lib.moe_permute_noalloc.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
 _lib.moe_permute_noalloc.restype = _I
 _lib.moe_permute_noalloc_scratch_bytes.restype = _S
@@ -250,6 +256,30 @@ def get_status(ws: torch.Tensor, stream=None):
     nb = ctypes.c_int(0)
     code = _lib.moe_get_status(_ptr(ws), _stream(stream), ctypes.byref(c), ctypes.byref(nb))
     return int(code), int(c.value), int(nb.value)
+
+
+def debug_stamps(ws: torch.Tensor, stream=None):
+    """Per-CTA stamps of the last persistent launch run with DBG_TIMESTAMPS: a
+    uint64 array [n_ctas][8] (start, GEMM1 queue drained, producer done,
+    consumer done -- globaltimer ns -- GEMM1 tiles, GEMM2 tiles, consumer bands,
+    cluster rank)."""
+    import numpy as np
+    out = np.zeros((256, 8), dtype=np.uint64)
+    n = ctypes.c_int(0)
+    _check(_lib.moe_debug_stamps(_ptr(ws), _stream(stream), out.ctypes.data_as(ctypes.c_void_p), 256,
+                                 ctypes.byref(n)), "moe_debug_stamps")
+    return out[:n.value]
+
+
+def debug_band_stamps(ws: torch.Tensor, n_bands: int, stream=None):
+    """Per consumed row band of the last DBG_TIMESTAMPS launch: [n][4] uint64 (ready
+    ns, combined ns, tokens completed, consuming CTA)."""
+    import numpy as np
+    n = max(1, min(int(n_bands), 2048))
+    out = np.zeros((n, 4), dtype=np.uint64)
+    _check(_lib.moe_debug_band_stamps(_ptr(ws), _stream(stream), out.ctypes.data_as(ctypes.c_void_p), n),
+           "moe_debug_band_stamps")
+    return out
 
 
 class MoELayer:

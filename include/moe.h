@@ -67,6 +67,10 @@ typedef enum {
                                         exercises MOE_ERR_TIMEOUT without a GPU fault */
 #define MOE_SCHED_NO_JOIN      0x2u  /* producer CTAs do not join the combine after the
                                         GEMM tile queue drains (dedicated consumers only) */
+#define MOE_DBG_TIMESTAMPS     0x8u  /* the persistent kernel records per-CTA globaltimer
+                                        stamps, read back with moe_debug_stamps */
+#define MOE_SCHED_ONE_CTA      0x4u  /* 128-row MMA tiles on single CTAs instead of
+                                        256-row tiles on CTA pairs (tcgen05 cta_group::2) */
 
 typedef struct {
   int T, d, f, E, k;        /* tokens, d_model, d_ff, experts, top-k                */
@@ -82,7 +86,8 @@ typedef struct {
   int32_t* counts;          /* [E] routed rows per expert                           */
   int32_t* offsets;         /* [E+1] exclusive prefix sum of counts                 */
   int32_t* perm;            /* [T*k] routed row r -> source slot p = t*k + j        */
-  int consumer_sms;         /* overlapped mode: 0 = cost model; > 0 = this many     */
+  int consumer_sms;         /* overlapped mode: 0 = cost model; > 0 = this many (rounded
+                               up to whole CTA pairs unless MOE_SCHED_ONE_CTA)       */
   int mgb;                  /* row bands per consumer item (paper's x), >= 1; 0 = 1 */
   unsigned flags;           /* MOE_DBG_* / MOE_SCHED_* bits                         */
   int timeout_us;           /* bound on each device wait; 0 = default (2 s)         */
@@ -169,6 +174,19 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode,
  * NULL: consumer_sms = the consumer SM count used (cost model or hint),
  * n_bands = row bands (tiles of 128 rows) over all experts. */
 moe_status moe_get_status(void* ws, void* stream, int* consumer_sms, int* n_bands);
+
+/* Debug aid: synchronises `stream` and copies the per-CTA stamps of the last
+ * persistent-kernel launch made with MOE_DBG_TIMESTAMPS into host_out
+ * (n_ctas x 8 uint64: [0] start, [1] GEMM1 queue drained, [2] producer role done,
+ * [3] consumer role done (all globaltimer ns), [4] GEMM1 tiles, [5] GEMM2 tiles,
+ * [6] consumer bands, [7] cluster rank).  *n_ctas = CTAs of that launch (<= 256);
+ * host_out must hold max_ctas x 8 values. */
+moe_status moe_debug_stamps(void* ws, void* stream, uint64_t* host_out, int max_ctas, int* n_ctas);
+
+/* Debug aid, same launch: per consumed row band b < min(max_bands, 2048), 4 uint64:
+ * [0] band ready (globaltimer ns), [1] band combined, [2] tokens it completed,
+ * [3] consuming CTA.  host_out must hold max_bands x 4 values. */
+moe_status moe_debug_band_stamps(void* ws, void* stream, uint64_t* host_out, int max_bands);
 
 /* Static English description of a status code. */
 const char* moe_status_string(moe_status s);

@@ -2,7 +2,8 @@
 
 * Small layers, every element: GPU vs the oracle within 2e-2 * max|ref|; routing
   outputs bit-exact (including layers whose tokens fill 3, 1 or none of the
-  consumer's staging slots); the overlapped mode bit-identical to the sequential mode
+  consumer's staging slots), for both the CTA-pair (default) and the single-CTA
+  tile variants; the overlapped mode bit-identical to the sequential mode
   for every consumer-SM count tried (cost model, 1, 2, 4, 8, 32), segment size
   mgb in {1, 2, 3} and with or without producers joining the combine.
 * Every benchmark workload at full size, in the configuration the benchmark
@@ -60,8 +61,15 @@ def test_layer_small(orc, wl):
                dict(consumer_sms=8), dict(consumer_sms=32), dict(mgb=2), dict(mgb=3, consumer_sms=3),
                dict(flags=moe.SCHED_NO_JOIN, consumer_sms=2)):
         ovl, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, **kw)
-        assert c >= 1
+        assert c >= 0 and c % 2 == 0      # whole CTA pairs (0: producers join at the end)
         assert np.array_equal(gu.host(ovl), seq_bits), f"overlapped {kw} differs from sequential"
+    # the single-CTA (128-row tile) variant: same checks
+    one = moe.SCHED_ONE_CTA
+    seq1, _, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL, flags=one)
+    gu.assert_close(gu.host(seq1), ref["out"], what=f"sequential, one CTA ({wl.name})")
+    for kw in (dict(), dict(consumer_sms=1), dict(consumer_sms=5, mgb=2)):
+        ovl1, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=one | kw.pop("flags", 0), **kw)
+        assert np.array_equal(gu.host(ovl1), gu.host(seq1)), f"one-CTA overlapped {kw} differs"
 
 
 def test_layer_repeat_bitwise():
