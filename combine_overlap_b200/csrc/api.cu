@@ -21,7 +21,8 @@ inline size_t up(size_t v) { return (v + ALIGN - 1) & ~(ALIGN - 1); }
 struct Layout {
   size_t status, sync, stamps, blk_hist, blk_base, counts, offsets, topk_idx, topk_gate, perm, row_of, arrive, ready_q;
   size_t routing_end;
-  size_t sorted_e, band_start, tile_start1, bands, band_done1, band_done2, groups, group_start;
+  size_t sorted_e, band_start, tile_start1, bands, band_done1, band_done2, groups, group_start,
+      tok_band, expert_rank;
   size_t plan_end;
   size_t x_perm, h, y;
   size_t total;
@@ -55,6 +56,8 @@ Layout layout(int T, int d, int f, int E, int k) {
   L.band_done2 = o; o = up(o + mb * 4);
   L.groups = o; o = up(o + mb * sizeof(Group));
   L.group_start = o; o = up(o + (size_t)(E + 1) * 4);
+  L.tok_band = o; o = up(o + mb * BM * 4);
+  L.expert_rank = o; o = up(o + (size_t)E * 4);
   L.plan_end = o;
   L.x_perm = o; o = up(o + R * d * 2);
   L.h = o; o = up(o + R * f * 2);
@@ -91,6 +94,8 @@ Work work_from(void* ws, const Layout& L, bool plan, bool acts) {
     w.band_done2 = at<uint32_t>(ws, L.band_done2);
     w.groups = at<Group>(ws, L.groups);
     w.group_start = at<int32_t>(ws, L.group_start);
+    w.tok_band = at<int32_t>(ws, L.tok_band);
+    w.expert_rank = at<int32_t>(ws, L.expert_rank);
   }
   if (acts) {
     w.x_perm = at<__nv_bfloat16>(ws, L.x_perm);
@@ -217,7 +222,7 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
   const int nblk = route_blocks(T);
   MOE_TRY(launch_hist(topk_idx, T, E, k, w.blk_hist, st));
   MOE_TRY(launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, default_cost_model(), st));
-  MOE_TRY(launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, st));
+  MOE_TRY(launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, nullptr, st));
   MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(x), perm, T * k, d, k,
                         static_cast<__nv_bfloat16*>(x_perm), nsm, st));
   return MOE_OK;
@@ -300,12 +305,20 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   const int join = (A.flags & MOE_SCHED_NO_JOIN) ? 0 : 1;
   MOE_TRY(launch_plan(w, nblk, nullptr, T, d, f, E, k, grid, A.consumer_sms, mgb, G, join,
                       default_cost_model(), st));
-  MOE_TRY(launch_scatter(w.topk_idx, T, E, k, w.blk_base, w.perm, w.row_of, st));
-  MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(A.x), w.perm, R, d, k, w.x_perm, nsm, st));
+  // Default: a gather kernel writes x_perm and GEMM1 reads it with tiled TMA loads.
+  // MOE_SCHED_GATHER_A: GEMM1 gathers its A rows from x with TMA gather4 instead
+  // (no x_perm pass, but 32 gather instructions per k-block).
+  const int gather_a = (A.flags & MOE_SCHED_GATHER_A) ? 1 : 0;
+  MOE_TRY(launch_scatter(w.topk_idx, T, E, k, w.blk_base, w.perm, w.row_of, gather_a ? &w : nullptr, st));
+  if (!gather_a)
+    MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(A.x), w.perm, R, d, k, w.x_perm, nsm, st));
   FfnArgs a;
   memset(&a, 0, sizeof(a));
   a.w = w;
   a.x_perm = w.x_perm;
+  a.x = static_cast<const __nv_bfloat16*>(A.x);
+  a.tok_band = w.tok_band;
+  a.gather = gather_a;
   a.h = w.h;
   a.y = w.y;
   a.W1 = A.W1; a.W3 = A.W3; a.W2 = A.W2;

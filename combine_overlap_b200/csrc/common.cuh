@@ -25,7 +25,7 @@ constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int FFN_THREADS = 192;                    // warp0 TMA, warp1 MMA, warps2-5 epilogue
 constexpr int SCHED_DEPTH = 4;
 
-constexpr int ROUTE_TOK = 128;  // tokens per route / scatter block
+constexpr int ROUTE_TOK = 32;   // tokens per route / scatter block
 constexpr int STAMP_CTAS = 256; // debug timestamps: at most this many CTAs ...
 constexpr int NSTAMP = 8;       // ... times this many 64-bit words each
 constexpr int STAMP_BANDS = 2048;  // debug per-band stamps: at most this many bands x 4 words
@@ -86,6 +86,9 @@ struct Work {
   int32_t* offsets;     // [E+1]
   int32_t* perm;        // [R]
   int32_t* row_of;      // [R]
+  int32_t* tok_band;    // [max_bands][BM] token of each row of each band (0 past the
+                        // band's rows): GEMM1's gather indices, 512 aligned bytes per band
+  int32_t* expert_rank; // [E] position of expert e in the priority order
   __nv_bfloat16* x_perm;  // [R][d]
   __nv_bfloat16* h;       // [R][f]
   __nv_bfloat16* y;       // [R][d]
@@ -219,6 +222,17 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
+// Four rows (coordinates y0..y3) of a 2-D tensor, 64 columns from x, into 4
+// consecutive 128-byte smem rows (the tensor map's box is one row high).
+__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, uint64_t* bar, int x,
+                                           int y0, int y1, int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+      :: "r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(tmap) : "memory");
 }
@@ -325,6 +339,15 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const void* tmap, ui
       "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];"
       :: "r"(smem_u32(dst)), "l"(tmap), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
+
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const void* tmap, uint32_t bar_cluster,
+                                                int x, int y0, int y1, int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+      :: "r"(smem_u32(dst)), "l"(tmap), "r"(bar_cluster), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {

@@ -83,7 +83,9 @@ struct SmemCtl {
   uint64_t mma_done;
   uint64_t cfull[CONS_SLOTS];    // consumer ring: a token's k expert rows landed in the slot
   uint64_t cempty[CONS_SLOTS];   // consumer ring: the slot's token is reduced and stored
+  uint64_t gbar[2];              // a GEMM1 tile's gather indices landed (two items in flight)
   Item ring[SCHED_DEPTH];
+  int4 gidx[2][BM / 4];          // token of each of this CTA's 128 rows of a GEMM1 tile
   uint32_t tmem_base;
   int item;
   int ok;
@@ -212,6 +214,10 @@ __device__ __forceinline__ void arrive_leader(uint64_t* bar, uint32_t rank) {
 // distributed shared memory).  The peer reads items from its own ring.  Each CTA
 // then loads its own 128 rows of A and its share of B for every k-block; in a
 // pair the loads count on the leader's `full` barrier.
+// GEMM1's A rows are gathered straight from x (a.gather): the tile's 128 token
+// indices (one aligned 512-byte row of tok_band) are bulk-copied into shared
+// memory one work item ahead, and each k-block's A tile is 32 TMA gather4 loads
+// of 4 token rows x 64 columns into the same swizzled layout a tiled load gives.
 template <int G>
 __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
                          const CUtensorMap* tm_w3, const CUtensorMap* tm_a2,
@@ -226,13 +232,16 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
   int stage = 0, slot = 0;
   uint32_t ph = 0, sph = 0;
   uint32_t pending = 0, pend_par = 0;   // stages with an issued fill, and its parity
+  uint32_t gph = 0;                     // parity of the next wait on gbar[0], gbar[1]
+  uint32_t gpend = 0;                   // index copies issued and not yet waited, per buffer
   bool g1 = run_g1, g2 = run_g2;
   bool ok = true;
   const bool stamp = (a.flags & MOE_DBG_TIMESTAMPS) && blockIdx.x < STAMP_CTAS;
   unsigned long long* my_stamps = w.stamps + (size_t)blockIdx.x * NSTAMP;
   unsigned long long n_g1 = 0, n_g2 = 0;
-  while (ok) {
-    Item it;
+
+  // Next work item: dequeued and published by a leader, read by a peer.
+  auto next_item = [&](Item& it) -> bool {
     if (leader) {
       it.kind = K_END;
       if (*abort) g1 = g2 = false;
@@ -248,7 +257,7 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
         const int t = (int)atomicAdd(&w.sync->q2, 1u);
         if (t < n2) it = decode_g2(w, t, NT2); else g2 = false;
       }
-      if (!wait_bar<G == 2>(&ctl->sempty[slot], sph ^ 1u, tmo, abort)) { set_error(w.status, W_SCHED_EMPTY); break; }
+      if (!wait_bar<G == 2>(&ctl->sempty[slot], sph ^ 1u, tmo, abort)) { set_error(w.status, W_SCHED_EMPTY); return false; }
       ctl->ring[slot] = it;
       if (G == 2) {
         const uint4* src = reinterpret_cast<const uint4*>(&it);
@@ -259,15 +268,43 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
       }
       mbar_arrive(&ctl->sfull[slot]);
     } else {
-      if (!wait_bar<true>(&ctl->sfull[slot], sph, tmo, abort)) { set_error(w.status, W_SCHED_FULL); break; }
+      if (!wait_bar<true>(&ctl->sfull[slot], sph, tmo, abort)) { set_error(w.status, W_SCHED_FULL); return false; }
       it = ctl->ring[slot];
       arrive_leader<G>(&ctl->sempty[slot], rank);
     }
     if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
-    if (it.kind == K_END) break;
-    const bool is1 = it.kind == K_G1;
-    if (is1) ++n_g1; else ++n_g2;
+    return true;
+  };
+  // Does this CTA gather indices for the item?  (GEMM1, gathered path, own rows)
+  auto gathers = [&](const Item& it) {
+    return a.gather && it.kind == K_G1 && my_rows<G>(it, rank).rows > 0;
+  };
+  auto fetch_indices = [&](const Item& it, int buf) {
+    if (!gathers(it)) return;
     const MyRows m = my_rows<G>(it, rank);
+    fence_proxy_async_shared();   // earlier generic reads of this buffer come first
+    gpend |= 1u << buf;
+    mbar_arrive_expect_tx(&ctl->gbar[buf], BM * 4);
+    bulk_load(&ctl->gidx[buf][0], a.tok_band + (size_t)m.band * BM, BM * 4, &ctl->gbar[buf]);
+  };
+
+  Item cur;
+  int buf = 0;
+  if (!next_item(cur)) ok = false;
+  else fetch_indices(cur, buf);
+  while (ok && cur.kind != K_END) {
+    Item nxt;
+    if (!next_item(nxt)) break;
+    fetch_indices(nxt, buf ^ 1);
+    const bool is1 = cur.kind == K_G1;
+    if (is1) ++n_g1; else ++n_g2;
+    const MyRows m = my_rows<G>(cur, rank);
+    const bool gat = a.gather && is1;
+    if (gat && m.rows > 0) {
+      if (!wait_bar(&ctl->gbar[buf], (gph >> buf) & 1u, tmo, abort)) { set_error(w.status, W_STAGE_FULL); break; }
+      gph ^= 1u << buf;
+      gpend &= ~(1u << buf);
+    }
     if (!is1 && m.rows > 0) {
       // GEMM2 reads this CTA's h rows: every GEMM1 column block of its band must be stored.
       if (!wait_count(&w.band_done1[m.band], (uint32_t)NT1, tmo, abort)) {
@@ -282,42 +319,55 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
       uint8_t* sa = smem + (size_t)stage * C::STAGE;
       uint8_t* sb = sa + A_STAGE_BYTES;
       uint64_t* fb = &ctl->full[stage];
+      const uint32_t fbl = G == 2 ? mapa_shared(smem_u32(fb), 0) : 0u;
+      if (leader) mbar_arrive_expect_tx(fb, G * C::STAGE);   // a pair's leader expects both CTAs' bytes
+      // A: 128 rows x 64 columns of x_perm (tiled) or of x (gathered); h for GEMM2
+      if (gat) {
+#pragma unroll 8
+        for (int q = 0; q < BM / 4; ++q) {
+          const int4 tk = m.rows > 0 ? ctl->gidx[buf][q] : make_int4(0, 0, 0, 0);
+          if (G == 1) tma_gather4(sa + q * 512, tm_a1, fb, kb * BK, tk.x, tk.y, tk.z, tk.w);
+          else tma_gather4_pair(sa + q * 512, tm_a1, fbl, kb * BK, tk.x, tk.y, tk.z, tk.w);
+        }
+      } else if (G == 1) {
+        tma_load_2d(sa, is1 ? tm_a1 : tm_a2, fb, kb * BK, m.row0);
+      } else {
+        tma_load_2d_pair(sa, is1 ? tm_a1 : tm_a2, fbl, kb * BK, m.row0);
+      }
+      // B
       if (G == 1) {
-        mbar_arrive_expect_tx(fb, C::STAGE);
         if (is1) {
-          tma_load_2d(sa, tm_a1, fb, kb * BK, m.row0);
-          tma_load_3d(sb, tm_w1, fb, it.nt * BN1, kb * BK, it.expert);
-          tma_load_3d(sb + B_BOX_BYTES, tm_w1, fb, it.nt * BN1 + 64, kb * BK, it.expert);
-          tma_load_3d(sb + 2 * B_BOX_BYTES, tm_w3, fb, it.nt * BN1, kb * BK, it.expert);
-          tma_load_3d(sb + 3 * B_BOX_BYTES, tm_w3, fb, it.nt * BN1 + 64, kb * BK, it.expert);
+          tma_load_3d(sb, tm_w1, fb, cur.nt * BN1, kb * BK, cur.expert);
+          tma_load_3d(sb + B_BOX_BYTES, tm_w1, fb, cur.nt * BN1 + 64, kb * BK, cur.expert);
+          tma_load_3d(sb + 2 * B_BOX_BYTES, tm_w3, fb, cur.nt * BN1, kb * BK, cur.expert);
+          tma_load_3d(sb + 3 * B_BOX_BYTES, tm_w3, fb, cur.nt * BN1 + 64, kb * BK, cur.expert);
         } else {
-          tma_load_2d(sa, tm_a2, fb, kb * BK, m.row0);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            tma_load_3d(sb + q * B_BOX_BYTES, tm_w2, fb, it.nt * BN2 + q * 64, kb * BK, it.expert);
+            tma_load_3d(sb + q * B_BOX_BYTES, tm_w2, fb, cur.nt * BN2 + q * 64, kb * BK, cur.expert);
         }
       } else {
-        // the leader expects both CTAs' bytes; the peer's copies may land first
-        if (leader) mbar_arrive_expect_tx(fb, 2 * C::STAGE);
-        const uint32_t fbl = mapa_shared(smem_u32(fb), 0);
         if (is1) {
           // B columns [0,128) of the N=256 MMA come from the leader (W1), [128,256) from the peer (W3)
           const CUtensorMap* tw = rank == 0 ? tm_w1 : tm_w3;
-          tma_load_2d_pair(sa, tm_a1, fbl, kb * BK, m.row0);
-          tma_load_3d_pair(sb, tw, fbl, it.nt * BN1, kb * BK, it.expert);
-          tma_load_3d_pair(sb + B_BOX_BYTES, tw, fbl, it.nt * BN1 + 64, kb * BK, it.expert);
+          tma_load_3d_pair(sb, tw, fbl, cur.nt * BN1, kb * BK, cur.expert);
+          tma_load_3d_pair(sb + B_BOX_BYTES, tw, fbl, cur.nt * BN1 + 64, kb * BK, cur.expert);
         } else {
-          tma_load_2d_pair(sa, tm_a2, fbl, kb * BK, m.row0);
-          const int n0 = it.nt * BN2 + (int)rank * 128;
-          tma_load_3d_pair(sb, tm_w2, fbl, n0, kb * BK, it.expert);
-          tma_load_3d_pair(sb + B_BOX_BYTES, tm_w2, fbl, n0 + 64, kb * BK, it.expert);
+          const int n0 = cur.nt * BN2 + (int)rank * 128;
+          tma_load_3d_pair(sb, tm_w2, fbl, n0, kb * BK, cur.expert);
+          tma_load_3d_pair(sb + B_BOX_BYTES, tm_w2, fbl, n0 + 64, kb * BK, cur.expert);
         }
       }
       pending |= 1u << stage;
       pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
       if (++stage == C::NST) { stage = 0; ph ^= 1u; }
     }
+    cur = nxt;
+    buf ^= 1;
   }
+  // Index copies issued for items that were not processed must land too.
+  for (int b = 0; b < 2; ++b)
+    if (gpend & (1u << b)) wait_bar(&ctl->gbar[b], (gph >> b) & 1u, tmo, nullptr);
   // Never leave with a copy still landing in shared memory.  A CTA alone (and a
   // pair leader) waits the last fill of each stage; a pair's peer, whose copies
   // count on the leader, waits until the MMAs released each stage, and if that
@@ -728,6 +778,8 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
     mbar_init(&ctl->epi_done[0], 4);
     mbar_init(&ctl->epi_done[1], 4);
     mbar_init(&ctl->mma_done, 1);
+    mbar_init(&ctl->gbar[0], 1);
+    mbar_init(&ctl->gbar[1], 1);
     for (int i = 0; i < CONS_SLOTS; ++i) { mbar_init(&ctl->cfull[i], 1); mbar_init(&ctl->cempty[i], FFN_THREADS / 32 - 1); }
     mbar_fence_init();
     fence_proxy_async_shared();
@@ -860,7 +912,11 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   CUtensorMap tm_a1, tm_w1, tm_w3, tm_a2, tm_w2;
   const cuuint64_t R = (cuuint64_t)a.R, d = (cuuint64_t)a.d, f = (cuuint64_t)a.f, E = (cuuint64_t)a.E;
-  {
+  if (a.gather) {
+    // token rows of x, boxes one row high for gather4
+    const cuuint64_t dims[2] = {d, (cuuint64_t)a.T}, st[1] = {d * 2};
+    if (!encode(&tm_a1, a.x, 2, dims, st, 1)) return cudaErrorInvalidValue;
+  } else {
     const cuuint64_t dims[2] = {d, R}, st[1] = {d * 2};
     if (!encode(&tm_a1, a.x_perm, 2, dims, st, BM)) return cudaErrorInvalidValue;
   }

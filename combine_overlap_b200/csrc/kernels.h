@@ -23,8 +23,9 @@ cudaError_t launch_colsum(const int32_t* blk_hist, int nblk, int E, int32_t* cou
 cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
                         int E, int k, int num_sms, int consumer_hint, int mgb, int G, int join,
                         const CostModel& cm, cudaStream_t s);
+// With a plan (w.bands etc. set), also fills w.tok_band, GEMM1's gather indices.
 cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const int32_t* blk_base,
-                           int32_t* perm, int32_t* row_of, cudaStream_t s);
+                           int32_t* perm, int32_t* row_of, const Work* plan, cudaStream_t s);
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, int R, int d, int k,
                           __nv_bfloat16* x_perm, int num_sms, cudaStream_t s);
 
@@ -37,7 +38,10 @@ enum : int { PH_G1 = 1, PH_G2 = 2, PH_CONS = 4 };
 
 struct FfnArgs {
   Work w;
-  const __nv_bfloat16* x_perm;   // A operand of GEMM1
+  const __nv_bfloat16* x_perm;   // A operand of GEMM1 (tiled path)
+  const __nv_bfloat16* x;        // token rows for GEMM1's gathered A path
+  const int32_t* tok_band;       // [bands][BM] token of each band row (gathered path)
+  int gather;                    // 1: GEMM1 gathers its A rows from x with TMA gather4
   __nv_bfloat16* h;              // GEMM1 output / GEMM2 A operand
   __nv_bfloat16* y;              // GEMM2 output
   const void* W1; const void* W3; const void* W2;

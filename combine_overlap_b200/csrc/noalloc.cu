@@ -107,7 +107,7 @@ extern "C" moe_status moe_permute_noalloc(const void* x, int T, int d, int E, in
   if (launch_hist(topk_idx, T, E, k, w.blk_hist, st) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, cm, st) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, st) != cudaSuccess)
+  if (launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, nullptr, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (launch_gather(static_cast<const __nv_bfloat16*>(x), perm, T * k, d, k,
                     static_cast<__nv_bfloat16*>(x_perm), nsm, st) != cudaSuccess)

@@ -74,19 +74,21 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
       sel_e[j] = be;
       sel_v[j] = bv;
     }
+    // gates: lane j < k forms w_j = exp(l_j - l_0) in double; lane 0 sums them in
+    // slot order; lane j writes slot j
+    double wj = 0.0;
+    int ej = 0;
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j)
+      if (j < k && lane == j) { ej = sel_e[j]; wj = exp((double)sel_v[j] - (double)sel_v[0]); }
+    double ssum = 0.0;
+    for (int j = 0; j < k; ++j) ssum += __shfl_sync(0xffffffffu, wj, j);
+    if (lane < k) {
+      topk_idx[(size_t)t * k + lane] = ej;
+      topk_gate[(size_t)t * k + lane] = (float)(wj / ssum);
+      atomicAdd(&hist[ej], 1);
+    }
     if (lane == 0) {
-      double w[MAX_K];
-      double s = 0.0;
-      const double m = (double)sel_v[0];
-      for (int j = 0; j < k; ++j) {
-        w[j] = exp((double)sel_v[j] - m);
-        s += w[j];
-      }
-      for (int j = 0; j < k; ++j) {
-        topk_idx[(size_t)t * k + j] = sel_e[j];
-        topk_gate[(size_t)t * k + j] = (float)(w[j] / s);
-        atomicAdd(&hist[sel_e[j]], 1);
-      }
       if (arrive) arrive[t] = 0u;
       if (ready_q) ready_q[t] = 0u;
     }
@@ -283,7 +285,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
     *w.sync = z;
   }
   if (w.bands == nullptr) return;   // permutation only: no tile plan wanted
-  for (int s = tid; s < E; s += blockDim.x) w.sorted_e[s] = sorted[s];
+  for (int s = tid; s < E; s += blockDim.x) {
+    w.sorted_e[s] = sorted[s];
+    if (w.expert_rank) w.expert_rank[sorted[s]] = s;
+  }
   __syncthreads();
   for (int s = tid; s < E; s += blockDim.x) {
     const int e = sorted[s];
@@ -307,6 +312,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
     }
   }
   for (int i = tid; i < nbands_s; i += blockDim.x) { w.band_done1[i] = 0u; w.band_done2[i] = 0u; }
+  if (w.tok_band) {
+    int4* tb = reinterpret_cast<int4*>(w.tok_band);
+    for (int i = tid; i < nbands_s * (BM / 4); i += blockDim.x) tb[i] = make_int4(0, 0, 0, 0);
+  }
 }
 
 cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
@@ -327,7 +336,11 @@ cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int 
 __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ topk_idx, int T,
                                                       int E, int k, const int32_t* __restrict__ blk_base,
                                                       int32_t* __restrict__ perm,
-                                                      int32_t* __restrict__ row_of) {
+                                                      int32_t* __restrict__ row_of,
+                                                      const int32_t* __restrict__ offsets,
+                                                      const int32_t* __restrict__ band_start,
+                                                      const int32_t* __restrict__ expert_rank,
+                                                      int32_t* __restrict__ tok_band) {
   __shared__ int running[MAX_E];
   __shared__ int wcnt[8][MAX_E];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -352,6 +365,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
       const int r = base[e] + pre + rank_w;
       perm[r] = (int32_t)p;
       row_of[p] = r;
+      if (tok_band) {
+        const int pos = r - offsets[e];
+        tok_band[(size_t)(band_start[expert_rank[e]] + pos / BM) * BM + pos % BM] = (int32_t)(p / k);
+      }
     }
     __syncthreads();
     for (int e2 = threadIdx.x; e2 < E; e2 += 256) {
@@ -364,8 +381,13 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
 }
 
 cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const int32_t* blk_base,
-                           int32_t* perm, int32_t* row_of, cudaStream_t s) {
-  scatter_kernel<<<route_blocks(T), 256, 0, s>>>(topk_idx, T, E, k, blk_base, perm, row_of);
+                           int32_t* perm, int32_t* row_of, const Work* plan, cudaStream_t s) {
+  const bool tb = plan && plan->tok_band;
+  scatter_kernel<<<route_blocks(T), 256, 0, s>>>(topk_idx, T, E, k, blk_base, perm, row_of,
+                                                 tb ? plan->offsets : nullptr,
+                                                 tb ? plan->band_start : nullptr,
+                                                 tb ? plan->expert_rank : nullptr,
+                                                 tb ? plan->tok_band : nullptr);
   return cudaGetLastError();
 }
 

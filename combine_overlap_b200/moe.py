@@ -29,6 +29,7 @@ DBG_SKIP_FLAG_BAND = 0x1
 SCHED_NO_JOIN = 0x2
 SCHED_ONE_CTA = 0x4
 DBG_TIMESTAMPS = 0x8
+SCHED_GATHER_A = 0x10
 
 
 class MoEError(RuntimeError):

@@ -69,6 +69,9 @@ typedef enum {
                                         GEMM tile queue drains (dedicated consumers only) */
 #define MOE_DBG_TIMESTAMPS     0x8u  /* the persistent kernel records per-CTA globaltimer
                                         stamps, read back with moe_debug_stamps */
+#define MOE_SCHED_GATHER_A     0x10u /* GEMM1 gathers its A rows from x with TMA gather4
+                                        instead of reading a permuted copy (measured slower
+                                        on B200: 32 gather instructions per k-block) */
 #define MOE_SCHED_ONE_CTA      0x4u  /* 128-row MMA tiles on single CTAs instead of
                                         256-row tiles on CTA pairs (tcgen05 cta_group::2) */
 

@@ -32,7 +32,7 @@ def test_workspace_size_rules():
                  (256, 512, 1024, 8, 4)):
         assert ws(*args) > base
     R = 4096 * 2
-    assert ws(4096, 4096, 14336, 8, 2) >= R * 4096 * 2 * 2 + R * 14336 * 2
+    assert ws(4096, 4096, 14336, 8, 2) >= R * 4096 * 2 + R * 14336 * 2   # y and h
 
 
 def test_status_strings():

@@ -70,6 +70,12 @@ def test_layer_small(orc, wl):
     for kw in (dict(), dict(consumer_sms=1), dict(consumer_sms=5, mgb=2)):
         ovl1, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=one | kw.pop("flags", 0), **kw)
         assert np.array_equal(gu.host(ovl1), gu.host(seq1)), f"one-CTA overlapped {kw} differs"
+    # GEMM1 reading its A rows with TMA gather4 from x instead of x_perm: same
+    # arithmetic on the same rows, so the same bits, in both tile variants
+    for fl in (moe.SCHED_GATHER_A, moe.SCHED_GATHER_A | one):
+        gat, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=fl)
+        base = seq_bits if not fl & one else gu.host(seq1)
+        assert np.array_equal(gu.host(gat), base), f"gathered A (flags {fl}) differs"
 
 
 def test_layer_repeat_bitwise():
