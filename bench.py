@@ -142,6 +142,36 @@ def dist_setup(n_gpus: int):
     return world, rank, local
 
 
+def shard_workload(wl: synth.Workload, rank: int) -> synth.Workload:
+    """Rank r's token shard of a replicated layer: same shapes and expert weights
+    (the weights keep wl's seed), its own tokens and gate logits."""
+    if rank == 0:
+        return wl
+    return synth.Workload(wl.name, wl.T, wl.d, wl.f, wl.E, wl.k, wl.router, wl.seed + 1000 * rank)
+
+
+def rank_inputs(wl: synth.Workload, rank: int, device="cpu"):
+    """x, logits of rank r's token shard and the replicated expert weights."""
+    shard = shard_workload(wl, rank)
+    W1, W3, W2 = synth.make_weights(wl, device)
+    return synth.make_x(shard, device), synth.make_logits(shard, device), W1, W3, W2
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of a list of floats over all ranks (device-timed numbers:
+    the job is as slow as its slowest rank)."""
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tokens_per_s(T: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes T tokens per step."""
+    return T * world / (ms_per_step * 1e-3)
+
+
 def flops_and_bytes(wl: synth.Workload, counts):
     """Algorithmic FLOPs (6 R d f, no masked rows) and minimum HBM bytes (active
     experts' weights + x + logits + out + routing indices) of one layer."""
@@ -165,11 +195,7 @@ def run_ours(args):
 
     wl = synth.WORKLOADS[args.workload]
     # each rank its own token shard; the same expert weights on every rank
-    shard = wl if rank == 0 else synth.Workload(wl.name, wl.T, wl.d, wl.f, wl.E, wl.k, wl.router,
-                                                 wl.seed + 1000 * rank)
-    x = synth.make_x(shard, dev)
-    logits = synth.make_logits(shard, dev)
-    W1, W3, W2 = synth.make_weights(wl, dev)
+    x, logits, W1, W3, W2 = rank_inputs(wl, rank, dev)
     ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k, dev)
     out = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device=dev)
     kw = dict(consumer_sms=args.consumer_sms, mgb=args.mgb,
@@ -266,11 +292,8 @@ def run_ours(args):
     if code != moe.MOE_OK:
         raise RuntimeError(f"timed runs: {moe.status_string(code)}")
 
-    times = torch.tensor([t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med],
-                         dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med = times.tolist()
+    t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med = max_over_ranks(
+        [t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med], world, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -289,7 +312,7 @@ def run_ours(args):
         T_all = wl.T * world
         res = {
             "metric": "MoE-layer tokens/s",
-            "value": T_all / (t_ovl * 1e-3),
+            "value": job_tokens_per_s(wl.T, world, t_ovl),
             "unit": "tokens/s",
             "n_gpus": world,
             "steps": args.steps,

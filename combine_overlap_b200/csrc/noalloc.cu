@@ -10,7 +10,7 @@
 // inputs and outputs.
 //
 // The scratch is one file-scope __device__ array of PERMUTE_NOALLOC_SCRATCH_BYTES
-// (a little over 1 MiB), present on every GPU that loads the library until the
+// (a little over 4 MiB), present on every GPU that loads the library until the
 // process exits.  In host code the array's name is only a host-side stand-in,
 // never a device address, so its device address is looked up once per device
 // with cudaGetSymbolAddress (with that device current) and cached.
@@ -25,7 +25,7 @@ namespace {
 using namespace moe;
 
 constexpr int NOALLOC_MAX_T = 65536;
-constexpr int NOALLOC_MAX_BLK = (NOALLOC_MAX_T + ROUTE_TOK - 1) / ROUTE_TOK;   // 512
+constexpr int NOALLOC_MAX_BLK = (NOALLOC_MAX_T + ROUTE_TOK - 1) / ROUTE_TOK;   // 2048
 constexpr size_t HDR_BYTES = 256;   // Status + Sync, padded to 256 bytes
 constexpr size_t CNT_BYTES = (size_t)MAX_E * sizeof(int32_t);   // counts when the caller passes none
 constexpr size_t HIST_BYTES = (size_t)NOALLOC_MAX_BLK * MAX_E * sizeof(int32_t);

@@ -150,7 +150,7 @@ moe_status moe_combine(const void* y, const int32_t* row_of, const float* topk_g
  * every allocation, or code that must not call cudaMalloc where it permutes.
  * Same arguments, outputs and results as moe_permute, minus the workspace: the
  * per-block histograms and scan bases live in one fixed array inside the library
- * (moe_permute_noalloc_scratch_bytes() bytes, a little over 1 MiB), which every
+ * (moe_permute_noalloc_scratch_bytes() bytes, a little over 4 MiB), which every
  * GPU that loads the library holds until the process exits.  This call allocates
  * nothing and calls no allocating routine.
  *  - Limits: T <= 65536 (MOE_ERR_UNSUPPORTED above that), E <= 256, k <= 8,
