@@ -334,6 +334,9 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
     a.phase = PH_G1 | PH_G2 | PH_CONS;
     a.join = join;
     MOE_TRY(launch_ffn(a, grid, st));
+    // Consumers stop once the GEMM work is done; a full-occupancy combine pass
+    // finishes every token they did not (same arithmetic, so the same bits).
+    MOE_TRY(launch_combine(w.y, w.row_of, w.topk_gate, T, d, k, a.out, nsm, st, w.arrive));
   } else {
     a.phase = PH_G1;
     MOE_TRY(launch_ffn(a, grid, st));

@@ -30,6 +30,7 @@ constexpr int STAMP_CTAS = 256; // debug timestamps: at most this many CTAs ...
 constexpr int NSTAMP = 8;       // ... times this many 64-bit words each
 constexpr int STAMP_BANDS = 2048;  // debug per-band stamps: at most this many bands x 4 words
 constexpr int MAX_E = 256;
+constexpr uint32_t TOKEN_DONE = 0x80000000u;   // arrive[t] flag: a consumer combined token t
 constexpr int MAX_K = 8;
 
 // ----------------------------------------------------------------- status ---
@@ -56,7 +57,8 @@ struct Sync {          // zeroed by the plan kernel on every call
   uint32_t q1, q2, qc;  // GEMM1 tiles, GEMM2 tiles, consumer band items taken
   uint32_t rq_alloc;    // ready-token queue: entries allocated
   uint32_t rq_head;     // ready-token queue: entries claimed for combining
-  uint32_t pad[3];
+  uint32_t prod_done;   // CTAs that have left the producer role
+  uint32_t pad[2];
 };
 
 struct Band {          // one row band: up to BM rows of one expert
@@ -100,7 +102,8 @@ struct Work {
   int32_t* group_start; // [E+1] first group of the s-th sorted expert
   uint32_t* band_done1; // [max_bands] GEMM1 tiles finished per band
   uint32_t* band_done2; // [max_bands] GEMM2 tiles finished per band
-  uint32_t* arrive;     // [T] rows of token t that have arrived
+  uint32_t* arrive;     // [T] rows of token t that have arrived; TOKEN_DONE set once out[t]
+                        // is written by a consumer
   uint32_t* ready_q;    // [T] tokens whose k rows all arrived (t + 1; 0 = entry not yet written)
   Sync* sync;
   Status* status;

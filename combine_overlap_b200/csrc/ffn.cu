@@ -520,7 +520,7 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
     // arrivals only.
     if (warp == 2 && lane == 0) {
       const bool stored = wait_bar(&ctl->epi_done[my_acc], (eph >> my_acc) & 1u, tmo, abort);
-      const bool skip = (a.flags & MOE_DBG_SKIP_FLAG_BAND) && it.kind == K_G2 && m.band == 0;
+      const bool skip = (a.flags & MOE_DBG_SKIP_FLAG_BAND) && it.kind == K_G1 && m.band == 0;
       if (!stored) set_error(w.status, W_DRAIN);
       else if (m.rows > 0 && !skip) {
         __threadfence();
@@ -545,7 +545,11 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
 //    (the arithmetic of combine_token_warp, so both modes agree bit for bit),
 //    storing out[t] with 16-byte stores.
 // Splitting arrival from reduction lets every consuming CTA share the tokens
-// that the last bands complete, instead of one CTA per band.
+// that the last bands complete, instead of one CTA per band.  Consumers work only
+// while GEMM work remains (dedicated consumers during GEMM2, producers that
+// finished early during its last wave); once every CTA has left the producer
+// role they stop, and a full-occupancy combine pass after this kernel handles
+// every token not flagged TOKEN_DONE.
 // If one token's rows do not fit the staging area, warps fall back to
 // combine_token_warp straight from global memory.
 enum : int { C_IDLE = 0, C_BAND = 1, C_COMBINE = 2, C_DONE = 3, C_ERROR = 4 };
@@ -581,6 +585,10 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
     if (threadIdx.x == 0) {
       int act = C_IDLE, arg0 = 0, arg1 = 0;
       if (*abort) act = C_ERROR;
+      // Once every CTA has left the producer role the GEMM work is over: stop, and
+      // leave what is not combined yet to the full-occupancy combine pass that
+      // follows this kernel.
+      else if (ld_relaxed(&w.sync->prod_done) >= gridDim.x) act = C_DONE;
       if (act == C_IDLE && my_item < 0 && items_left) {
         const int t = (int)atomicAdd(&w.sync->qc, 1u);
         if (t < n_items) my_item = t; else items_left = false;
@@ -649,28 +657,34 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
       continue;
     }
     // ---- C_COMBINE: queue entries [arg0, arg0 + arg1)
-    const int n = arg1;
+    if (threadIdx.x == 0) ctl->cn = 0;
+    __syncthreads();
     bool got = true;
-    if (threadIdx.x < n) {
-      // the entry is (or will be) allocated and written by a band's arrivals: bounded spin
+    if (threadIdx.x < arg1) {
+      // The entry is (or will be) written by some band's arrivals.  Spin, bounded;
+      // give up once the GEMM work is over (that token is then combined by the
+      // pass after this kernel).
       uint32_t* q = &w.ready_q[arg0 + threadIdx.x];
       uint32_t v = ld_acquire(q);
       const uint64_t deadline = globaltimer() + a.timeout_ns;
-      while (v == 0u && globaltimer() < deadline && !*abort) {
+      while (v == 0u && !*abort) {
+        if (ld_relaxed(&w.sync->prod_done) >= gridDim.x) break;
+        if (globaltimer() > deadline) { set_error(w.status, W_CONS_QUEUE); got = false; break; }
         __nanosleep(64);
         v = ld_acquire(q);
       }
-      if (v == 0u) { set_error(w.status, W_CONS_QUEUE); got = false; }
-      else {
+      if (v != 0u) {
         const int t = (int)v - 1;
-        ctl->ctok[threadIdx.x] = t;
+        const int i = atomicAdd(&ctl->cn, 1);
+        ctl->ctok[i] = t;
         for (int j = 0; j < k; ++j) {
-          ctl->crow[threadIdx.x][j] = w.row_of[(size_t)t * k + j];
-          ctl->cgate[threadIdx.x][j] = a.gate[(size_t)t * k + j];
+          ctl->crow[i][j] = w.row_of[(size_t)t * k + j];
+          ctl->cgate[i][j] = a.gate[(size_t)t * k + j];
         }
       }
     }
     if (!__syncthreads_and(got)) break;
+    const int n = ctl->cn;
     if (S < 1) {
       for (int i = warp; i < n; i += NWARPS)
         combine_token_warp(a.y, w.row_of, a.gate, ctl->ctok[i], d, k, a.out, lane);
@@ -731,6 +745,9 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
       }
     }
     base += (uint32_t)n;
+    __syncthreads();
+    // every warp's slice of these tokens is stored: mark them combined
+    if (threadIdx.x < n) atomicOr(&w.arrive[ctl->ctok[threadIdx.x]], TOKEN_DONE);
     __syncthreads();
   }
   // Never leave with a bulk copy still landing in shared memory.
@@ -811,6 +828,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   }
   __syncthreads();
   if (stamp && threadIdx.x == 0) my_stamps[2] = globaltimer();
+  if (threadIdx.x == 0 && (a.phase & PH_CONS)) atomicAdd(&a.w.sync->prod_done, 1u);
   // A pair's peer may still be read by the leader's MMAs until the leader is
   // done; nobody reuses the operand ring before both CTAs finished producing.
   if (G == 2) cluster_sync();

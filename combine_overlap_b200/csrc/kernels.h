@@ -30,8 +30,10 @@ cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, int R, in
                           __nv_bfloat16* x_perm, int num_sms, cudaStream_t s);
 
 // combine.cu
+// skip (optional): arrive words; tokens flagged TOKEN_DONE are not recomputed.
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* row_of, const float* gate,
-                           int T, int d, int k, __nv_bfloat16* out, int num_sms, cudaStream_t s);
+                           int T, int d, int k, __nv_bfloat16* out, int num_sms, cudaStream_t s,
+                           const uint32_t* skip = nullptr);
 
 // ffn.cu
 enum : int { PH_G1 = 1, PH_G2 = 2, PH_CONS = 4 };

@@ -280,8 +280,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
     st.n_groups = ng;
     *w.status = st;
     Sync z;
-    z.q1 = z.q2 = z.qc = z.rq_alloc = z.rq_head = 0;
-    z.pad[0] = z.pad[1] = z.pad[2] = 0;
+    z.q1 = z.q2 = z.qc = z.rq_alloc = z.rq_head = z.prod_done = 0;
+    z.pad[0] = z.pad[1] = 0;
     *w.sync = z;
   }
   if (w.bands == nullptr) return;   // permutation only: no tile plan wanted

@@ -62,8 +62,9 @@ typedef enum {
 } moe_mode;
 
 /* Debug flags (moe_layer_args.flags). */
-#define MOE_DBG_SKIP_FLAG_BAND 0x1u  /* the producer never flags the first row band of
-                                        GEMM2, so the consumer's bounded wait runs out:
+#define MOE_DBG_SKIP_FLAG_BAND 0x1u  /* the producer never publishes that the first row
+                                        band's GEMM1 tiles are stored, so the GEMM2 tile that
+                                        reads those h rows waits until its bound runs out:
                                         exercises MOE_ERR_TIMEOUT without a GPU fault */
 #define MOE_SCHED_NO_JOIN      0x2u  /* producer CTAs do not join the combine after the
                                         GEMM tile queue drains (dedicated consumers only) */
