@@ -14,6 +14,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
                                                       const float* __restrict__ gate, int T, int d,
                                                       int k, __nv_bfloat16* __restrict__ out,
                                                       const uint32_t* __restrict__ skip) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
@@ -26,8 +28,7 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* row_of, const 
                            int T, int d, int k, __nv_bfloat16* out, int num_sms, cudaStream_t s,
                            const uint32_t* skip) {
   const int grid = max(1, min(cdiv(T, 8), num_sms * 8));
-  combine_kernel<<<grid, 256, 0, s>>>(y, row_of, gate, T, d, k, out, skip);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, s, y, row_of, gate, T, d, k, out, skip);
 }
 
 }  // namespace moe

@@ -115,6 +115,14 @@ __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ inline int max_bands(int R, int E) { return R / BM + E; }
 __host__ __device__ inline int route_blocks(int T) { return cdiv(T, ROUTE_TOK); }
 
+// --------------------------------------------------- programmatic launch ---
+// Every kernel of a layer call lets the next one launch as soon as all of its
+// own blocks are running (launch_dependents), and waits for the previous grid
+// to complete and flush (wait) before touching any of its outputs, so only the
+// launch latency between kernels is hidden, never a data dependence.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------ PTX helpers ---
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -767,24 +767,11 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + (size_t)STAGE_AREA);
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = G == 2 ? cluster_ctarank() : 0u;
-  Status* st = a.w.status;
-  const volatile uint32_t* abort = &st->code;
-  const int n1 = st->n_tiles1, n2 = st->n_tiles2, nb = st->n_bands, n_items = st->n_items;
-  // consumer CTAs come in whole groups (the plan rounds C to a multiple of G)
-  const bool consumer_cta = (a.phase & PH_CONS) && (int)blockIdx.x < st->consumer_sms;
-  const bool run_g1 = (a.phase & PH_G1) != 0;
-  const bool run_g2 = (a.phase & PH_G2) && !consumer_cta;
-  const bool do_consume = (a.phase & PH_CONS) && (consumer_cta || a.join);
-  const bool stamp = (a.flags & MOE_DBG_TIMESTAMPS) && blockIdx.x < STAMP_CTAS;
-  unsigned long long* my_stamps = a.w.stamps + (size_t)blockIdx.x * NSTAMP;
-  if (stamp && threadIdx.x == 0) {
-    my_stamps[0] = globaltimer();
-    for (int i = 1; i < NSTAMP; ++i) my_stamps[i] = 0;
-    my_stamps[7] = rank;
-  }
 
+  // prologue (touches nothing the previous kernel writes): barriers, TMEM, descriptors
   if (threadIdx.x == 0) {
     for (int i = 0; i < MAX_NST; ++i) { mbar_init(&ctl->full[i], 1); mbar_init(&ctl->empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&ctl->tfull[i], 1); mbar_init(&ctl->tempty[i], 4 * G); }
@@ -814,6 +801,24 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   if (G == 2) cluster_sync();   // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
+
+  pdl_wait();   // the plan and the operands of the previous kernels are complete from here on
+  Status* st = a.w.status;
+  const volatile uint32_t* abort = &st->code;
+  const int n1 = st->n_tiles1, n2 = st->n_tiles2, nb = st->n_bands, n_items = st->n_items;
+  // consumer CTAs come in whole groups (the plan rounds C to a multiple of G)
+  const bool consumer_cta = (a.phase & PH_CONS) && (int)blockIdx.x < st->consumer_sms;
+  const bool run_g1 = (a.phase & PH_G1) != 0;
+  const bool run_g2 = (a.phase & PH_G2) && !consumer_cta;
+  const bool do_consume = (a.phase & PH_CONS) && (consumer_cta || a.join);
+  const bool stamp = (a.flags & MOE_DBG_TIMESTAMPS) && blockIdx.x < STAMP_CTAS;
+  unsigned long long* my_stamps = a.w.stamps + (size_t)blockIdx.x * NSTAMP;
+  if (stamp && threadIdx.x == 0) {
+    my_stamps[0] = globaltimer();
+    for (int i = 1; i < NSTAMP; ++i) my_stamps[i] = 0;
+    my_stamps[7] = rank;
+  }
+  __syncthreads();
 
   if (run_g1 || run_g2) {
     if (warp == 0) {
@@ -956,18 +961,22 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   cfg.blockDim = dim3(FFN_THREADS);
   cfg.dynamicSmemBytes = ffn_smem_bytes();
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   if (a.G == 2) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // launch overlaps the previous kernel's tail; the kernel waits before its plan reads
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
   } else {
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
+    cfg.numAttrs = 1;
   }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
   if (a.G == 2) return cudaLaunchKernelEx(&cfg, ffn_kernel<2>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, a);
   return cudaLaunchKernelEx(&cfg, ffn_kernel<1>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, a);
 }

@@ -5,7 +5,27 @@
 #include <cuda_runtime.h>
 #include "common.cuh"
 
+#include <utility>
+
 namespace moe {
+
+// Launch with programmatic stream serialization (the kernel calls pdl_trigger /
+// pdl_wait), so its launch overlaps the tail of the previous kernel on `s`.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // route.cu
 // arrive / ready_q (optional): per-token counters the route kernel zeroes.

@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                                                     int32_t* __restrict__ blk_hist,
                                                     uint32_t* __restrict__ arrive,
                                                     uint32_t* __restrict__ ready_q) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int hist[MAX_E];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
@@ -100,13 +102,14 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx,
                          float* topk_gate, int32_t* blk_hist, uint32_t* arrive, uint32_t* ready_q,
                          cudaStream_t s) {
-  route_kernel<<<route_blocks(T), 256, 0, s>>>(logits, T, E, k, topk_idx, topk_gate, blk_hist, arrive,
-                                               ready_q);
-  return cudaGetLastError();
+  return launch_pdl(route_kernel, dim3(route_blocks(T)), dim3(256), 0, s, logits, T, E, k, topk_idx,
+                    topk_gate, blk_hist, arrive, ready_q);
 }
 
 __global__ void colsum_kernel(const int32_t* __restrict__ blk_hist, int nblk, int E,
                               int32_t* __restrict__ counts) {
+  pdl_trigger();
+  pdl_wait();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= E) return;
   int s = 0;
@@ -115,14 +118,15 @@ __global__ void colsum_kernel(const int32_t* __restrict__ blk_hist, int nblk, in
 }
 
 cudaError_t launch_colsum(const int32_t* blk_hist, int nblk, int E, int32_t* counts, cudaStream_t s) {
-  colsum_kernel<<<cdiv(E, 256), 256, 0, s>>>(blk_hist, nblk, E, counts);
-  return cudaGetLastError();
+  return launch_pdl(colsum_kernel, dim3(cdiv(E, 256)), dim3(256), 0, s, blk_hist, nblk, E, counts);
 }
 
 // Per-block expert histogram of given top-k ids (moe_permute's entry, where the
 // routing came from the caller rather than route_kernel).
 __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ topk_idx, int T,
                                                    int E, int k, int32_t* __restrict__ blk_hist) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int hist[MAX_E];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -135,8 +139,7 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ t
 
 cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int32_t* blk_hist,
                         cudaStream_t s) {
-  hist_kernel<<<route_blocks(T), 256, 0, s>>>(topk_idx, T, E, k, blk_hist);
-  return cudaGetLastError();
+  return launch_pdl(hist_kernel, dim3(route_blocks(T)), dim3(256), 0, s, topk_idx, T, E, k, blk_hist);
 }
 
 // ------------------------------------------------------------------- plan ---
@@ -175,6 +178,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
                                                     int T, int d, int f, int E, int k, int num_sms,
                                                     int consumer_hint, int mgb, int G, int join,
                                                     CostModel cm) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int cnt[MAX_E];
   __shared__ int offs[MAX_E + 1];
   __shared__ int sorted[MAX_E];
@@ -321,9 +326,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
 cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
                         int E, int k, int num_sms, int consumer_hint, int mgb, int G, int join,
                         const CostModel& cm, cudaStream_t s) {
-  plan_kernel<<<1, 1024, 0, s>>>(w, nblk, offsets_in, T, d, f, E, k, num_sms, consumer_hint, mgb, G,
-                                 join, cm);
-  return cudaGetLastError();
+  return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, w, nblk, offsets_in, T, d, f, E, k, num_sms,
+                    consumer_hint, mgb, G, join, cm);
 }
 
 // ---------------------------------------------------------------- scatter ---
@@ -341,6 +345,8 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
                                                       const int32_t* __restrict__ band_start,
                                                       const int32_t* __restrict__ expert_rank,
                                                       int32_t* __restrict__ tok_band) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int running[MAX_E];
   __shared__ int wcnt[8][MAX_E];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -383,12 +389,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
 cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const int32_t* blk_base,
                            int32_t* perm, int32_t* row_of, const Work* plan, cudaStream_t s) {
   const bool tb = plan && plan->tok_band;
-  scatter_kernel<<<route_blocks(T), 256, 0, s>>>(topk_idx, T, E, k, blk_base, perm, row_of,
-                                                 tb ? plan->offsets : nullptr,
-                                                 tb ? plan->band_start : nullptr,
-                                                 tb ? plan->expert_rank : nullptr,
-                                                 tb ? plan->tok_band : nullptr);
-  return cudaGetLastError();
+  return launch_pdl(scatter_kernel, dim3(route_blocks(T)), dim3(256), 0, s, topk_idx, T, E, k, blk_base,
+                    perm, row_of, (const int32_t*)(tb ? plan->offsets : nullptr),
+                    (const int32_t*)(tb ? plan->band_start : nullptr),
+                    (const int32_t*)(tb ? plan->expert_rank : nullptr), (tb ? plan->tok_band : nullptr));
 }
 
 // ----------------------------------------------------------------- gather ---
@@ -396,6 +400,8 @@ cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const i
 __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x,
                                                      const int32_t* __restrict__ perm, int R,
                                                      int dv, int k, uint4* __restrict__ x_perm) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb) {
@@ -409,9 +415,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, int R, int d, int k,
                           __nv_bfloat16* x_perm, int num_sms, cudaStream_t s) {
   const int grid = max(1, min(cdiv(R, 8), num_sms * 8));
-  gather_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const uint4*>(x), perm, R, d / 8, k,
-                                     reinterpret_cast<uint4*>(x_perm));
-  return cudaGetLastError();
+  return launch_pdl(gather_kernel, dim3(grid), dim3(256), 0, s, reinterpret_cast<const uint4*>(x), perm, R,
+                    d / 8, k, reinterpret_cast<uint4*>(x_perm));
 }
 
 }  // namespace moe
