@@ -74,6 +74,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="d=4096/E=32/top-4 sweep: T x router x consumer SMs, overlapped vs "
+                         "sequential; one JSON line per cell (not the benchmark line)")
     return ap.parse_args()
 
 
@@ -431,8 +434,59 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+def run_sweep(args):
+    """Every sweep cell: the overlapped mode at a fixed consumer-SM count (2, 4, 8)
+    or the cost model's choice (0), against the sequential mode, timed as paired
+    alternating steps (medians)."""
+    from combine_overlap_b200 import moe
+    torch.cuda.set_device(0)
+    peaks, src = load_peaks()
+    peak_tf = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+    names = [n for n in synth.WORKLOADS if n.startswith("sweep_")]
+    for name in names:
+        wl = synth.WORKLOADS[name]
+        x, logits, W1, W3, W2 = rank_inputs(wl, 0, "cuda")
+        ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
+        out = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+        counts = moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, outputs=True)[1]["counts"].cpu().tolist()
+        F, B = flops_and_bytes(wl, counts)
+        t_roof = max(F / (peak_tf * 1e12), B / (peaks["hbm_gbs"] * 1e9)) * 1e3
+        for C in (2, 4, 8, 0):
+            def step(mode):
+                moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, mode, out=out, consumer_sms=C)
+            for _ in range(args.warmup):
+                step(moe.MODE_OVERLAPPED)
+                step(moe.MODE_SEQUENTIAL)
+            evs = {m: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(args.steps)] for m in ("seq", "ovl")}
+            torch.cuda.synchronize()
+            for i in range(args.steps):
+                for m, mode in (("seq", moe.MODE_SEQUENTIAL), ("ovl", moe.MODE_OVERLAPPED)):
+                    evs[m][i][0].record()
+                    step(mode)
+                    evs[m][i][1].record()
+            torch.cuda.synchronize()
+            code, c_used, _ = moe.get_status(ws)
+            if code != moe.MOE_OK:
+                raise RuntimeError(f"{name} C={C}: {moe.status_string(code)}")
+            med = {m: statistics.median(a.elapsed_time(b) for a, b in evs[m]) for m in evs}
+            print(json.dumps({
+                "sweep": name, "T": wl.T, "router": wl.router,
+                "consumer_sms": "cost model" if C == 0 else C, "consumer_sms_used": c_used,
+                "ovl_ms": med["ovl"], "seq_ms": med["seq"], "speedup_vs_sequential": med["seq"] / med["ovl"],
+                "tokens_per_s": wl.T / (med["ovl"] * 1e-3), "tflops": F / (med["ovl"] * 1e-3) / 1e12,
+                "roofline_frac_layer": t_roof / med["ovl"],
+                "roofline_bound": "tensor" if F / (peak_tf * 1e12) >= B / (peaks["hbm_gbs"] * 1e9) else "hbm",
+            }), flush=True)
+        del x, logits, W1, W3, W2, ws, out
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.steps < 1 or args.warmup < 0:
         raise SystemExit("--steps must be >= 1 and --warmup >= 0")
     if args.impl == "reference":

@@ -174,6 +174,33 @@ __host__ __device__ inline int n_items_for(int nb, int mgb) {
   return 2 + cdiv(nb - 2, mgb);
 }
 
+// One warp: exclusive scan in place of a[0..n), n <= 256 (8 values per lane);
+// returns the total.
+__device__ int warp_scan_smem(int* a, int n, int lane) {
+  int v[8];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int idx = lane * 8 + i;
+    v[i] = idx < n ? a[idx] : 0;
+    sum += v[i];
+  }
+  int inc = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += t;
+  }
+  int run = inc - sum;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int idx = lane * 8 + i;
+    if (idx < n) a[idx] = run;
+    run += v[i];
+  }
+  return __shfl_sync(0xffffffffu, inc, 31);
+}
+
 __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int32_t* offsets_in,
                                                     int T, int d, int f, int E, int k, int num_sms,
                                                     int consumer_hint, int mgb, int G, int join,
@@ -185,47 +212,37 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
   __shared__ int sorted[MAX_E];
   __shared__ int bstart[MAX_E + 1];
   __shared__ int gstart[MAX_E + 1];
-  __shared__ int nbands_s;
-  const int tid = threadIdx.x;
-  // counts and per-block bases (exclusive scan down each expert's column): the
-  // blocks are split into P contiguous parts per expert, each thread sums its part,
-  // the part sums are scanned in shared memory, then each thread writes its bases.
-  __shared__ int part_sum[1024];
-  const int P = max(1, (int)blockDim.x / E);
-  const int e_me = tid % E, p_me = tid / E;
-  const bool scanner = nblk > 0 && p_me < P;
-  const int per = nblk > 0 ? cdiv(nblk, P) : 0;
-  const int bl0 = min(nblk, p_me * per), bl1 = min(nblk, bl0 + per);
-  if (scanner) {
-    int run = 0;
-#pragma unroll 8
-    for (int b = bl0; b < bl1; ++b) run += w.blk_hist[(size_t)b * E + e_me];
-    part_sum[p_me * E + e_me] = run;
-  }
-  __syncthreads();
+  __shared__ int t1start[MAX_E + 1];
+  __shared__ int lane_base[MAX_E][32];
+  __shared__ int totals[3];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nwarps = blockDim.x >> 5;
+  // Counts and per-block scatter bases: warp w scans expert e = w, w + 32, ...
+  // over the blocks (lane i owns a contiguous chunk of blocks).
+  const int chunk = nblk > 0 ? cdiv(nblk, 32) : 0;
+  const int cb0 = min(nblk, lane * chunk), cb1 = min(nblk, cb0 + chunk);
   if (nblk > 0) {
-    for (int e = tid; e < E; e += blockDim.x) {
-      int run = 0;
-      for (int q = 0; q < P; ++q) { const int v = part_sum[q * E + e]; part_sum[q * E + e] = run; run += v; }
-      cnt[e] = run;
+    for (int e = warp; e < E; e += nwarps) {
+      int sum = 0;
+      for (int b = cb0; b < cb1; ++b) sum += w.blk_hist[(size_t)b * E + e];
+      int inc = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += t;
+      }
+      lane_base[e][lane] = inc - sum;
+      if (lane == 31) cnt[e] = inc;
     }
   } else {
     for (int e = tid; e < E; e += blockDim.x) cnt[e] = offsets_in[e + 1] - offsets_in[e];
   }
   __syncthreads();
-  if (scanner) {
-    int run = part_sum[p_me * E + e_me];
-    for (int b = bl0; b < bl1; ++b) {
-      const int hcount = w.blk_hist[(size_t)b * E + e_me];
-      w.blk_base[(size_t)b * E + e_me] = run;
-      run += hcount;
-    }
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int e = 0; e < E; ++e) { offs[e] = run; run += cnt[e]; }
-    offs[E] = run;
+  if (warp == 0) {
+    for (int e = lane; e < E; e += 32) offs[e] = cnt[e];
+    __syncwarp();
+    const int total = warp_scan_smem(offs, E, lane);
+    if (lane == 0) offs[E] = total;
   }
   __syncthreads();
   for (int e = tid; e <= E; e += blockDim.x) {
@@ -233,7 +250,14 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
     w.offsets[e] = offs[e];
   }
   if (nblk > 0) {
-    for (int i = tid; i < nblk * E; i += blockDim.x) w.blk_base[i] += offs[i % E];
+    for (int e = warp; e < E; e += nwarps) {
+      int run = offs[e] + lane_base[e][lane];
+      for (int b = cb0; b < cb1; ++b) {
+        const int hcount = w.blk_hist[(size_t)b * E + e];
+        w.blk_base[(size_t)b * E + e] = run;
+        run += hcount;
+      }
+    }
   }
   // expert priority: rows descending, id ascending (rank by comparison count)
   for (int e = tid; e < E; e += blockDim.x) {
@@ -243,31 +267,30 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
   }
   __syncthreads();
   const int NT1 = f / BN1, NT2 = d / BN2;
+  // bands, groups and GEMM1 tiles of the experts in priority order, prefix-summed
+  for (int s2 = tid; s2 < E; s2 += blockDim.x) {
+    const int bands = cdiv(cnt[sorted[s2]], BM);
+    const int groups = cdiv(bands, G);
+    bstart[s2] = bands;
+    gstart[s2] = groups;
+    t1start[s2] = groups * NT1;
+  }
+  __syncthreads();
+  if (warp < 3) {
+    int* arr = warp == 0 ? bstart : (warp == 1 ? gstart : t1start);
+    const int total = warp_scan_smem(arr, E, lane);
+    if (lane == 0) { arr[E] = total; totals[warp] = total; }
+  }
+  __syncthreads();
+  const int nb = totals[0], ng = totals[1], nt1 = totals[2];
+  if (w.bands) {
+    for (int s2 = tid; s2 <= E; s2 += blockDim.x) {
+      w.band_start[s2] = bstart[s2];
+      w.group_start[s2] = gstart[s2];
+      w.tile_start1[s2] = t1start[s2];
+    }
+  }
   if (tid == 0) {
-    int nb = 0, ng = 0, nt1 = 0;
-    for (int s = 0; s < E; ++s) {
-      const int e = sorted[s];
-      bstart[s] = nb;
-      gstart[s] = ng;
-      if (w.bands) {
-        w.band_start[s] = nb;
-        w.group_start[s] = ng;
-        w.tile_start1[s] = nt1;
-      }
-      const int bands = cdiv(cnt[e], BM);
-      const int groups = cdiv(bands, G);
-      nb += bands;
-      ng += groups;
-      nt1 += groups * NT1;
-    }
-    bstart[E] = nb;
-    gstart[E] = ng;
-    if (w.bands) {
-      w.band_start[E] = nb;
-      w.group_start[E] = ng;
-      w.tile_start1[E] = nt1;
-    }
-    nbands_s = nb;
     const long long R = offs[E];
     // without producers joining, at least one CTA group must consume from the start
     const int cmin = join ? 0 : G;
@@ -289,6 +312,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
     z.pad[0] = z.pad[1] = 0;
     *w.sync = z;
   }
+  const int nbands_s = nb;
   if (w.bands == nullptr) return;   // permutation only: no tile plan wanted
   for (int s = tid; s < E; s += blockDim.x) {
     w.sorted_e[s] = sorted[s];
