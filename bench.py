@@ -379,7 +379,7 @@ def run_ours(args):
                     "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
                     "d2h_bytes_per_step": out.numel() * 2,
                     "method": "pinned host buffers; double-buffered device buffers; H2D and D2H on their own streams, overlapping the neighbouring steps' compute"},
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": 6 * args.steps,   # route, plan, scatter, gather, persistent FFN, combine
             "clocks": clocks,
             "kernel_hash": h,
         }
