@@ -70,7 +70,8 @@ def parse():
     ap.add_argument("--consumer-sms", type=int, default=0, help="0 = cost model")
     ap.add_argument("--mgb", type=int, default=1)
     ap.add_argument("--no-join", action="store_true", help="producers do not join the combine")
-    ap.add_argument("--one-cta", action="store_true", help="128-row tiles on single CTAs instead of CTA pairs")
+    ap.add_argument("--one-cta", action="store_true", help="force 128-row tiles on single CTAs")
+    ap.add_argument("--cta-pair", action="store_true", help="force 256-row tiles on CTA pairs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -202,7 +203,8 @@ def run_ours(args):
     ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k, dev)
     out = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device=dev)
     kw = dict(consumer_sms=args.consumer_sms, mgb=args.mgb,
-              flags=(moe.SCHED_NO_JOIN if args.no_join else 0) | (moe.SCHED_ONE_CTA if args.one_cta else 0))
+              flags=(moe.SCHED_NO_JOIN if args.no_join else 0) | (moe.SCHED_ONE_CTA if args.one_cta else 0)
+              | (moe.SCHED_CTA_PAIR if args.cta_pair else 0))
 
     def step(mode, evb=None, eve=None):
         moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, mode, out=out, ev_begin=evb, ev_end=eve, **kw)
@@ -355,7 +357,8 @@ def run_ours(args):
             "data": "synthetic: seeded counter-based N(0,1) tokens and gate logits, random-init N(0,0.02) bf16 expert weights",
             "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "d_ff": wl.f, "E": wl.E,
                        "top_k": wl.k, "router": wl.router, "mode": "overlapped",
-                       "mma_tile": "128x256 per CTA" if args.one_cta else "256x256 per CTA pair (cta_group::2)",
+                       "mma_tile": ("128x256 per CTA" if args.one_cta else "256x256 per CTA pair (cta_group::2)"
+                                    if args.cta_pair or wl.R >= 512 * wl.E else "128x256 per CTA"),
                        "parallelism": f"replicas x{world} (token shards, no collective)",
                        "l2": "inputs larger than L2: active expert weights %.2f GB per step" % (B / 1e9)},
             "tflops": world * F / (t_ovl * 1e-3) / 1e12,

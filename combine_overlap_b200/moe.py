@@ -30,6 +30,7 @@ SCHED_NO_JOIN = 0x2
 SCHED_ONE_CTA = 0x4
 DBG_TIMESTAMPS = 0x8
 SCHED_GATHER_A = 0x10
+SCHED_CTA_PAIR = 0x20
 
 
 class MoEError(RuntimeError):

@@ -73,8 +73,12 @@ typedef enum {
 #define MOE_SCHED_GATHER_A     0x10u /* GEMM1 gathers its A rows from x with TMA gather4
                                         instead of reading a permuted copy (measured slower
                                         on B200: 32 gather instructions per k-block) */
-#define MOE_SCHED_ONE_CTA      0x4u  /* 128-row MMA tiles on single CTAs instead of
-                                        256-row tiles on CTA pairs (tcgen05 cta_group::2) */
+#define MOE_SCHED_ONE_CTA      0x4u  /* force 128-row MMA tiles on single CTAs          */
+#define MOE_SCHED_CTA_PAIR     0x20u /* force 256-row MMA tiles on CTA pairs (tcgen05
+                                        cta_group::2).  Without either flag the call picks
+                                        pairs when the average rows per expert, T*k/E, is at
+                                        least 512, else single CTAs (a pair tile wastes up to
+                                        255 masked rows per expert, a single one up to 127) */
 
 typedef struct {
   int T, d, f, E, k;        /* tokens, d_model, d_ff, experts, top-k                */

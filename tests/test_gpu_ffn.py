@@ -20,6 +20,7 @@ CASES = [
     synth.small("multi_band", 700, 256, 384, 3, 3),
     synth.small("empty_experts", 200, 256, 256, 32, 2, "zipf"),
     synth.WORKLOADS["tiny"],
+    synth.small("pair_tiles", 1100, 256, 256, 4, 2, "zipf"),   # T*k/E >= 512: CTA-pair tiles
 ]
 
 

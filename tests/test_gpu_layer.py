@@ -49,7 +49,8 @@ def test_layer_small(orc, wl):
     ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
     ref = orc.forward(gu.host(inp["x"]), gu.host(inp["logits"]), gu.host(inp["W1"]),
                       gu.host(inp["W3"]), gu.host(inp["W2"]), wl.k)
-    seq, extra, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL)
+    pair = moe.SCHED_CTA_PAIR
+    seq, extra, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL, flags=pair)
     assert np.array_equal(gu.host(extra["topk_idx"]), ref["topk_idx"])
     gu.assert_gates(gu.host(extra["topk_gate"]), ref["topk_gate"])
     assert np.array_equal(gu.host(extra["counts"]), ref["counts"])
@@ -60,7 +61,7 @@ def test_layer_small(orc, wl):
     for kw in (dict(), dict(consumer_sms=1), dict(consumer_sms=2), dict(consumer_sms=4),
                dict(consumer_sms=8), dict(consumer_sms=32), dict(mgb=2), dict(mgb=3, consumer_sms=3),
                dict(flags=moe.SCHED_NO_JOIN, consumer_sms=2)):
-        ovl, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, **kw)
+        ovl, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=pair | kw.pop("flags", 0), **kw)
         assert c >= 0 and c % 2 == 0      # whole CTA pairs (0: producers join at the end)
         assert np.array_equal(gu.host(ovl), seq_bits), f"overlapped {kw} differs from sequential"
     # the single-CTA (128-row tile) variant: same checks
@@ -72,9 +73,13 @@ def test_layer_small(orc, wl):
         assert np.array_equal(gu.host(ovl1), gu.host(seq1)), f"one-CTA overlapped {kw} differs"
     # GEMM1 reading its A rows with TMA gather4 from x instead of x_perm: same
     # arithmetic on the same rows, so the same bits, in both tile variants
-    for fl in (moe.SCHED_GATHER_A, moe.SCHED_GATHER_A | one):
+    # the default picks the variant from T*k/E; it must match one of the two
+    dflt, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED)
+    expect = seq_bits if wl.T * wl.k >= 512 * wl.E else gu.host(seq1)
+    assert np.array_equal(gu.host(dflt), expect)
+    for fl in (moe.SCHED_GATHER_A | pair, moe.SCHED_GATHER_A | one):
         gat, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=fl)
-        base = seq_bits if not fl & one else gu.host(seq1)
+        base = seq_bits if fl & pair else gu.host(seq1)
         assert np.array_equal(gu.host(gat), base), f"gathered A (flags {fl}) differs"
 
 
