@@ -71,6 +71,8 @@ def parse():
     ap.add_argument("--mgb", type=int, default=1)
     ap.add_argument("--no-join", action="store_true", help="producers do not join the combine")
     ap.add_argument("--one-cta", action="store_true", help="force 128-row tiles on single CTAs")
+    ap.add_argument("--b-per-atom", action="store_true",
+                    help="load weight tiles with one TMA copy per 64-column atom")
     ap.add_argument("--cta-pair", action="store_true", help="force 256-row tiles on CTA pairs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -204,7 +206,8 @@ def run_ours(args):
     out = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device=dev)
     kw = dict(consumer_sms=args.consumer_sms, mgb=args.mgb,
               flags=(moe.SCHED_NO_JOIN if args.no_join else 0) | (moe.SCHED_ONE_CTA if args.one_cta else 0)
-              | (moe.SCHED_CTA_PAIR if args.cta_pair else 0))
+              | (moe.SCHED_CTA_PAIR if args.cta_pair else 0)
+              | (moe.SCHED_B_PER_ATOM if args.b_per_atom else 0))
 
     def step(mode, evb=None, eve=None):
         moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, mode, out=out, ev_begin=evb, ev_end=eve, **kw)

@@ -6,6 +6,15 @@
 #include <stdint.h>
 #include <string.h>
 
+namespace moe {
+namespace {
+// The CUDA error behind the calling thread's latest MOE_ERR_CUDA.
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+}  // namespace
+void record_cuda_error(cudaError_t e) { g_last_cuda = e; }
+cudaError_t last_cuda_error() { return g_last_cuda; }
+}  // namespace moe
+
 namespace {
 
 using namespace moe;
@@ -129,6 +138,11 @@ inline bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
 
 int sms_cache[64] = {0};
 
+inline moe_status cuda_fail(cudaError_t e) {
+  moe::record_cuda_error(e);
+  return MOE_ERR_CUDA;
+}
+
 int device_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -152,7 +166,7 @@ CostModel default_cost_model() {
   return cm;
 }
 
-inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : cuda_fail(e); }
 
 // CTAs per MMA tile.  A CTA pair (256-row tiles, cta_group::2) streams a third less
 // operand data per FLOP, but every expert's last tile wastes up to 255 masked rows
@@ -167,7 +181,7 @@ int choose_group(int T, int E, int k, unsigned flags) {
 #define MOE_TRY(expr)                                   \
   do {                                                  \
     cudaError_t e_ = (expr);                            \
-    if (e_ != cudaSuccess) return MOE_ERR_CUDA;         \
+    if (e_ != cudaSuccess) return cuda_fail(e_);        \
   } while (0)
 
 }  // namespace
@@ -177,6 +191,12 @@ extern "C" {
 size_t moe_workspace_size(int T, int d, int f, int E, int k) {
   if (check_shape(T, d, f, E, k) != MOE_OK) return 0;
   return layout(T, d, f, E, k).total;
+}
+
+int moe_last_cuda_error(void) { return (int)moe::last_cuda_error(); }
+
+const char* moe_cuda_error_string(int code) {
+  return cudaGetErrorString(static_cast<cudaError_t>(code));
 }
 
 const char* moe_status_string(moe_status s) {
@@ -222,7 +242,7 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
   const Layout L = layout(T, BN2, BN1, E, k);
   if (!ws || !aligned16(ws) || ws_bytes < L.routing_end) return MOE_ERR_WORKSPACE;
   const int nsm = device_sms();
-  if (nsm <= 0) return MOE_ERR_CUDA;
+  if (nsm <= 0) return cuda_fail(cudaErrorInvalidDevice);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Work w = work_from(ws, L, false, false);
   if (counts) w.counts = counts;
@@ -249,8 +269,9 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
   const Layout L = layout(T, d, f, E, k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   const int G = choose_group(T, E, k, 0u);
-  const int grid = ffn_grid(G);
-  if (grid <= G) return MOE_ERR_CUDA;
+  int grid = 0;
+  MOE_TRY(ffn_grid(G, &grid));
+  if (grid <= G) return cuda_fail(cudaErrorInvalidConfiguration);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Work w = work_from(ws, L, true, true);
   MOE_TRY(launch_plan(w, 0, offsets, T, d, f, E, k, grid, 1, 1, G, 1, default_cost_model(), st));
@@ -277,7 +298,7 @@ moe_status moe_combine(const void* y, const int32_t* row_of, const float* topk_g
   if (k > MAX_K || d % 8 != 0) return MOE_ERR_UNSUPPORTED;
   if (!ok_ptr(y) || !ok_ptr(row_of) || !ok_ptr(topk_gate) || !ok_ptr(out)) return MOE_ERR_INVALID;
   const int nsm = device_sms();
-  if (nsm <= 0) return MOE_ERR_CUDA;
+  if (nsm <= 0) return cuda_fail(cudaErrorInvalidDevice);
   return cuda_status(launch_combine(static_cast<const __nv_bfloat16*>(y), row_of, topk_gate, T, d, k,
                                     static_cast<__nv_bfloat16*>(out), nsm,
                                     static_cast<cudaStream_t>(stream)));
@@ -299,8 +320,9 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   const int nsm = device_sms();
   const int G = choose_group(A.T, A.E, A.k, A.flags);
-  const int grid = ffn_grid(G);
-  if (nsm <= 1 || grid <= G) return MOE_ERR_CUDA;
+  int grid = 0;
+  MOE_TRY(ffn_grid(G, &grid));
+  if (nsm <= 1 || grid <= G) return cuda_fail(cudaErrorInvalidConfiguration);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Work w = work_from(ws, L, true, true);
   if (A.topk_idx) w.topk_idx = A.topk_idx;
@@ -360,24 +382,22 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
 
 moe_status moe_debug_band_stamps(void* ws, void* stream, uint64_t* host_out, int max_bands) {
   if (!ws || !aligned16(ws) || !host_out || max_bands < 1) return MOE_ERR_INVALID;
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  MOE_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
   const Layout L = layout(1, BN2, BN1, 1, 1);
   const int n = max_bands < STAMP_BANDS ? max_bands : STAMP_BANDS;
-  if (cudaMemcpy(host_out, static_cast<char*>(ws) + L.stamps + (size_t)STAMP_CTAS * NSTAMP * 8,
-                 (size_t)n * 4 * 8, cudaMemcpyDeviceToHost) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  MOE_TRY(cudaMemcpy(host_out, static_cast<char*>(ws) + L.stamps + (size_t)STAMP_CTAS * NSTAMP * 8,
+                     (size_t)n * 4 * 8, cudaMemcpyDeviceToHost));
   return MOE_OK;
 }
 
 moe_status moe_debug_stamps(void* ws, void* stream, uint64_t* host_out, int max_ctas, int* n_ctas) {
   if (!ws || !aligned16(ws) || !host_out || max_ctas < 1) return MOE_ERR_INVALID;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  MOE_TRY(cudaStreamSynchronize(st));
   const Layout L = layout(1, BN2, BN1, 1, 1);   // the stamps sit at a shape-independent offset
   const int n = max_ctas < STAMP_CTAS ? max_ctas : STAMP_CTAS;
-  if (cudaMemcpy(host_out, static_cast<char*>(ws) + L.stamps, (size_t)n * NSTAMP * 8,
-                 cudaMemcpyDeviceToHost) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  MOE_TRY(cudaMemcpy(host_out, static_cast<char*>(ws) + L.stamps, (size_t)n * NSTAMP * 8,
+                     cudaMemcpyDeviceToHost));
   if (n_ctas) {
     int g = 0;
     for (int i = 0; i < n; ++i) g += host_out[(size_t)i * NSTAMP] != 0;
@@ -389,9 +409,9 @@ moe_status moe_debug_stamps(void* ws, void* stream, uint64_t* host_out, int max_
 moe_status moe_get_status(void* ws, void* stream, int* consumer_sms, int* n_bands) {
   if (!ws || !aligned16(ws)) return MOE_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  MOE_TRY(cudaStreamSynchronize(st));
   Status h;
-  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  MOE_TRY(cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost));
   if (consumer_sms) *consumer_sms = h.consumer_sms;
   if (n_bands) *n_bands = h.n_bands;
   if (h.code == ST_TIMEOUT) return MOE_ERR_TIMEOUT;

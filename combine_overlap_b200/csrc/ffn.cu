@@ -187,19 +187,37 @@ __device__ __forceinline__ float silu_mul(float a, float b) {
   return __fdividef(a, 1.0f + __expf(-a)) * b;
 }
 
-// This CTA's rows of a row group (CTA `rank` of a G-CTA group owns band band0+rank).
+// A CTA pair's row group of one band only (an expert's last, odd band) runs as
+// a half tile: an M=128 cta_group::2 MMA, each CTA supplying 64 rows of A, at
+// half the tensor time of the M=256 tile whose second band would be all masked.
+// Its accumulator holds, in each CTA, 64 rows x N/2 columns twice: TMEM lanes
+// 0-63 the columns that the leader's B half supplies, lanes 64-127 (the same 64
+// rows) the peer's.  (The gathered-A path keeps full tiles, as does
+// MOE_SCHED_FULL_TILES.)
+template <int G>
+__device__ __forceinline__ bool half_tile(const Item& it, const FfnArgs& a) {
+  return G == 2 && !a.gather && !(a.flags & MOE_SCHED_FULL_TILES) && it.rows <= BM;
+}
+
+// This CTA's rows of a row group: CTA `rank` of a G-CTA group owns band
+// band0+rank; in a half tile, rows 64*rank.. of band0.
 struct MyRows {
   int row0, rows, band;
 };
 
 template <int G>
-__device__ __forceinline__ MyRows my_rows(const Item& it, uint32_t rank) {
+__device__ __forceinline__ MyRows my_rows(const Item& it, uint32_t rank, bool half) {
   MyRows m;
-  m.row0 = it.row0 + (int)rank * BM;
-  m.rows = min(BM, max(0, it.rows - (int)rank * BM));
-  m.band = it.band0 + (int)rank;
+  const int h = half ? BM / 2 : BM;
+  m.row0 = it.row0 + (int)rank * h;
+  m.rows = min(h, max(0, it.rows - (int)rank * h));
+  m.band = it.band0 + (half ? 0 : (int)rank);
   return m;
 }
+
+// Band counters: each tile adds 2 to its band's counter (1 from each CTA of a
+// half tile), so a band is complete at twice its tile count.
+constexpr uint32_t BAND_UNIT = 2;
 
 // Arrive on a barrier that lives in the pair leader (local when this CTA leads).
 template <int G>
@@ -277,11 +295,11 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
   };
   // Does this CTA gather indices for the item?  (GEMM1, gathered path, own rows)
   auto gathers = [&](const Item& it) {
-    return a.gather && it.kind == K_G1 && my_rows<G>(it, rank).rows > 0;
+    return a.gather && it.kind == K_G1 && my_rows<G>(it, rank, false).rows > 0;
   };
   auto fetch_indices = [&](const Item& it, int buf) {
     if (!gathers(it)) return;
-    const MyRows m = my_rows<G>(it, rank);
+    const MyRows m = my_rows<G>(it, rank, false);
     fence_proxy_async_shared();   // earlier generic reads of this buffer come first
     gpend |= 1u << buf;
     mbar_arrive_expect_tx(&ctl->gbar[buf], BM * 4);
@@ -298,7 +316,8 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
     fetch_indices(nxt, buf ^ 1);
     const bool is1 = cur.kind == K_G1;
     if (is1) ++n_g1; else ++n_g2;
-    const MyRows m = my_rows<G>(cur, rank);
+    const bool half = half_tile<G>(cur, a);
+    const MyRows m = my_rows<G>(cur, rank, half);
     const bool gat = a.gather && is1;
     if (gat && m.rows > 0) {
       if (!wait_bar(&ctl->gbar[buf], (gph >> buf) & 1u, tmo, abort)) { set_error(w.status, W_STAGE_FULL); break; }
@@ -307,7 +326,7 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
     }
     if (!is1 && m.rows > 0) {
       // GEMM2 reads this CTA's h rows: every GEMM1 column block of its band must be stored.
-      if (!wait_count(&w.band_done1[m.band], (uint32_t)NT1, tmo, abort)) {
+      if (!wait_count(&w.band_done1[m.band], BAND_UNIT * (uint32_t)NT1, tmo, abort)) {
         set_error(w.status, W_BAND1);
         break;
       }
@@ -334,8 +353,18 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
       } else {
         tma_load_2d_pair(sa, is1 ? tm_a1 : tm_a2, fbl, kb * BK, m.row0);
       }
-      // B
-      if (G == 1) {
+      // B: 64-column atoms of W1/W3 (GEMM1) or W2 (GEMM2), K-rows kb*BK.., each
+      // atom 64 K rows x 128 B, atom after atom (the MMA's leading-byte offset)
+      if (G == 1 && a.b_atoms) {
+        // 4-D maps {64 columns, K, atom, expert}: one copy per operand
+        const int k0 = kb * BK;
+        if (is1) {
+          tma_load_4d(sb, tm_w1, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
+          tma_load_4d(sb + 2 * B_BOX_BYTES, tm_w3, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
+        } else {
+          tma_load_4d(sb, tm_w2, fb, 0, k0, cur.nt * (BN2 / 64), cur.expert);
+        }
+      } else if (G == 1) {
         if (is1) {
           tma_load_3d(sb, tm_w1, fb, cur.nt * BN1, kb * BK, cur.expert);
           tma_load_3d(sb + B_BOX_BYTES, tm_w1, fb, cur.nt * BN1 + 64, kb * BK, cur.expert);
@@ -347,7 +376,14 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
             tma_load_3d(sb + q * B_BOX_BYTES, tm_w2, fb, cur.nt * BN2 + q * 64, kb * BK, cur.expert);
         }
       } else {
-        if (is1) {
+        if (is1 && half) {
+          // half tile: each CTA's B half is [W1 | W3] of one 64-column atom (the
+          // leader's the first, the peer's the second), so every accumulator
+          // lane holds matching W1 and W3 columns
+          const int n0 = cur.nt * BN1 + (int)rank * 64;
+          tma_load_3d_pair(sb, tm_w1, fbl, n0, kb * BK, cur.expert);
+          tma_load_3d_pair(sb + B_BOX_BYTES, tm_w3, fbl, n0, kb * BK, cur.expert);
+        } else if (is1) {
           // B columns [0,128) of the N=256 MMA come from the leader (W1), [128,256) from the peer (W3)
           const CUtensorMap* tw = rank == 0 ? tm_w1 : tm_w3;
           tma_load_3d_pair(sb, tw, fbl, cur.nt * BN1, kb * BK, cur.expert);
@@ -393,7 +429,8 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
                          const volatile uint32_t* abort) {
   using C = Cfg<G>;
   const uint64_t tmo = a.timeout_ns;
-  constexpr uint32_t idesc = idesc_bf16_f32(BM * G, 256, true);
+  constexpr uint32_t idesc_full = idesc_bf16_f32(BM * G, 256, true);
+  constexpr uint32_t idesc_half = idesc_bf16_f32(BM, 256, true);   // G == 2 only
   int stage = 0, slot = 0, acc = 0;
   uint32_t ph = 0, sph = 0, aph = 0;
   while (true) {
@@ -405,6 +442,7 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
     if (!wait_bar<G == 2>(&ctl->tempty[acc], aph ^ 1u, tmo, abort)) { set_error(a.w.status, W_TMEM_EMPTY); break; }
     tc_fence_after();
     const uint32_t dt = tmem_base + (uint32_t)(acc * ACC_COLS);
+    const uint32_t idesc = half_tile<G>(it, a) ? idesc_half : idesc_full;
     const int nk = (it.kind == K_G1 ? a.d : a.f) / BK;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
@@ -464,16 +502,24 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
     ok = __all_sync(0xffffffffu, wait_bar<G == 2>(&ctl->tfull[acc], aph, tmo, abort));
     if (!ok) { if (lane == 0) set_error(w.status, W_TMEM_FULL); break; }
     tc_fence_after();
-    const MyRows m = my_rows<G>(it, rank);
+    const bool half = half_tile<G>(it, a);
+    const MyRows m = my_rows<G>(it, rank, half);
     const uint32_t tb = tmem_base + (uint32_t)(acc * ACC_COLS) + ((uint32_t)(q * 32) << 16);
-    const bool valid = row < m.rows;
+    // full tile: lane `row` is row `row`, all N columns; half tile: lane `row` is
+    // row row % 64, and the N/2 columns of the B half row / 64 supplied
+    const int r = half ? (row & (BM / 2 - 1)) : row;
+    const int ch = half ? (row >> 6) : 0;
+    const bool valid = r < m.rows;
     if (it.kind == K_G1) {
-      uint4* dst = reinterpret_cast<uint4*>(a.h + (size_t)(m.row0 + row) * a.f + it.nt * BN1);
+      // h columns: full tile nt*128 + [0,128) from W1 columns [0,128) and W3
+      // columns [128,256); half tile nt*128 + 64*ch + [0,64) from [0,64) and [64,128)
+      const int nh = half ? BN1 / 2 : BN1;
+      uint4* dst = reinterpret_cast<uint4*>(a.h + (size_t)(m.row0 + r) * a.f + it.nt * BN1 + ch * (BN1 / 2));
 #pragma unroll 1
-      for (int c = 0; c < BN1 / 32; ++c) {
+      for (int c = 0; c < nh / 32; ++c) {
         uint32_t ra[32], rb[32];
         tmem_ld32(tb + c * 32, ra);
-        tmem_ld32(tb + BN1 + c * 32, rb);
+        tmem_ld32(tb + nh + c * 32, rb);
         tmem_ld_wait();
         uint32_t pk[16];
 #pragma unroll
@@ -488,15 +534,17 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
       }
       fence_proxy_async_global();   // h is read back by TMA in other CTAs
     } else {
-      uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)(m.row0 + row) * a.d + it.nt * BN2);
+      // y columns: full tile nt*256 + [0,256); half tile nt*256 + 128*ch + [0,128)
+      const int ny = half ? BN2 / 2 : BN2;
+      uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)(m.row0 + r) * a.d + it.nt * BN2 + ch * (BN2 / 2));
 #pragma unroll 1
-      for (int c = 0; c < BN2 / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tb + c * 32, r);
+      for (int c = 0; c < ny / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tb + c * 32, rr);
         tmem_ld_wait();
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
         if (valid) {
 #pragma unroll
           for (int v = 0; v < 4; ++v)
@@ -522,9 +570,11 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
       const bool stored = wait_bar(&ctl->epi_done[my_acc], (eph >> my_acc) & 1u, tmo, abort);
       const bool skip = (a.flags & MOE_DBG_SKIP_FLAG_BAND) && it.kind == K_G1 && m.band == 0;
       if (!stored) set_error(w.status, W_DRAIN);
-      else if (m.rows > 0 && !skip) {
+      else if ((half || m.rows > 0) && !skip) {
+        // a half tile's band is published by both CTAs (even one with no valid rows)
         __threadfence();
-        red_release_add(it.kind == K_G1 ? &w.band_done1[m.band] : &w.band_done2[m.band], 1u);
+        red_release_add(it.kind == K_G1 ? &w.band_done1[m.band] : &w.band_done2[m.band],
+                        half ? BAND_UNIT / 2 : BAND_UNIT);
       }
     }
     eph ^= 1u << my_acc;
@@ -597,7 +647,7 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
         int b0, b1;
         item_range(my_item, nb, a.mgb, b0, b1);
         bool ready = true;
-        for (int b = b0; b < b1 && ready; ++b) ready = ld_acquire(&w.band_done2[b]) >= NT2;
+        for (int b = b0; b < b1 && ready; ++b) ready = ld_acquire(&w.band_done2[b]) >= BAND_UNIT * NT2;
         if (ready) {
           act = C_BAND; arg0 = b0; arg1 = b1;
           my_item = -1;
@@ -878,6 +928,18 @@ static bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t*
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 weights as 4-D {64, K, atoms, E}: box 64 x 64 x `atoms` x 1, 128-B swizzle.
+static bool encode4(CUtensorMap* m, const void* base, const cuuint64_t* dims,
+                    const cuuint64_t* strides_bytes, cuuint32_t atoms) {
+  EncodeTiledFn fn = get_encode();
+  if (!fn) return false;
+  cuuint32_t box[4] = {64, 64, atoms, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides_bytes,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 constexpr int MAX_DEV = 64;
 int g_configured[2][MAX_DEV] = {{0}};
@@ -919,12 +981,15 @@ cudaError_t configure(int dev) {
 }
 }  // namespace
 
-int ffn_grid(int G) {
+cudaError_t ffn_grid(int G, int* grid) {
+  *grid = 0;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  const cudaError_t e = G == 2 ? configure<2>(dev) : configure<1>(dev);
-  if (e != cudaSuccess) return 0;
-  return g_grid[G - 1][dev];
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = G == 2 ? configure<2>(dev) : configure<1>(dev);
+  if (e != cudaSuccess) return e;
+  *grid = g_grid[G - 1][dev];
+  return cudaSuccess;
 }
 
 cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
@@ -944,17 +1009,29 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
     if (!encode(&tm_a1, a.x_perm, 2, dims, st, BM)) return cudaErrorInvalidValue;
   }
   {
-    const cuuint64_t dims[3] = {f, d, E}, st[2] = {f * 2, d * f * 2};
-    if (!encode(&tm_w1, a.W1, 3, dims, st, 64)) return cudaErrorInvalidValue;
-    if (!encode(&tm_w3, a.W3, 3, dims, st, 64)) return cudaErrorInvalidValue;
-  }
-  {
     const cuuint64_t dims[2] = {f, R}, st[1] = {f * 2};
     if (!encode(&tm_a2, a.h, 2, dims, st, BM)) return cudaErrorInvalidValue;
   }
-  {
-    const cuuint64_t dims[3] = {d, f, E}, st[2] = {d * 2, f * d * 2};
-    if (!encode(&tm_w2, a.W2, 3, dims, st, 64)) return cudaErrorInvalidValue;
+  // Single CTAs read the weights through 4-D maps {64 columns, K, 64-column
+  // atom, expert} with the atom stride 128 B, so that one box holds all the
+  // atoms of the CTA's tile, atom after atom: 2-3 copies per k-block instead of
+  // 5 (measured faster).  CTA pairs take 2 atoms per CTA and per operand through
+  // the 3-D maps {columns, K, expert}, one box per atom (a 4-D copy there
+  // measured slower), as do single CTAs if the driver refuses the 4-D maps.
+  FfnArgs args = a;
+  args.b_atoms = 0;
+  if (a.G == 1 && !(a.flags & MOE_SCHED_B_PER_ATOM)) {
+    const cuuint64_t d1[4] = {64, d, f / 64, E}, s1[3] = {f * 2, 128, d * f * 2};
+    const cuuint64_t d2[4] = {64, f, d / 64, E}, s2[3] = {d * 2, 128, f * d * 2};
+    args.b_atoms = encode4(&tm_w1, a.W1, d1, s1, 2) && encode4(&tm_w3, a.W3, d1, s1, 2) &&
+                   encode4(&tm_w2, a.W2, d2, s2, 4);
+  }
+  if (!args.b_atoms) {
+    const cuuint64_t dims[3] = {f, d, E}, st[2] = {f * 2, d * f * 2};
+    if (!encode(&tm_w1, a.W1, 3, dims, st, 64)) return cudaErrorInvalidValue;
+    if (!encode(&tm_w3, a.W3, 3, dims, st, 64)) return cudaErrorInvalidValue;
+    const cuuint64_t dims2[3] = {d, f, E}, st2[2] = {d * 2, f * d * 2};
+    if (!encode(&tm_w2, a.W2, 3, dims2, st2, 64)) return cudaErrorInvalidValue;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
@@ -977,8 +1054,8 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
     cfg.numAttrs = 1;
   }
   cfg.attrs = attr;
-  if (a.G == 2) return cudaLaunchKernelEx(&cfg, ffn_kernel<2>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, a);
-  return cudaLaunchKernelEx(&cfg, ffn_kernel<1>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, a);
+  if (a.G == 2) return cudaLaunchKernelEx(&cfg, ffn_kernel<2>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+  return cudaLaunchKernelEx(&cfg, ffn_kernel<1>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
 }
 
 }  // namespace moe

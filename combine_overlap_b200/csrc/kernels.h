@@ -74,14 +74,19 @@ struct FfnArgs {
   int phase;                     // PH_* bits
   int join;                      // producers join the combine when the tile queue drains
   int mgb;
+  int b_atoms;                   // single CTA: weight maps are 4-D, one box carries all 64-column atoms
   uint32_t flags;
   uint64_t timeout_ns;
 };
 
 size_t ffn_smem_bytes();
-// CTAs the persistent kernel runs with for group size G (0 on error); also sets
-// the kernel's shared-memory attribute for the current device.
-int ffn_grid(int G);
+// CTAs the persistent kernel runs with for group size G; also sets the kernel's
+// shared-memory attribute for the current device.
+cudaError_t ffn_grid(int G, int* grid);
+
+// The CUDA error behind the calling thread's latest MOE_ERR_CUDA (api.cu).
+void record_cuda_error(cudaError_t e);
+cudaError_t last_cuda_error();
 cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s);
 
 }  // namespace moe

@@ -61,6 +61,11 @@ cudaError_t scratch_address(void** out) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+inline moe_status fail(cudaError_t e) {
+  record_cuda_error(e);
+  return MOE_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" size_t moe_permute_noalloc_scratch_bytes(void) { return PERMUTE_NOALLOC_SCRATCH_BYTES; }
@@ -78,7 +83,7 @@ extern "C" moe_status moe_permute_noalloc(const void* x, int T, int d, int E, in
   if (counts && !aligned16(counts)) return MOE_ERR_INVALID;
 
   void* base = nullptr;
-  if (scratch_address(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  if (const cudaError_t e = scratch_address(&base); e != cudaSuccess) return fail(e);
   char* s = static_cast<char*>(base);
   const int nblk = route_blocks(T);
   Work w;
@@ -95,22 +100,22 @@ extern "C" moe_status moe_permute_noalloc(const void* x, int T, int d, int E, in
   // Nothing in the scratch has to start at zero: the histogram kernel writes
   // every block's counts, the plan kernel writes the bases, counts and status.
   int nsm = 0, dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (const cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return fail(e);
+  if (const cudaError_t e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+      e != cudaSuccess)
+    return fail(e);
   CostModel cm;
   cm.mma_flops_per_sm = 1.0f;
   cm.copy_bytes_per_sm = 1.0f;
   cm.hbm_bytes = 1.0f;
   cm.max_consumers = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (launch_hist(topk_idx, T, E, k, w.blk_hist, st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, cm, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, nullptr, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (launch_gather(static_cast<const __nv_bfloat16*>(x), perm, T * k, d, k,
-                    static_cast<__nv_bfloat16*>(x_perm), nsm, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  cudaError_t e = launch_hist(topk_idx, T, E, k, w.blk_hist, st);
+  if (e == cudaSuccess) e = launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, cm, st);
+  if (e == cudaSuccess) e = launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, nullptr, st);
+  if (e == cudaSuccess)
+    e = launch_gather(static_cast<const __nv_bfloat16*>(x), perm, T * k, d, k,
+                      static_cast<__nv_bfloat16*>(x_perm), nsm, st);
+  if (e != cudaSuccess) return fail(e);
   return MOE_OK;
 }

@@ -31,12 +31,17 @@ SCHED_ONE_CTA = 0x4
 DBG_TIMESTAMPS = 0x8
 SCHED_GATHER_A = 0x10
 SCHED_CTA_PAIR = 0x20
+SCHED_B_PER_ATOM = 0x40
+SCHED_FULL_TILES = 0x80
 
 
 class MoEError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
-        super().__init__(f"{what}: {status_string(code)} (code {code})")
+        self.cuda_error = last_cuda_error() if code == MOE_ERR_CUDA else 0
+        detail = f"; {cuda_error_string(self.cuda_error)} (cudaError {self.cuda_error})" \
+            if self.cuda_error else ""
+        super().__init__(f"{what}: {status_string(code)} (code {code}){detail}")
 
 
 class LayerArgs(ctypes.Structure):
@@ -66,6 +71,9 @@ _lib.moe_get_status.argtypes = [_P, _P, ctypes.POINTER(_I), ctypes.POINTER(_I)]
 _lib.moe_status_string.argtypes = [_I]
 _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_num_sms.restype = _I
+_lib.moe_last_cuda_error.restype = _I
+_lib.moe_cuda_error_string.argtypes = [_I]
+_lib.moe_cuda_error_string.restype = ctypes.c_char_p
 _lib.moe_debug_stamps.argtypes = [_P, _P, _P, _I, ctypes.POINTER(_I)]
 _lib.moe_debug_stamps.restype = _I
 _lib.moe_debug_band_stamps.argtypes = [_P, _P, _P, _I]
@@ -87,6 +95,15 @@ def declared_symbols() -> list[str]:
 
 def status_string(code: int) -> str:
     return _lib.moe_status_string(int(code)).decode()
+
+
+def last_cuda_error() -> int:
+    """The cudaError_t value behind this thread's latest MOE_ERR_CUDA (0: none)."""
+    return int(_lib.moe_last_cuda_error())
+
+
+def cuda_error_string(code: int) -> str:
+    return _lib.moe_cuda_error_string(int(code)).decode()
 
 
 def _check(code: int, what: str):

@@ -79,6 +79,13 @@ typedef enum {
                                         pairs when the average rows per expert, T*k/E, is at
                                         least 512, else single CTAs (a pair tile wastes up to
                                         255 masked rows per expert, a single one up to 127) */
+#define MOE_SCHED_B_PER_ATOM   0x40u /* single-CTA tiles load each 64-column atom of the
+                                        weight tiles with a TMA copy of its own (3-D maps),
+                                        as CTA pairs always do, instead of one 4-D copy
+                                        carrying all the atoms of the tile */
+#define MOE_SCHED_FULL_TILES   0x80u /* CTA pairs run an expert's odd last row band as a
+                                        full 256-row tile (half of it masked) instead of a
+                                        128-row half tile (M=128 cta_group::2 MMA) */
 
 typedef struct {
   int T, d, f, E, k;        /* tokens, d_model, d_ff, experts, top-k                */
@@ -198,6 +205,15 @@ moe_status moe_debug_band_stamps(void* ws, void* stream, uint64_t* host_out, int
 
 /* Static English description of a status code. */
 const char* moe_status_string(moe_status s);
+
+/* The cudaError_t value behind the calling thread's most recent MOE_ERR_CUDA
+ * from any entry point (a launch refused, a device fault surfacing at a launch
+ * or synchronisation, a failed copy); 0 (cudaSuccess) if none so far.  Not
+ * cleared by later successful calls. */
+int moe_last_cuda_error(void);
+
+/* Static description of a cudaError_t value (from moe_last_cuda_error). */
+const char* moe_cuda_error_string(int code);
 
 /* The number of SMs the persistent kernels use on the current device (a host
  * query, cached per device). */

@@ -38,6 +38,15 @@ def test_workspace_size_rules():
 def test_status_strings():
     for c in range(6):
         assert moe.status_string(c)
+
+
+def test_cuda_error_reporting():
+    assert isinstance(moe.last_cuda_error(), int)
+    assert moe.cuda_error_string(0) == "no error"
+    assert "illegal instruction" in moe.cuda_error_string(715)
+    # host-side rejections are not CUDA errors: no CUDA detail is attached to them
+    err = moe.MoEError(moe.MOE_ERR_INVALID, "call")
+    assert err.cuda_error == 0 and "invalid argument" in str(err) and "cudaError" not in str(err)
     assert moe.status_string(4).startswith("a bounded device wait")
 
 

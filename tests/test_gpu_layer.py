@@ -71,16 +71,20 @@ def test_layer_small(orc, wl):
     for kw in (dict(), dict(consumer_sms=1), dict(consumer_sms=5, mgb=2)):
         ovl1, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=one | kw.pop("flags", 0), **kw)
         assert np.array_equal(gu.host(ovl1), gu.host(seq1)), f"one-CTA overlapped {kw} differs"
-    # GEMM1 reading its A rows with TMA gather4 from x instead of x_perm: same
-    # arithmetic on the same rows, so the same bits, in both tile variants
     # the default picks the variant from T*k/E; it must match one of the two
     dflt, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED)
     expect = seq_bits if wl.T * wl.k >= 512 * wl.E else gu.host(seq1)
     assert np.array_equal(gu.host(dflt), expect)
-    for fl in (moe.SCHED_GATHER_A | pair, moe.SCHED_GATHER_A | one):
+    # GEMM1 reading its A rows with TMA gather4 from x instead of x_perm: same
+    # arithmetic on the same rows, so the same bits, in both tile variants;
+    # and single CTAs loading the weight tiles one 64-column atom per copy (3-D
+    # maps) instead of one 4-D copy per operand: the same bytes in the same places
+    # and CTA pairs running an expert's odd last band as a full 256-row tile
+    for fl in (moe.SCHED_GATHER_A | pair, moe.SCHED_GATHER_A | one, moe.SCHED_B_PER_ATOM | one,
+               moe.SCHED_FULL_TILES | pair):
         gat, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=fl)
         base = seq_bits if fl & pair else gu.host(seq1)
-        assert np.array_equal(gu.host(gat), base), f"gathered A (flags {fl}) differs"
+        assert np.array_equal(gu.host(gat), base), f"flags {fl:#x} differ"
 
 
 def test_layer_repeat_bitwise():
