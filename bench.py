@@ -38,13 +38,14 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the persistent FFN kernel, keyed by workload, valid only for the kernel sources
 # whose hash is recorded with it (see profiles/).
-TRAFFIC = {}
+TRAFFIC = {"mixtral": {"bytes": 3793449000 + 318090240, "kernel_hash": "c89cc0a7cfc6"}}
 
 
 def kernel_source_hash() -> str:
     h = hashlib.sha1()
     for rel in ("combine_overlap_b200/csrc/ffn.cu", "combine_overlap_b200/csrc/common.cuh",
-                "combine_overlap_b200/csrc/combine.cuh"):
+                "combine_overlap_b200/csrc/combine.cuh", "combine_overlap_b200/csrc/kernels.h",
+                "combine_overlap_b200/csrc/api.cu"):
         with open(os.path.join(ROOT, rel), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:12]
@@ -360,8 +361,10 @@ def run_ours(args):
             "data": "synthetic: seeded counter-based N(0,1) tokens and gate logits, random-init N(0,0.02) bf16 expert weights",
             "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "d_ff": wl.f, "E": wl.E,
                        "top_k": wl.k, "router": wl.router, "mode": "overlapped",
-                       "mma_tile": ("128x256 per CTA" if args.one_cta else "256x256 per CTA pair (cta_group::2)"
-                                    if args.cta_pair or wl.R >= 512 * wl.E else "128x256 per CTA"),
+                       "mma_tile": ("256x256 per CTA pair (cta_group::2)"
+                                    if not args.one_cta and (args.cta_pair or (
+                                        wl.R >= 512 * wl.E and wl.f >= 8192))
+                                    else "128x256 per CTA"),
                        "parallelism": f"replicas x{world} (token shards, no collective)",
                        "l2": "inputs larger than L2: active expert weights %.2f GB per step" % (B / 1e9)},
             "tflops": world * F / (t_ovl * 1e-3) / 1e12,

@@ -168,14 +168,18 @@ CostModel default_cost_model() {
 
 inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : cuda_fail(e); }
 
-// CTAs per MMA tile.  A CTA pair (256-row tiles, cta_group::2) streams a third less
-// operand data per FLOP, but every expert's last tile wastes up to 255 masked rows
-// instead of 127: with few rows per expert (T*k/E < 512) the single-CTA tiles win
-// (measured on B200: 18 % faster at 64 rows per expert, 8 % at 256).
-int choose_group(int T, int E, int k, unsigned flags) {
+// CTAs per MMA tile.  A CTA pair (256-row tiles, cta_group::2) streams a third
+// less operand data per FLOP than a single CTA (128-row tiles, whose weight tiles
+// come in one 4-D TMA copy per operand), but each pair tile carries more fixed
+// cost and, below 512 rows per expert, more masked rows.  Measured on B200, one
+// variant per process (alternating the two kernels step by step penalises the
+// pair): pairs are 2 % faster at d_ff = 14336 with 1024-2048 rows per expert,
+// even at d_ff = 4096-8192, and 3-14 % slower at d_ff <= 2048 or below 512 rows
+// per expert.  So pairs are picked when T*k/E >= 512 and d_ff >= 8192.
+int choose_group(int T, int f, int E, int k, unsigned flags) {
   if (flags & MOE_SCHED_ONE_CTA) return 1;
   if (flags & MOE_SCHED_CTA_PAIR) return 2;
-  return (long long)T * k >= 512LL * E ? 2 : 1;
+  return (long long)T * k >= 512LL * E && f >= 8192 ? 2 : 1;
 }
 
 #define MOE_TRY(expr)                                   \
@@ -260,15 +264,18 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
 
 moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, int d, int f, int E,
                            int k, const void* W1, const void* W3, const void* W2, void* h, void* y,
-                           void* ws, size_t ws_bytes, void* stream) {
+                           unsigned flags, void* ws, size_t ws_bytes, void* stream) {
   moe_status s = check_shape(T, d, f, E, k);
   if (s != MOE_OK) return s;
   if (!ok_ptr(x_perm) || !ok_ptr(offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
       !ok_ptr(y) || !ok_opt(h))
     return MOE_ERR_INVALID;
+  constexpr unsigned tile_flags =
+      MOE_SCHED_ONE_CTA | MOE_SCHED_CTA_PAIR | MOE_SCHED_B_PER_ATOM | MOE_SCHED_FULL_TILES;
+  if (flags & ~tile_flags) return MOE_ERR_INVALID;
   const Layout L = layout(T, d, f, E, k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  const int G = choose_group(T, E, k, 0u);
+  const int G = choose_group(T, f, E, k, flags);
   int grid = 0;
   MOE_TRY(ffn_grid(G, &grid));
   if (grid <= G) return cuda_fail(cudaErrorInvalidConfiguration);
@@ -287,6 +294,7 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
   a.phase = PH_G1 | PH_G2;
   a.join = 0;
   a.mgb = 1;
+  a.flags = flags;
   a.timeout_ns = 2000000000ull;
   MOE_TRY(launch_ffn(a, grid, st));
   return MOE_OK;
@@ -319,7 +327,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   const Layout L = layout(A.T, A.d, A.f, A.E, A.k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   const int nsm = device_sms();
-  const int G = choose_group(A.T, A.E, A.k, A.flags);
+  const int G = choose_group(A.T, A.f, A.E, A.k, A.flags);
   int grid = 0;
   MOE_TRY(ffn_grid(G, &grid));
   if (nsm <= 1 || grid <= G) return cuda_fail(cudaErrorInvalidConfiguration);

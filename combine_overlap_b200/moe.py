@@ -64,7 +64,8 @@ _lib.moe_workspace_size.argtypes = [_I, _I, _I, _I, _I]
 _lib.moe_workspace_size.restype = _S
 _lib.moe_route.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P, _S, _P]
 _lib.moe_permute.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _S, _P]
-_lib.moe_grouped_ffn.argtypes = [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P]
+_lib.moe_grouped_ffn.argtypes = [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_uint,
+                                 _P, _S, _P]
 _lib.moe_combine.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.moe_layer_forward.argtypes = [ctypes.POINTER(LayerArgs), _I, _P, _S, _P]
 _lib.moe_get_status.argtypes = [_P, _P, ctypes.POINTER(_I), ctypes.POINTER(_I)]
@@ -192,8 +193,9 @@ def permute_noalloc(x: torch.Tensor, topk_idx: torch.Tensor, E: int):
 
 
 def grouped_ffn(x_perm: torch.Tensor, offsets: torch.Tensor, W1, W3, W2, T: int, k: int,
-                ws: torch.Tensor, want_h: bool = True):
-    """x_perm: [T*k][d] bf16 (rows past offsets[E] unused)."""
+                ws: torch.Tensor, want_h: bool = True, flags: int = 0):
+    """x_perm: [T*k][d] bf16 (rows past offsets[E] unused); flags: SCHED_ONE_CTA,
+    SCHED_CTA_PAIR, SCHED_B_PER_ATOM, SCHED_FULL_TILES."""
     _need(x_perm, torch.bfloat16, "x_perm")
     _need(offsets, torch.int32, "offsets")
     for n, w in (("W1", W1), ("W3", W3), ("W2", W2)):
@@ -203,7 +205,8 @@ def grouped_ffn(x_perm: torch.Tensor, offsets: torch.Tensor, W1, W3, W2, T: int,
     y = torch.empty((T * k, d), dtype=torch.bfloat16, device=dev)
     h = torch.empty((T * k, f), dtype=torch.bfloat16, device=dev) if want_h else None
     _check(_lib.moe_grouped_ffn(_ptr(x_perm), _ptr(offsets), T, d, f, E, k, _ptr(W1), _ptr(W3),
-                                _ptr(W2), _ptr(h), _ptr(y), _ptr(ws), ws.numel(), _stream()),
+                                _ptr(W2), _ptr(h), _ptr(y), int(flags), _ptr(ws), ws.numel(),
+                                _stream()),
            "moe_grouped_ffn")
     return h, y
 

@@ -75,10 +75,11 @@ typedef enum {
                                         on B200: 32 gather instructions per k-block) */
 #define MOE_SCHED_ONE_CTA      0x4u  /* force 128-row MMA tiles on single CTAs          */
 #define MOE_SCHED_CTA_PAIR     0x20u /* force 256-row MMA tiles on CTA pairs (tcgen05
-                                        cta_group::2).  Without either flag the call picks
-                                        pairs when the average rows per expert, T*k/E, is at
-                                        least 512, else single CTAs (a pair tile wastes up to
-                                        255 masked rows per expert, a single one up to 127) */
+                                        cta_group::2); an expert's odd last row band runs
+                                        as a 128-row half tile.  Without either flag the
+                                        call picks pairs when T*k/E >= 512 and f >= 8192,
+                                        else single CTAs (measured on B200).  ONE_CTA
+                                        wins if both are set */
 #define MOE_SCHED_B_PER_ATOM   0x40u /* single-CTA tiles load each 64-column atom of the
                                         weight tiles with a TMA copy of its own (3-D maps),
                                         as CTA pairs always do, instead of one 4-D copy
@@ -102,7 +103,7 @@ typedef struct {
   int32_t* offsets;         /* [E+1] exclusive prefix sum of counts                 */
   int32_t* perm;            /* [T*k] routed row r -> source slot p = t*k + j        */
   int consumer_sms;         /* overlapped mode: 0 = cost model; > 0 = this many (rounded
-                               up to whole CTA pairs unless MOE_SCHED_ONE_CTA)       */
+                               up to whole CTA pairs under MOE_SCHED_CTA_PAIR)       */
   int mgb;                  /* row bands per consumer item (paper's x), >= 1; 0 = 1 */
   unsigned flags;           /* MOE_DBG_* / MOE_SCHED_* bits                         */
   int timeout_us;           /* bound on each device wait; 0 = default (2 s)         */
@@ -145,10 +146,13 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
  *   h[r] = bf16(silu(x_perm[r] W1_e) * (x_perm[r] W3_e)),  y[r] = bf16(h[r] W2_e)
  * (fp32 accumulation).  x_perm [R][d], y [R][d] bf16, R = offsets[E] <= T*k;
  * h [R][f] bf16 is written to the caller's buffer if non-NULL, else kept in the
- * workspace. */
+ * workspace.  flags: 0, or MOE_SCHED_ONE_CTA / MOE_SCHED_CTA_PAIR /
+ * MOE_SCHED_B_PER_ATOM / MOE_SCHED_FULL_TILES (tile variant); any other bit is
+ * MOE_ERR_INVALID. */
 moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, int d, int f,
                            int E, int k, const void* W1, const void* W3, const void* W2,
-                           void* h, void* y, void* ws, size_t ws_bytes, void* stream);
+                           void* h, void* y, unsigned flags, void* ws, size_t ws_bytes,
+                           void* stream);
 
 /* Step (d) alone, the weighted reduction (paper Section 2.1, "Weighted reduction
  * (scale)"): out[t] = bf16( sum_{j<k} g[t][j] * y[row_of[t*k+j]] ), fp32 in slot

@@ -2,8 +2,8 @@
 
 * Small layers, every element: GPU vs the oracle within 2e-2 * max|ref|; routing
   outputs bit-exact (including layers whose tokens fill 3, 1 or none of the
-  consumer's staging slots), for both the CTA-pair (default) and the single-CTA
-  tile variants; the overlapped mode bit-identical to the sequential mode
+  consumer's staging slots), for both the CTA-pair and the single-CTA tile
+  variants; the overlapped mode bit-identical to the sequential mode
   for every consumer-SM count tried (cost model, 1, 2, 4, 8, 32), segment size
   mgb in {1, 2, 3} and with or without producers joining the combine.
 * Every benchmark workload at full size, in the configuration the benchmark
@@ -71,9 +71,9 @@ def test_layer_small(orc, wl):
     for kw in (dict(), dict(consumer_sms=1), dict(consumer_sms=5, mgb=2)):
         ovl1, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=one | kw.pop("flags", 0), **kw)
         assert np.array_equal(gu.host(ovl1), gu.host(seq1)), f"one-CTA overlapped {kw} differs"
-    # the default picks the variant from T*k/E; it must match one of the two
+    # the default picks pairs when T*k/E >= 512 and d_ff >= 8192, else single CTAs
     dflt, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED)
-    expect = seq_bits if wl.T * wl.k >= 512 * wl.E else gu.host(seq1)
+    expect = seq_bits if wl.T * wl.k >= 512 * wl.E and wl.f >= 8192 else gu.host(seq1)
     assert np.array_equal(gu.host(dflt), expect)
     # GEMM1 reading its A rows with TMA gather4 from x instead of x_perm: same
     # arithmetic on the same rows, so the same bits, in both tile variants;
@@ -100,17 +100,22 @@ def test_layer_repeat_bitwise():
 
 FULL = ["mixtral", "fine_grained", "imbalanced", "sweep_T512_hot", "sweep_T2048_uniform",
         "sweep_T8192_zipf", "sweep_T32768_uniform"]
+# (workload, flags): every layer in its default variant (CTA pairs on the
+# Mixtral-shaped layer, single CTAs elsewhere), and the other variant on two
+FULL_CASES = [(n, 0) for n in FULL] + [("mixtral", 0x4), ("fine_grained", 0x20)]
 
 
-@pytest.mark.parametrize("name", FULL)
-def test_layer_full_size_sampled(orc, name):
+@pytest.mark.parametrize("name,flags", FULL_CASES,
+                         ids=[f"{n}-{ {0: 'default', 0x4: 'one', 0x20: 'pair'}[f]}" for n, f in FULL_CASES])
+def test_layer_full_size_sampled(orc, name, flags):
+    assert flags in (0, moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR)
     wl = synth.WORKLOADS[name]
     orc.set_threads(os.cpu_count() or 1)
     inp = gu.inputs(wl)
     ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
-    ovl, extra, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED)
+    ovl, extra, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=flags)
     ovl_bits = gu.host(ovl)
-    seq, _, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL)
+    seq, _, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL, flags=flags)
     assert np.array_equal(gu.host(seq), ovl_bits), "overlapped differs from sequential"
     # routing in full
     oidx, ogate = orc.route(gu.host(inp["logits"]), wl.k)
