@@ -13,6 +13,10 @@ job value is N*T tokens over the slowest rank's time (weak scaling).
 
 --impl reference times the CPU oracle (plain C++) on the host cores, a bounded
 token sample per step; it is a deliberately slow baseline, not a target.
+
+Besides the benchmark line: --sweep times every cell of the d=4096/E=32 grid
+(overlapped vs sequential per consumer-SM setting), and --oracle-timings times
+the CPU oracle on each configuration; each prints one JSON line per case.
 """
 from __future__ import annotations
 
@@ -38,7 +42,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the persistent FFN kernel, keyed by workload, valid only for the kernel sources
 # whose hash is recorded with it (see profiles/).
-TRAFFIC = {"mixtral": {"bytes": 3793449000 + 318090240, "kernel_hash": "c89cc0a7cfc6"}}
+TRAFFIC = {"mixtral": {"bytes": 3837271000 + 320849152, "kernel_hash": "c7290ca38ba9"}}
 
 
 def kernel_source_hash() -> str:
@@ -81,6 +85,9 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="d=4096/E=32/top-4 sweep: T x router x consumer SMs, overlapped vs "
                          "sequential; one JSON line per cell (not the benchmark line)")
+    ap.add_argument("--oracle-timings", action="store_true",
+                    help="time the CPU oracle on each benchmark configuration; one JSON line "
+                         "per configuration (not the benchmark line)")
     return ap.parse_args()
 
 
@@ -228,10 +235,10 @@ def run_ours(args):
     counts = moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, moe.MODE_OVERLAPPED, outputs=True,
                                **kw)[1]["counts"].cpu().tolist()
 
-    def timed(mode, clocks=False):
+    def timed(mode, clocks=False, hooks=False):
         K = args.steps
-        evb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        eve = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        evb = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if hooks else [None] * K
+        eve = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if hooks else [None] * K
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
@@ -244,11 +251,16 @@ def run_ours(args):
         barrier()
         c = clk.stop() if clk else None
         total = e0.elapsed_time(e1) / K
-        ffn = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / K
+        ffn = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / K if hooks else None
         return total, ffn, c
 
-    # the contract's timed region: K overlapped steps (clocks sampled meanwhile)
-    t_ovl, ffn_ovl, clocks = timed(moe.MODE_OVERLAPPED, clocks=True)
+    # The contract's timed region: K overlapped steps, clocks sampled meanwhile.
+    # It runs without the library's timing hooks: a recorded event between two
+    # launches costs them their programmatic overlap.
+    t_ovl, _, clocks = timed(moe.MODE_OVERLAPPED, clocks=True)
+    # The persistent FFN kernel's average launch duration, from K more overlapped
+    # steps with the hooks (events recorded on the launching stream around it).
+    t_ovl_hooked, ffn_ovl, _ = timed(moe.MODE_OVERLAPPED, hooks=True)
     # overlapped vs sequential: the two modes alternate step by step (paired
     # samples under the same clock and power state), each step timed with events
     # on the stream; medians per mode
@@ -268,10 +280,33 @@ def run_ours(args):
     barrier()
     step_ms = {m: [e0.elapsed_time(e1) for e0, e1, _, _ in ev[m]] for m in ev}
     ffn_ms = {m: [fb.elapsed_time(fe) for _, _, fb, fe in ev[m]] for m in ev}
+    # the combine after the expert FFN: the full pass (sequential) or the remainder
+    # pass (overlapped)
+    post_ms = {m: [fe.elapsed_time(e1) for _, e1, _, fe in ev[m]] for m in ev}
     t_seq = statistics.median(step_ms["seq"])
     ffn_seq = statistics.median(ffn_ms["seq"])
     t_ovl_med = statistics.median(step_ms["ovl"])
     ffn_ovl_med = statistics.median(ffn_ms["ovl"])
+    post_seq = statistics.median(post_ms["seq"])
+    post_ovl = statistics.median(post_ms["ovl"])
+
+    # The same overlapped call captured once in a CUDA graph and replayed K times.
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(moe.MODE_OVERLAPPED)
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_graph = e0.elapsed_time(e1) / args.steps
+    del g
 
     # End to end through the public call: every step copies its inputs (x, logits)
     # from pinned host memory and reads its output back to pinned host memory.
@@ -328,8 +363,10 @@ def run_ours(args):
     if code != moe.MOE_OK:
         raise RuntimeError(f"timed runs: {moe.status_string(code)}")
 
-    t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med = max_over_ranks(
-        [t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med], world, dev)
+    (t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med, post_seq, post_ovl,
+     t_graph, t_ovl_hooked) = max_over_ranks([t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med,
+                                              ffn_ovl_med, post_seq, post_ovl, t_graph,
+                                              t_ovl_hooked], world, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -377,12 +414,28 @@ def run_ours(args):
                            "overlapped_ms_per_step": t_ovl_med, "overlapped_ffn_ms": ffn_ovl_med,
                            "method": "K steps of each mode, alternating step by step; medians"},
             "speedup_vs_sequential": t_seq / t_ovl_med,
+            # Overlap accounting from the paired steps (medians):
+            #   producer only = the sequential mode's GEMM1 and GEMM2 launches,
+            #   combine only  = the sequential mode's combine pass,
+            #   overlapped    = the overlapped mode's persistent launch + remainder pass;
+            #   ratio = 1 - (overlapped - producer only) / combine only  (1: the combine
+            #   is fully hidden; above 1: the single launch also saves the GEMM1 -> GEMM2
+            #   launch boundary); op_speedup = (producer only + combine only) / overlapped.
+            "overlap": {"producer_only_ms": ffn_seq, "combine_only_ms": post_seq,
+                        "overlapped_ms": ffn_ovl_med + post_ovl, "remainder_combine_ms": post_ovl,
+                        "ratio": 1.0 - (ffn_ovl_med + post_ovl - ffn_seq) / post_seq,
+                        "op_speedup": (ffn_seq + post_seq) / (ffn_ovl_med + post_ovl)},
+            "graph": {"ms_per_step": t_graph, "eager_ms_per_step": t_ovl,
+                      "method": "the overlapped call captured once in a CUDA graph, K replays"},
             "consumer_sms": consumer_sms,
             "n_bands": n_bands,
             "masked_row_waste": (n_bands * 128 - wl.R) / (n_bands * 128),
             "roofline": {"kernel": "ffn_kernel (persistent GEMM1+GEMM2+combine)", "bound": "tensor",
                          "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s", "frac": ach / peak_tf,
                          "traffic": traffic, "launch_ms": ffn_ovl,
+                         "launch_timing": "CUDA events on the launching stream around the "
+                                          "persistent kernel, K overlapped steps after the "
+                                          "contract region (%.4f ms per step there)" % t_ovl_hooked,
                          "peak_kind": f"{src} sustained bf16 (cuBLAS 8192^3 under the power cap)"},
             "e2e": {"value": job_tokens_per_s(wl.T, world, t_e2e), "unit": "tokens/s", "ms_per_step": t_e2e,
                     "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
@@ -471,6 +524,57 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_oracle_timings(args):
+    """The CPU oracle's own speed on each benchmark configuration, as it stands:
+    single-threaded on the tiny layer (whole layer, permuted path) and on the T=512
+    sweep layer; on every host thread for the Mixtral-shaped, fine-grained and
+    imbalanced layers.  Beyond the tiny layer a token sample of about
+    `--cpu-seconds` of work is timed through the token-by-token definition path and
+    the whole layer is extrapolated from it (marked so)."""
+    import oracle
+    o = oracle.get()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    nproc = os.cpu_count() or 1
+    cpu = _cpu_model()
+    for name, threads in (("tiny", 1), ("sweep_T512_uniform", 1), ("mixtral", nproc),
+                          ("fine_grained", nproc), ("imbalanced", nproc)):
+        wl = synth.WORKLOADS[name]
+        inp = synth.make_inputs(wl, dev)
+        xh = synth.bf16_bits(inp["x"])
+        lh = inp["logits"].detach().cpu().numpy()
+        W = [synth.bf16_bits(inp[n]) for n in ("W1", "W3", "W2")]
+        del inp
+        used = o.set_threads(threads)
+        if name == "tiny":
+            t0 = time.perf_counter()
+            o.forward(xh, lh, W[0], W[1], W[2], wl.k)
+            dt = time.perf_counter() - t0
+            n, extrap = wl.T, False
+        else:
+            idx, gate = o.route(lh, wl.k)
+            n, dt = _oracle_tokens_per_s(o, xh, idx, gate, W, max(used, 2), wl.T, 1)
+            n = int(min(wl.T, max(used, n * args.cpu_seconds / max(dt, 1e-6))))
+            n, dt = _oracle_tokens_per_s(o, xh, idx, gate, W, n, wl.T, 2)
+            extrap = n < wl.T
+        tps = n / dt
+        print(json.dumps({"oracle_timing": name, "threads": used, "nproc": nproc, "cpu": cpu,
+                          "tokens_timed": n, "seconds": dt, "tokens_per_s": tps,
+                          "layer_seconds": wl.T / tps, "extrapolated": extrap,
+                          "path": "whole layer (permuted)" if name == "tiny"
+                          else "token-by-token definition path"}), flush=True)
+
+
 def run_sweep(args):
     """Every sweep cell: the overlapped mode at a fixed consumer-SM count (2, 4, 8)
     or the cost model's choice (0), against the sequential mode, timed as paired
@@ -523,6 +627,9 @@ def main():
     args = parse()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.oracle_timings:
+        run_oracle_timings(args)
         return
     if args.steps < 1 or args.warmup < 0:
         raise SystemExit("--steps must be >= 1 and --warmup >= 0")

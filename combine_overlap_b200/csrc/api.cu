@@ -374,6 +374,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
     a.phase = PH_G1 | PH_G2 | PH_CONS;
     a.join = join;
     MOE_TRY(launch_ffn(a, grid, st));
+    if (A.ev_ffn_end) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_end), st));
     // Consumers stop once the GEMM work is done; a full-occupancy combine pass
     // finishes every token they did not (same arithmetic, so the same bits).
     MOE_TRY(launch_combine(w.y, w.row_of, w.topk_gate, T, d, k, a.out, nsm, st, w.arrive));
@@ -382,9 +383,9 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
     MOE_TRY(launch_ffn(a, grid, st));
     a.phase = PH_G2;
     MOE_TRY(launch_ffn(a, grid, st));
+    if (A.ev_ffn_end) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_end), st));
     MOE_TRY(launch_combine(w.y, w.row_of, w.topk_gate, T, d, k, a.out, nsm, st));
   }
-  if (A.ev_ffn_end) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_end), st));
   return MOE_OK;
 }
 

@@ -108,9 +108,12 @@ typedef struct {
   unsigned flags;           /* MOE_DBG_* / MOE_SCHED_* bits                         */
   int timeout_us;           /* bound on each device wait; 0 = default (2 s)         */
   /* Optional timing hooks (cudaEvent_t as void*, NULL = none): recorded on the
-   * stream just before the first and just after the last expert-FFN launch
-   * (overlapped: the one persistent kernel, which also runs the combine;
-   * sequential: GEMM1, GEMM2 and the combine kernel). */
+   * stream just before the first and just after the last expert-FFN launch,
+   * i.e. around the one persistent kernel (overlapped mode; it also runs the
+   * overlapped part of the combine) or around GEMM1 and GEMM2 (sequential mode).
+   * The combine pass that follows (the remainder, or the full combine) is
+   * outside the span.  A recorded event separates the launches on either side,
+   * so their programmatic overlap is lost while the hooks are in use. */
   void* ev_ffn_begin;
   void* ev_ffn_end;
 } moe_layer_args;
