@@ -257,7 +257,7 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
   MOE_TRY(launch_hist(topk_idx, T, E, k, w.blk_hist, st));
   MOE_TRY(launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, default_cost_model(), st));
   MOE_TRY(launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, nullptr, st));
-  MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(x), perm, T * k, d, k,
+  MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(x), row_of, T, d, k,
                         static_cast<__nv_bfloat16*>(x_perm), nsm, st));
   return MOE_OK;
 }
@@ -351,7 +351,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   const int gather_a = (A.flags & MOE_SCHED_GATHER_A) ? 1 : 0;
   MOE_TRY(launch_scatter(w.topk_idx, T, E, k, w.blk_base, w.perm, w.row_of, gather_a ? &w : nullptr, st));
   if (!gather_a)
-    MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(A.x), w.perm, R, d, k, w.x_perm, nsm, st));
+    MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(A.x), w.row_of, T, d, k, w.x_perm, nsm, st));
   FfnArgs a;
   memset(&a, 0, sizeof(a));
   a.w = w;

@@ -46,7 +46,8 @@ cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int 
 // With a plan (w.bands etc. set), also fills w.tok_band, GEMM1's gather indices.
 cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const int32_t* blk_base,
                            int32_t* perm, int32_t* row_of, const Work* plan, cudaStream_t s);
-cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, int R, int d, int k,
+// x_perm[row_of[p]] = x[p / k] for every slot p < T*k (token-major copy).
+cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* row_of, int T, int d, int k,
                           __nv_bfloat16* x_perm, int num_sms, cudaStream_t s);
 
 // combine.cu

@@ -114,7 +114,7 @@ extern "C" moe_status moe_permute_noalloc(const void* x, int T, int d, int E, in
   if (e == cudaSuccess) e = launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, cm, st);
   if (e == cudaSuccess) e = launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, nullptr, st);
   if (e == cudaSuccess)
-    e = launch_gather(static_cast<const __nv_bfloat16*>(x), perm, T * k, d, k,
+    e = launch_gather(static_cast<const __nv_bfloat16*>(x), row_of, T, d, k,
                       static_cast<__nv_bfloat16*>(x_perm), nsm, st);
   if (e != cudaSuccess) return fail(e);
   return MOE_OK;

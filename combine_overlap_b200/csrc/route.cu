@@ -16,83 +16,99 @@
 namespace moe {
 
 // ------------------------------------------------------------------ route ---
-// One warp per token.  Lane l holds logits of experts l, l+32, ... (E <= 256).
-// k rounds of a warp arg-max under the order (logit desc, id asc).  Lane 0 then
-// forms the gates in double (exp of l_j - l_0, summed in slot order) and adds the
-// token's experts to the block's histogram (blk_hist[b][e], no global atomics:
-// the plan kernel scans the per-block counts, so ranks come out deterministic).
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E,
-                                                    int k, int32_t* __restrict__ topk_idx,
-                                                    float* __restrict__ topk_gate,
-                                                    int32_t* __restrict__ blk_hist,
-                                                    uint32_t* __restrict__ arrive,
-                                                    uint32_t* __restrict__ ready_q) {
+// A warp ranks RT_W tokens in lockstep (their shuffle chains interleave); a block
+// of ROUTE_TOK / RT_W warps takes ROUTE_TOK tokens.  Lane l holds logits of
+// experts l, l+32, ... (E <= 256).  k rounds of a warp arg-max under the order
+// (logit desc, id asc); after round j, lane j keeps slot j's expert and logit.
+// Lane j then forms w_j = exp(l_j - l_0) in double, every lane sums the w_j in
+// slot order, and lane j writes slot j and adds its expert to the block's
+// histogram (blk_hist[b][e], no global atomics: the plan kernel scans the
+// per-block counts, so ranks come out deterministic).
+constexpr int RT_W = 4;
+constexpr int ROUTE_THREADS = ROUTE_TOK / RT_W * 32;
+
+__global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(const float* __restrict__ logits,
+                                                              int T, int E, int k,
+                                                              int32_t* __restrict__ topk_idx,
+                                                              float* __restrict__ topk_gate,
+                                                              int32_t* __restrict__ blk_hist,
+                                                              uint32_t* __restrict__ arrive,
+                                                              uint32_t* __restrict__ ready_q) {
   pdl_trigger();
   pdl_wait();
   __shared__ int hist[MAX_E];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  const int t0 = blockIdx.x * ROUTE_TOK;
-  const int t1 = min(T, t0 + ROUTE_TOK);
+  const int tb = blockIdx.x * ROUTE_TOK + warp * RT_W;
   const int nv = (E + 31) >> 5;
-  // software pipeline: the next token's logits are loaded while this one is ranked
-  float vn[8];
+  float v[RT_W][8];
+  uint32_t used[RT_W];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    vn[i] = (t0 + warp < t1 && i < nv && e < E) ? __ldg(logits + (size_t)(t0 + warp) * E + e) : -FLT_MAX;
-  }
-  for (int t = t0 + warp; t < t1; t += 8) {
-    float v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = vn[i];
-    const int tn = t + 8;
+  for (int q = 0; q < RT_W; ++q) {
+    used[q] = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane + 32 * i;
-      vn[i] = (tn < t1 && i < nv && e < E) ? __ldg(logits + (size_t)tn * E + e) : -FLT_MAX;
+      const bool ok = tb + q < T && i < nv && e < E;
+      v[q][i] = ok ? __ldg(logits + (size_t)(tb + q) * E + e) : -FLT_MAX;
+      if (!(i < nv && e < E)) used[q] |= 1u << i;
     }
-    uint32_t used = 0;
-    for (int i = 0; i < 8; ++i)
-      if (!(i < nv && lane + 32 * i < E)) used |= 1u << i;
-    int sel_e[MAX_K];
-    float sel_v[MAX_K];
-    for (int j = 0; j < k; ++j) {
-      float bv = -FLT_MAX;
-      int be = 0x7fffffff;
+  }
+  int my_e[RT_W];
+  float my_v[RT_W], vmax[RT_W];
+#pragma unroll
+  for (int q = 0; q < RT_W; ++q) { my_e[q] = 0; my_v[q] = 0.0f; vmax[q] = 0.0f; }
+  for (int j = 0; j < k; ++j) {
+    float bv[RT_W];
+    int be[RT_W];
+#pragma unroll
+    for (int q = 0; q < RT_W; ++q) {
+      bv[q] = -FLT_MAX;
+      be[q] = 0x7fffffff;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int e = lane + 32 * i;
-        if (!(used & (1u << i)) && (v[i] > bv || (v[i] == bv && e < be))) { bv = v[i]; be = e; }
+        if (!(used[q] & (1u << i)) && (v[q][i] > bv[q] || (v[q][i] == bv[q] && e < be[q]))) {
+          bv[q] = v[q][i];
+          be[q] = e;
+        }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-      }
-      if ((be & 31) == lane) used |= 1u << (be >> 5);
-      sel_e[j] = be;
-      sel_v[j] = bv;
     }
-    // gates: lane j < k forms w_j = exp(l_j - l_0) in double; lane 0 sums them in
-    // slot order; lane j writes slot j
-    double wj = 0.0;
-    int ej = 0;
 #pragma unroll
-    for (int j = 0; j < MAX_K; ++j)
-      if (j < k && lane == j) { ej = sel_e[j]; wj = exp((double)sel_v[j] - (double)sel_v[0]); }
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int q = 0; q < RT_W; ++q) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv[q], off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be[q], off);
+        if (ov > bv[q] || (ov == bv[q] && oe < be[q])) { bv[q] = ov; be[q] = oe; }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < RT_W; ++q) {
+      if ((be[q] & 31) == lane) used[q] |= 1u << (be[q] >> 5);
+      if (lane == j) { my_e[q] = be[q]; my_v[q] = bv[q]; }
+      if (j == 0) vmax[q] = bv[q];
+    }
+  }
+  // gates: lane j < k forms w_j = exp(l_j - l_0) in double; the sum runs in slot
+  // order; lane j writes slot j
+#pragma unroll
+  for (int q = 0; q < RT_W; ++q) {
+    const int t = tb + q;
+    const double wj = lane < k ? exp((double)my_v[q] - (double)vmax[q]) : 0.0;
     double ssum = 0.0;
     for (int j = 0; j < k; ++j) ssum += __shfl_sync(0xffffffffu, wj, j);
-    if (lane < k) {
-      topk_idx[(size_t)t * k + lane] = ej;
-      topk_gate[(size_t)t * k + lane] = (float)(wj / ssum);
-      atomicAdd(&hist[ej], 1);
-    }
-    if (lane == 0) {
-      if (arrive) arrive[t] = 0u;
-      if (ready_q) ready_q[t] = 0u;
+    if (t < T) {
+      if (lane < k) {
+        topk_idx[(size_t)t * k + lane] = my_e[q];
+        topk_gate[(size_t)t * k + lane] = (float)(wj / ssum);
+        atomicAdd(&hist[my_e[q]], 1);
+      }
+      if (lane == 0) {
+        if (arrive) arrive[t] = 0u;
+        if (ready_q) ready_q[t] = 0u;
+      }
     }
   }
   __syncthreads();
@@ -102,8 +118,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx,
                          float* topk_gate, int32_t* blk_hist, uint32_t* arrive, uint32_t* ready_q,
                          cudaStream_t s) {
-  return launch_pdl(route_kernel, dim3(route_blocks(T)), dim3(256), 0, s, logits, T, E, k, topk_idx,
-                    topk_gate, blk_hist, arrive, ready_q);
+  return launch_pdl(route_kernel, dim3(route_blocks(T)), dim3(ROUTE_THREADS), 0, s, logits, T, E,
+                    k, topk_idx, topk_gate, blk_hist, arrive, ready_q);
 }
 
 __global__ void colsum_kernel(const int32_t* __restrict__ blk_hist, int nblk, int E,
@@ -213,26 +229,40 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
   __shared__ int bstart[MAX_E + 1];
   __shared__ int gstart[MAX_E + 1];
   __shared__ int t1start[MAX_E + 1];
-  __shared__ int lane_base[MAX_E][32];
+  __shared__ int part[1024];        // [g][e]: rows' sums of chunk g, then its exclusive base
   __shared__ int totals[3];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nwarps = blockDim.x >> 5;
-  // Counts and per-block scatter bases: warp w scans expert e = w, w + 32, ...
-  // over the blocks (lane i owns a contiguous chunk of blocks).
-  const int chunk = nblk > 0 ? cdiv(nblk, 32) : 0;
-  const int cb0 = min(nblk, lane * chunk), cb1 = min(nblk, cb0 + chunk);
+  // Counts and per-block scatter bases.  Thread (g, e) = (tid / E, tid % E) owns
+  // expert e over the contiguous chunk g of route blocks, so a warp's loads and
+  // stores cover consecutive experts of the same rows (coalesced).
+  const int NG = nblk > 0 ? (int)blockDim.x / E : 0;    // chunks (E <= 256 <= blockDim)
+  const int chunk = NG > 0 ? cdiv(nblk, NG) : 0;
+  const int g = tid / E, ge = tid - g * E;
+  const bool owner = nblk > 0 && g < NG;
+  const int cb0 = owner ? min(nblk, g * chunk) : 0, cb1 = owner ? min(nblk, cb0 + chunk) : 0;
+  const int32_t* __restrict__ bh = w.blk_hist;
   if (nblk > 0) {
-    for (int e = warp; e < E; e += nwarps) {
-      int sum = 0;
-      for (int b = cb0; b < cb1; ++b) sum += w.blk_hist[(size_t)b * E + e];
-      int inc = sum;
+    // 8 independent loads in flight per thread
+    int sum = 0, b = cb0;
+    for (; b + 8 <= cb1; b += 8) {
+      int hv[8];
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, inc, off);
-        if (lane >= off) inc += t;
+      for (int u = 0; u < 8; ++u) hv[u] = bh[(size_t)(b + u) * E + ge];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += hv[u];
+    }
+    for (; b < cb1; ++b) sum += bh[(size_t)b * E + ge];
+    if (owner) part[tid] = sum;
+    __syncthreads();
+    // per expert, an exclusive scan over the NG chunks (NG <= 128 sequential steps)
+    for (int e = tid; e < E; e += blockDim.x) {
+      int run = 0;
+      for (int c = 0; c < NG; ++c) {
+        const int v = part[c * E + e];
+        part[c * E + e] = run;
+        run += v;
       }
-      lane_base[e][lane] = inc - sum;
-      if (lane == 31) cnt[e] = inc;
+      cnt[e] = run;
     }
   } else {
     for (int e = tid; e < E; e += blockDim.x) cnt[e] = offsets_in[e + 1] - offsets_in[e];
@@ -249,14 +279,21 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
     if (e < E) w.counts[e] = cnt[e];
     w.offsets[e] = offs[e];
   }
-  if (nblk > 0) {
-    for (int e = warp; e < E; e += nwarps) {
-      int run = offs[e] + lane_base[e][lane];
-      for (int b = cb0; b < cb1; ++b) {
-        const int hcount = w.blk_hist[(size_t)b * E + e];
-        w.blk_base[(size_t)b * E + e] = run;
-        run += hcount;
-      }
+  if (owner) {
+    int32_t* __restrict__ bb = w.blk_base;
+    int run = offs[ge] + part[tid];
+    int b = cb0;
+    for (; b + 8 <= cb1; b += 8) {
+      int hv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) hv[u] = bh[(size_t)(b + u) * E + ge];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) { bb[(size_t)(b + u) * E + ge] = run; run += hv[u]; }
+    }
+    for (; b < cb1; ++b) {
+      const int hcount = bh[(size_t)b * E + ge];
+      bb[(size_t)b * E + ge] = run;
+      run += hcount;
     }
   }
   // expert priority: rows descending, id ascending (rank by comparison count)
@@ -421,26 +458,51 @@ cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const i
 
 // ----------------------------------------------------------------- gather ---
 // x_perm[r] = x[perm[r] / k]: one warp per row, 16-byte vector loads and stores.
+// x_perm[row_of[t*k + j]] = x[t] for every slot: token-major, so each x row is
+// read from memory once and written to its k expert rows (a row-major walk of
+// x_perm would re-read x[t] k times, from DRAM once x outgrows L2).  One warp per
+// token; 4 x 16-byte vectors per lane in flight, then k stores of each.
 __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x,
-                                                     const int32_t* __restrict__ perm, int R,
+                                                     const int32_t* __restrict__ row_of, int T,
                                                      int dv, int k, uint4* __restrict__ x_perm) {
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
-  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < R; r += gridDim.x * wpb) {
-    const size_t t = (size_t)(perm[r] / k);
-    const uint4* src = x + t * dv;
-    uint4* dst = x_perm + (size_t)r * dv;
-    for (int v = lane; v < dv; v += 32) dst[v] = __ldg(src + v);
+  constexpr int U = 4;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    const int my_row = lane < k ? row_of[(size_t)t * k + lane] : 0;
+    int rows[MAX_K];
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+    const uint4* src = x + (size_t)t * dv;
+    for (int v0 = 0; v0 < dv; v0 += 32 * U) {
+      uint4 buf[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < dv) buf[u] = __ldcs(src + v);
+      }
+#pragma unroll
+      for (int j = 0; j < MAX_K; ++j) {
+        if (j < k) {
+          uint4* dst = x_perm + (size_t)rows[j] * dv;
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * 32 + lane;
+            if (v < dv) dst[v] = buf[u];
+          }
+        }
+      }
+    }
   }
 }
 
-cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* perm, int R, int d, int k,
+cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* row_of, int T, int d, int k,
                           __nv_bfloat16* x_perm, int num_sms, cudaStream_t s) {
-  const int grid = max(1, min(cdiv(R, 8), num_sms * 8));
-  return launch_pdl(gather_kernel, dim3(grid), dim3(256), 0, s, reinterpret_cast<const uint4*>(x), perm, R,
-                    d / 8, k, reinterpret_cast<uint4*>(x_perm));
+  const int grid = max(1, min(cdiv(T, 8), num_sms * 8));
+  return launch_pdl(gather_kernel, dim3(grid), dim3(256), 0, s, reinterpret_cast<const uint4*>(x),
+                    row_of, T, d / 8, k, reinterpret_cast<uint4*>(x_perm));
 }
 
 }  // namespace moe
