@@ -42,16 +42,22 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the persistent FFN kernel, keyed by workload, valid only for the kernel sources
 # whose hash is recorded with it (see profiles/).
-TRAFFIC = {"mixtral": {"bytes": 3795754000 + 319245568, "kernel_hash": "6d336c6e34e0"}}
+TRAFFIC = {"mixtral": {"bytes": 3795754000 + 319245568, "kernel_hash": "753fdff4af9e"}}
 
 
 def kernel_source_hash() -> str:
+    """Hash of the code (comments and whitespace removed) of the files that make
+    and launch the persistent FFN kernel."""
+    import re
     h = hashlib.sha1()
     for rel in ("combine_overlap_b200/csrc/ffn.cu", "combine_overlap_b200/csrc/common.cuh",
                 "combine_overlap_b200/csrc/combine.cuh", "combine_overlap_b200/csrc/kernels.h",
                 "combine_overlap_b200/csrc/api.cu"):
-        with open(os.path.join(ROOT, rel), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)   # block comments
+        src = re.sub(r"//[^\n]*", " ", src)                 # line comments
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:12]
 
 

@@ -19,26 +19,29 @@
 // once the GEMM tile queue is empty.
 //
 // B200 mapping (differs from the paper's A100 CUTLASS/NVSHMEM kernels):
-//   * one launch of one CTA per SM (cooperative launch: all CTAs co-resident),
-//     each CTA taking tiles from an atomic work queue in priority order instead
-//     of a fixed stride;
+//   * one launch of one CTA per SM (G = 1: a cooperative launch; G = 2: a
+//     cluster launch of as many pairs as can be resident at once), each CTA
+//     taking tiles from an atomic work queue in priority order instead of a
+//     fixed stride;
 //   * per CTA: warp 0 = tile scheduler + TMA producer, warp 1 = TMEM allocator
 //     + single-thread tcgen05.mma issuer, warps 2-5 = epilogue (TMEM -> registers
 //     -> bf16 -> global), a 192 KB smem operand ring, two 256-column TMEM
 //     accumulators so the epilogue of one tile overlaps the main loop of the next;
-//   * two variants, G = CTAs per MMA: G = 1, one CTA per 128-row tile; G = 2
-//     (default), a cluster pair per 256-row tile with tcgen05 cta_group::2 -- the
-//     leader issues the MMAs, each CTA loads its 128 rows of A and half of B (no
-//     multicast), and work items are mirrored into the peer over DSMEM;
+//   * two variants, G = CTAs per MMA, chosen per call by the host: G = 1, one
+//     CTA per 128-row tile (weight tiles in one 4-D TMA copy per operand); G = 2,
+//     a cluster pair per 256-row tile with tcgen05 cta_group::2 -- the leader
+//     issues the MMAs, each CTA loads its 128 rows of A and half of B (no
+//     multicast), work items are mirrored into the peer over DSMEM, and an
+//     expert's odd last band runs as an M=128 half tile;
 //   * GEMM1 tile: 128*G rows x 128 h-columns; one N=256 MMA accumulates x*W1 and
 //     x*W3 side by side (the B tile holds the W1 and W3 column blocks), and the
 //     epilogue applies silu(a)*b;  GEMM2 tile: 128*G rows x 256 y-columns;
 //   * A (x_perm or h) is K-major, W is stored [K][N] (N-major): both are read
 //     by TMA with 128-byte swizzle and fed to tcgen05 as K-major / MN-major
 //     operands, so the weights need no repacking;
-//   * signals are counters per row band (GEMM1 tiles done, GEMM2 tiles done)
-//     published with red.release and polled with ld.acquire; every wait is
-//     bounded and reports MOE_ERR_TIMEOUT through the status block.
+//   * signals are counters per row band (GEMM1 tiles done, GEMM2 tiles done,
+//     2 per tile) published with red.release and polled with ld.acquire; every
+//     wait is bounded and reports MOE_ERR_TIMEOUT through the status block.
 #include "kernels.h"
 #include "combine.cuh"
 #include "../../include/moe.h"

@@ -132,3 +132,36 @@ def test_layer_full_size_sampled(orc, name, flags):
     ref = orc.tokens(gu.host(inp["x"]), oidx, ogate, gu.host(inp["W1"]), gu.host(inp["W3"]),
                      gu.host(inp["W2"]), toks)
     gu.assert_close(ovl_bits[toks], ref, what=f"{name} sampled tokens")
+
+
+def _check_variants(orc, wl, inp):
+    """Both tile variants against the oracle, and overlapped == sequential in each."""
+    ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
+    ref = orc.forward(gu.host(inp["x"]), gu.host(inp["logits"]), gu.host(inp["W1"]),
+                      gu.host(inp["W3"]), gu.host(inp["W2"]), wl.k)
+    for fl in (moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR):
+        seq, extra, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL, flags=fl)
+        assert np.array_equal(gu.host(extra["topk_idx"]), ref["topk_idx"])
+        assert np.array_equal(gu.host(extra["counts"]), ref["counts"])
+        assert np.array_equal(gu.host(extra["perm"]), ref["perm"])
+        gu.assert_close(gu.host(seq), ref["out"], what=f"{wl.name} flags {fl:#x}")
+        for kw in (dict(), dict(consumer_sms=4)):
+            ovl, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=fl, **kw)
+            assert np.array_equal(gu.host(ovl), gu.host(seq)), (fl, kw)
+
+
+def test_layer_max_experts(orc):
+    # the largest expert count and top-k the library accepts: E = 256, k = 8, so
+    # about 9 rows per expert and hundreds of one-band groups (pairs: half tiles)
+    wl = synth.small("max_experts", 300, 256, 128, 256, 8, "normal2")
+    _check_variants(orc, wl, gu.inputs(wl))
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_layer_every_token_one_expert(orc, k):
+    # every token's first choice is expert 3 (its logit raised by 50): one expert
+    # holds T rows in 8 bands (k = 1 leaves the other 7 experts empty)
+    wl = synth.small(f"one_expert_k{k}", 1000, 256, 256, 8, k)
+    inp = gu.inputs(wl)
+    inp["logits"][:, 3] += 50.0
+    _check_variants(orc, wl, inp)
