@@ -42,7 +42,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the persistent FFN kernel, keyed by workload, valid only for the kernel sources
 # whose hash is recorded with it (see profiles/).
-TRAFFIC = {"mixtral": {"bytes": 3795754000 + 319245568, "kernel_hash": "753fdff4af9e"}}
+TRAFFIC = {"mixtral": {"bytes": 4314479000 + 312666112, "kernel_hash": "82c8f29a620f"}}
 
 
 def kernel_source_hash() -> str:
@@ -85,6 +85,8 @@ def parse():
     ap.add_argument("--b-per-atom", action="store_true",
                     help="load weight tiles with one TMA copy per 64-column atom")
     ap.add_argument("--cta-pair", action="store_true", help="force 256-row tiles on CTA pairs")
+    ap.add_argument("--wide-cta", action="store_true",
+                    help="force 256-row tiles on single CTAs (two 128-row MMAs per K step)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -221,7 +223,8 @@ def run_ours(args):
     kw = dict(consumer_sms=args.consumer_sms, mgb=args.mgb,
               flags=(moe.SCHED_NO_JOIN if args.no_join else 0) | (moe.SCHED_ONE_CTA if args.one_cta else 0)
               | (moe.SCHED_CTA_PAIR if args.cta_pair else 0)
-              | (moe.SCHED_B_PER_ATOM if args.b_per_atom else 0))
+              | (moe.SCHED_B_PER_ATOM if args.b_per_atom else 0)
+              | (moe.SCHED_WIDE_CTA if args.wide_cta else 0))
 
     def step(mode, evb=None, eve=None):
         moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, mode, out=out, ev_begin=evb, ev_end=eve, **kw)
@@ -404,10 +407,8 @@ def run_ours(args):
             "data": "synthetic: seeded counter-based N(0,1) tokens and gate logits, random-init N(0,0.02) bf16 expert weights",
             "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "d_ff": wl.f, "E": wl.E,
                        "top_k": wl.k, "router": wl.router, "mode": "overlapped",
-                       "mma_tile": ("256x256 per CTA pair (cta_group::2)"
-                                    if not args.one_cta and (args.cta_pair or (
-                                        wl.R >= 512 * wl.E and wl.f >= 8192))
-                                    else "128x256 per CTA"),
+                       "mma_tile": moe.TILE_VARIANTS[moe.tile_variant(wl.T, wl.f, wl.E, wl.k,
+                                                                      kw["flags"])],
                        "parallelism": f"replicas x{world} (token shards, no collective)",
                        "l2": "inputs larger than L2: active expert weights %.2f GB per step" % (B / 1e9)},
             "tflops": world * F / (t_ovl * 1e-3) / 1e12,

@@ -168,19 +168,28 @@ CostModel default_cost_model() {
 
 inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : cuda_fail(e); }
 
-// CTAs per MMA tile.  A CTA pair (256-row tiles, cta_group::2) streams a third
-// less operand data per FLOP than a single CTA (128-row tiles, whose weight tiles
-// come in one 4-D TMA copy per operand), but each pair tile carries more fixed
-// cost and, below 512 rows per expert, more masked rows.  Measured on B200, one
-// variant per process (alternating the two kernels step by step penalises the
-// pair): pairs are 2 % faster at d_ff = 14336 with 1024-2048 rows per expert,
-// even at d_ff = 4096-8192, and 3-14 % slower at d_ff <= 2048 or below 512 rows
-// per expert.  So pairs are picked when T*k/E >= 512 and d_ff >= 8192.
-int choose_group(int T, int f, int E, int k, unsigned flags) {
+// Tile variant (FfnArgs::V).  A CTA pair (V = 2: 256-row tiles, cta_group::2) or
+// a single CTA with two 128-row MMAs per K step (V = 3: 256-row tiles) streams a
+// third less operand data per FLOP than a single CTA with 128-row tiles (V = 1),
+// but a 256-row tile wastes more masked rows when experts are small, a pair
+// couples two SMs' loads, and V = 3 gives up the accumulator double-buffering.
+// Measured on B200, one variant per process (alternating two kernels step by
+// step penalises the pair): V = 3 is 4-9 % faster than V = 1 from 256 rows per
+// expert up (T=2048-32768 at d_ff = 2048, the fine-grained and imbalanced
+// layers) and 6-8 % faster than pairs on the Mixtral-shaped layer; at 64 rows
+// per expert V = 1 is 4 % faster.  So V = 3 when T*k/E >= 256, else V = 1.
+// Flags force a variant (MOE_SCHED_ONE_CTA before MOE_SCHED_CTA_PAIR before
+// MOE_SCHED_WIDE_CTA).
+int choose_variant(int T, int f, int E, int k, unsigned flags) {
+  (void)f;
   if (flags & MOE_SCHED_ONE_CTA) return 1;
   if (flags & MOE_SCHED_CTA_PAIR) return 2;
-  return (long long)T * k >= 512LL * E && f >= 8192 ? 2 : 1;
+  if (flags & MOE_SCHED_WIDE_CTA) return 3;
+  return (long long)T * k >= 256LL * E ? 3 : 1;
 }
+
+inline int bands_per_tile(int V) { return V == 1 ? 1 : 2; }
+inline int ctas_per_tile(int V) { return V == 2 ? 2 : 1; }
 
 #define MOE_TRY(expr)                                   \
   do {                                                  \
@@ -195,6 +204,11 @@ extern "C" {
 size_t moe_workspace_size(int T, int d, int f, int E, int k) {
   if (check_shape(T, d, f, E, k) != MOE_OK) return 0;
   return layout(T, d, f, E, k).total;
+}
+
+int moe_tile_variant(int T, int f, int E, int k, unsigned flags) {
+  if (T < 1 || f < 1 || E < 1 || k < 1) return 0;
+  return choose_variant(T, f, E, k, flags);
 }
 
 int moe_last_cuda_error(void) { return (int)moe::last_cuda_error(); }
@@ -255,7 +269,7 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
   w.row_of = row_of;
   const int nblk = route_blocks(T);
   MOE_TRY(launch_hist(topk_idx, T, E, k, w.blk_hist, st));
-  MOE_TRY(launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, default_cost_model(), st));
+  MOE_TRY(launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, 1, default_cost_model(), st));
   MOE_TRY(launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, nullptr, st));
   MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(x), row_of, T, d, k,
                         static_cast<__nv_bfloat16*>(x_perm), nsm, st));
@@ -270,18 +284,19 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
   if (!ok_ptr(x_perm) || !ok_ptr(offsets) || !ok_ptr(W1) || !ok_ptr(W3) || !ok_ptr(W2) ||
       !ok_ptr(y) || !ok_opt(h))
     return MOE_ERR_INVALID;
-  constexpr unsigned tile_flags =
-      MOE_SCHED_ONE_CTA | MOE_SCHED_CTA_PAIR | MOE_SCHED_B_PER_ATOM | MOE_SCHED_FULL_TILES;
+  constexpr unsigned tile_flags = MOE_SCHED_ONE_CTA | MOE_SCHED_CTA_PAIR | MOE_SCHED_WIDE_CTA |
+                                  MOE_SCHED_B_PER_ATOM | MOE_SCHED_FULL_TILES;
   if (flags & ~tile_flags) return MOE_ERR_INVALID;
   const Layout L = layout(T, d, f, E, k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  const int G = choose_group(T, f, E, k, flags);
+  const int V = choose_variant(T, f, E, k, flags);
   int grid = 0;
-  MOE_TRY(ffn_grid(G, &grid));
-  if (grid <= G) return cuda_fail(cudaErrorInvalidConfiguration);
+  MOE_TRY(ffn_grid(V, &grid));
+  if (grid <= ctas_per_tile(V)) return cuda_fail(cudaErrorInvalidConfiguration);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Work w = work_from(ws, L, true, true);
-  MOE_TRY(launch_plan(w, 0, offsets, T, d, f, E, k, grid, 1, 1, G, 1, default_cost_model(), st));
+  MOE_TRY(launch_plan(w, 0, offsets, T, d, f, E, k, grid, 1, 1, bands_per_tile(V), ctas_per_tile(V),
+                      1, default_cost_model(), st));
   FfnArgs a;
   memset(&a, 0, sizeof(a));
   a.w = w;
@@ -290,7 +305,7 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
   a.y = static_cast<__nv_bfloat16*>(y);
   a.W1 = W1; a.W3 = W3; a.W2 = W2;
   a.R = T * k; a.T = T; a.d = d; a.f = f; a.E = E; a.k = k;
-  a.G = G;
+  a.V = V;
   a.phase = PH_G1 | PH_G2;
   a.join = 0;
   a.mgb = 1;
@@ -327,10 +342,18 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   const Layout L = layout(A.T, A.d, A.f, A.E, A.k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   const int nsm = device_sms();
-  const int G = choose_group(A.T, A.f, A.E, A.k, A.flags);
+  // MOE_SCHED_GATHER_A: GEMM1 gathers its A rows from x with TMA gather4 instead
+  // of reading x_perm (no x_perm pass, but 32 gather instructions per k-block);
+  // 128-row gathers only, so not with V = 3
+  const int gather_a = (A.flags & MOE_SCHED_GATHER_A) ? 1 : 0;
+  int V = choose_variant(A.T, A.f, A.E, A.k, A.flags);
+  if (gather_a && V == 3) {
+    if (A.flags & MOE_SCHED_WIDE_CTA) return MOE_ERR_UNSUPPORTED;
+    V = 1;
+  }
   int grid = 0;
-  MOE_TRY(ffn_grid(G, &grid));
-  if (nsm <= 1 || grid <= G) return cuda_fail(cudaErrorInvalidConfiguration);
+  MOE_TRY(ffn_grid(V, &grid));
+  if (nsm <= 1 || grid <= ctas_per_tile(V)) return cuda_fail(cudaErrorInvalidConfiguration);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Work w = work_from(ws, L, true, true);
   if (A.topk_idx) w.topk_idx = A.topk_idx;
@@ -343,12 +366,10 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   const int nblk = route_blocks(T);
   MOE_TRY(launch_route(A.logits, T, E, k, w.topk_idx, w.topk_gate, w.blk_hist, w.arrive, w.ready_q, st));
   const int join = (A.flags & MOE_SCHED_NO_JOIN) ? 0 : 1;
-  MOE_TRY(launch_plan(w, nblk, nullptr, T, d, f, E, k, grid, A.consumer_sms, mgb, G, join,
+  MOE_TRY(launch_plan(w, nblk, nullptr, T, d, f, E, k, grid, A.consumer_sms, mgb, bands_per_tile(V),
+                      ctas_per_tile(V), join,
                       default_cost_model(), st));
   // Default: a gather kernel writes x_perm and GEMM1 reads it with tiled TMA loads.
-  // MOE_SCHED_GATHER_A: GEMM1 gathers its A rows from x with TMA gather4 instead
-  // (no x_perm pass, but 32 gather instructions per k-block).
-  const int gather_a = (A.flags & MOE_SCHED_GATHER_A) ? 1 : 0;
   MOE_TRY(launch_scatter(w.topk_idx, T, E, k, w.blk_base, w.perm, w.row_of, gather_a ? &w : nullptr, st));
   if (!gather_a)
     MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(A.x), w.row_of, T, d, k, w.x_perm, nsm, st));
@@ -365,7 +386,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   a.gate = w.topk_gate;
   a.out = static_cast<__nv_bfloat16*>(A.out);
   a.R = R; a.T = T; a.d = d; a.f = f; a.E = E; a.k = k;
-  a.G = G;
+  a.V = V;
   a.mgb = mgb;
   a.flags = A.flags;
   a.timeout_ns = (A.timeout_us > 0 ? (uint64_t)A.timeout_us : 2000000ull) * 1000ull;

@@ -57,14 +57,21 @@ constexpr int CONS_SLOTS = 16;    // at most this many tokens in flight per cons
 constexpr int MAX_NST = 6;        // pipeline depth of the CTA-pair variant
 constexpr int STAGE_AREA = 196608;  // shared memory of the operand ring (and the consumer's slots)
 
-// Per-variant tiling.  G = CTAs per MMA: G = 1 computes a 128x256 tile per CTA
-// (A: 128 rows, B: all 256 columns); G = 2 computes a 256x256 tile per CTA pair
-// with tcgen05 cta_group::2 (each CTA: 128 rows of A and 128 columns of B), so a
-// CTA streams 32 KB per 64-deep k-block instead of 48 KB.
-template <int G>
+// Tile variants, V:
+//   V = 1  one CTA per 128x256 tile (A: 128 rows, B: all 256 columns);
+//   V = 2  a CTA pair per 256x256 tile with tcgen05 cta_group::2 (each CTA: 128
+//          rows of A and 128 columns of B);
+//   V = 3  one CTA per 256x256 tile, as two 128-row MMAs (two A boxes, one B
+//          stage) into its two accumulators.
+// V = 2 and V = 3 stream 32 KB of operands per 128x256x64 of MMA work, V = 1 48 KB.
+template <int V>
 struct Cfg {
-  static constexpr int NBOX = G == 1 ? 4 : 2;                      // 64-column B boxes per CTA
-  static constexpr int STAGE = A_STAGE_BYTES + NBOX * B_BOX_BYTES;
+  static_assert(V >= 1 && V <= 3, "tile variant");
+  static constexpr int CTAS = V == 2 ? 2 : 1;                      // CTAs per tile
+  static constexpr int BANDS = V == 1 ? 1 : 2;                     // row bands per tile
+  static constexpr int ABOX = V == 3 ? 2 : 1;                      // 128-row A boxes per CTA
+  static constexpr int NBOX = V == 2 ? 2 : 4;                      // 64-column B boxes per CTA
+  static constexpr int STAGE = ABOX * A_STAGE_BYTES + NBOX * B_BOX_BYTES;
   static constexpr int NST = STAGE_AREA / STAGE;
   static_assert(NST <= MAX_NST && NST * STAGE == STAGE_AREA, "stage ring must fill the area");
 };
@@ -197,20 +204,27 @@ __device__ __forceinline__ float silu_mul(float a, float b) {
 // 0-63 the columns that the leader's B half supplies, lanes 64-127 (the same 64
 // rows) the peer's.  (The gathered-A path keeps full tiles, as does
 // MOE_SCHED_FULL_TILES.)
-template <int G>
+template <int V>
 __device__ __forceinline__ bool half_tile(const Item& it, const FfnArgs& a) {
-  return G == 2 && !a.gather && !(a.flags & MOE_SCHED_FULL_TILES) && it.rows <= BM;
+  return V == 2 && !a.gather && !(a.flags & MOE_SCHED_FULL_TILES) && it.rows <= BM;
 }
 
-// This CTA's rows of a row group: CTA `rank` of a G-CTA group owns band
-// band0+rank; in a half tile, rows 64*rank.. of band0.
+// This CTA's rows of a row group: CTA `rank` of a pair owns band band0+rank (in
+// a half tile, rows 64*rank.. of band0); a single CTA owns the whole group (V = 3:
+// up to two bands, band0 and band0+1).
 struct MyRows {
   int row0, rows, band;
 };
 
-template <int G>
+template <int V>
 __device__ __forceinline__ MyRows my_rows(const Item& it, uint32_t rank, bool half) {
   MyRows m;
+  if (V == 3) {
+    m.row0 = it.row0;
+    m.rows = min(2 * BM, it.rows);
+    m.band = it.band0;
+    return m;
+  }
   const int h = half ? BM / 2 : BM;
   m.row0 = it.row0 + (int)rank * h;
   m.rows = min(h, max(0, it.rows - (int)rank * h));
@@ -223,33 +237,35 @@ __device__ __forceinline__ MyRows my_rows(const Item& it, uint32_t rank, bool ha
 constexpr uint32_t BAND_UNIT = 2;
 
 // Arrive on a barrier that lives in the pair leader (local when this CTA leads).
-template <int G>
+template <int V>
 __device__ __forceinline__ void arrive_leader(uint64_t* bar, uint32_t rank) {
-  if (G == 1 || rank == 0) mbar_arrive(bar);
+  if (V != 2 || rank == 0) mbar_arrive(bar);
   else mbar_arrive_remote(mapa_shared(smem_u32(bar), 0));
 }
 
 // ------------------------------------------------------------ TMA producer ---
-// G == 1, or the pair leader: takes work items from the atomic queues and puts
+// A single CTA, or the pair leader: takes work items from the atomic queues and puts
 // them in the ring (the leader also writes them into its peer's ring over
 // distributed shared memory).  The peer reads items from its own ring.  Each CTA
 // then loads its own 128 rows of A and its share of B for every k-block; in a
 // pair the loads count on the leader's `full` barrier.
-// GEMM1's A rows are gathered straight from x (a.gather): the tile's 128 token
-// indices (one aligned 512-byte row of tok_band) are bulk-copied into shared
-// memory one work item ahead, and each k-block's A tile is 32 TMA gather4 loads
-// of 4 token rows x 64 columns into the same swizzled layout a tiled load gives.
-template <int G>
+// V = 3 loads two 128-row A boxes (one when the group holds a single band).
+// GEMM1's A rows are gathered straight from x (a.gather, V = 1 and 2): the
+// tile's 128 token indices (one aligned 512-byte row of tok_band) are
+// bulk-copied into shared memory one work item ahead, and each k-block's A tile
+// is 32 TMA gather4 loads of 4 token rows x 64 columns into the same swizzled
+// layout a tiled load gives.
+template <int V>
 __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
                          const CUtensorMap* tm_w3, const CUtensorMap* tm_a2,
                          const CUtensorMap* tm_w2, const FfnArgs& a, SmemCtl* ctl,
                          uint8_t* smem, uint32_t rank, bool run_g1, bool run_g2, int n1, int n2,
                          const volatile uint32_t* abort) {
-  using C = Cfg<G>;
+  using C = Cfg<V>;
   const Work& w = a.w;
   const int NT1 = a.f / BN1, NT2 = a.d / BN2;
   const uint64_t tmo = a.timeout_ns;
-  const bool leader = (G == 1) || rank == 0;
+  const bool leader = V != 2 || rank == 0;
   int stage = 0, slot = 0;
   uint32_t ph = 0, sph = 0;
   uint32_t pending = 0, pend_par = 0;   // stages with an issued fill, and its parity
@@ -278,9 +294,9 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
         const int t = (int)atomicAdd(&w.sync->q2, 1u);
         if (t < n2) it = decode_g2(w, t, NT2); else g2 = false;
       }
-      if (!wait_bar<G == 2>(&ctl->sempty[slot], sph ^ 1u, tmo, abort)) { set_error(w.status, W_SCHED_EMPTY); return false; }
+      if (!wait_bar<V == 2>(&ctl->sempty[slot], sph ^ 1u, tmo, abort)) { set_error(w.status, W_SCHED_EMPTY); return false; }
       ctl->ring[slot] = it;
-      if (G == 2) {
+      if (V == 2) {
         const uint4* src = reinterpret_cast<const uint4*>(&it);
         const uint32_t dst = mapa_shared(smem_u32(&ctl->ring[slot]), 1);
         st_cluster_v4(dst, src[0]);
@@ -291,18 +307,18 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
     } else {
       if (!wait_bar<true>(&ctl->sfull[slot], sph, tmo, abort)) { set_error(w.status, W_SCHED_FULL); return false; }
       it = ctl->ring[slot];
-      arrive_leader<G>(&ctl->sempty[slot], rank);
+      arrive_leader<V>(&ctl->sempty[slot], rank);
     }
     if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
     return true;
   };
   // Does this CTA gather indices for the item?  (GEMM1, gathered path, own rows)
   auto gathers = [&](const Item& it) {
-    return a.gather && it.kind == K_G1 && my_rows<G>(it, rank, false).rows > 0;
+    return a.gather && it.kind == K_G1 && my_rows<V>(it, rank, false).rows > 0;
   };
   auto fetch_indices = [&](const Item& it, int buf) {
     if (!gathers(it)) return;
-    const MyRows m = my_rows<G>(it, rank, false);
+    const MyRows m = my_rows<V>(it, rank, false);
     fence_proxy_async_shared();   // earlier generic reads of this buffer come first
     gpend |= 1u << buf;
     mbar_arrive_expect_tx(&ctl->gbar[buf], BM * 4);
@@ -319,8 +335,9 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
     fetch_indices(nxt, buf ^ 1);
     const bool is1 = cur.kind == K_G1;
     if (is1) ++n_g1; else ++n_g2;
-    const bool half = half_tile<G>(cur, a);
-    const MyRows m = my_rows<G>(cur, rank, half);
+    const bool half = half_tile<V>(cur, a);
+    const MyRows m = my_rows<V>(cur, rank, half);
+    const bool two = V == 3 && m.rows > BM;   // V = 3: the group's second band is present
     const bool gat = a.gather && is1;
     if (gat && m.rows > 0) {
       if (!wait_bar(&ctl->gbar[buf], (gph >> buf) & 1u, tmo, abort)) { set_error(w.status, W_STAGE_FULL); break; }
@@ -329,7 +346,8 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
     }
     if (!is1 && m.rows > 0) {
       // GEMM2 reads this CTA's h rows: every GEMM1 column block of its band must be stored.
-      if (!wait_count(&w.band_done1[m.band], BAND_UNIT * (uint32_t)NT1, tmo, abort)) {
+      if (!wait_count(&w.band_done1[m.band], BAND_UNIT * (uint32_t)NT1, tmo, abort) ||
+          (two && !wait_count(&w.band_done1[m.band + 1], BAND_UNIT * (uint32_t)NT1, tmo, abort))) {
         set_error(w.status, W_BAND1);
         break;
       }
@@ -337,28 +355,32 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
     }
     const int nk = (is1 ? a.d : a.f) / BK;
     for (int kb = 0; kb < nk; ++kb) {
-      if (!wait_bar<G == 2>(&ctl->empty[stage], ph ^ 1u, tmo, abort)) { set_error(w.status, W_STAGE_EMPTY); ok = false; break; }
+      if (!wait_bar<V == 2>(&ctl->empty[stage], ph ^ 1u, tmo, abort)) { set_error(w.status, W_STAGE_EMPTY); ok = false; break; }
       uint8_t* sa = smem + (size_t)stage * C::STAGE;
-      uint8_t* sb = sa + A_STAGE_BYTES;
+      uint8_t* sb = sa + C::ABOX * A_STAGE_BYTES;
       uint64_t* fb = &ctl->full[stage];
-      const uint32_t fbl = G == 2 ? mapa_shared(smem_u32(fb), 0) : 0u;
-      if (leader) mbar_arrive_expect_tx(fb, G * C::STAGE);   // a pair's leader expects both CTAs' bytes
+      const uint32_t fbl = V == 2 ? mapa_shared(smem_u32(fb), 0) : 0u;
+      // a pair's leader expects both CTAs' bytes; V = 3 without a second band
+      // loads one A box
+      if (leader)
+        mbar_arrive_expect_tx(fb, C::CTAS * C::STAGE - (V == 3 && !two ? A_STAGE_BYTES : 0));
       // A: 128 rows x 64 columns of x_perm (tiled) or of x (gathered); h for GEMM2
       if (gat) {
 #pragma unroll 8
         for (int q = 0; q < BM / 4; ++q) {
           const int4 tk = m.rows > 0 ? ctl->gidx[buf][q] : make_int4(0, 0, 0, 0);
-          if (G == 1) tma_gather4(sa + q * 512, tm_a1, fb, kb * BK, tk.x, tk.y, tk.z, tk.w);
+          if (V != 2) tma_gather4(sa + q * 512, tm_a1, fb, kb * BK, tk.x, tk.y, tk.z, tk.w);
           else tma_gather4_pair(sa + q * 512, tm_a1, fbl, kb * BK, tk.x, tk.y, tk.z, tk.w);
         }
-      } else if (G == 1) {
+      } else if (V != 2) {
         tma_load_2d(sa, is1 ? tm_a1 : tm_a2, fb, kb * BK, m.row0);
+        if (two) tma_load_2d(sa + A_STAGE_BYTES, is1 ? tm_a1 : tm_a2, fb, kb * BK, m.row0 + BM);
       } else {
         tma_load_2d_pair(sa, is1 ? tm_a1 : tm_a2, fbl, kb * BK, m.row0);
       }
       // B: 64-column atoms of W1/W3 (GEMM1) or W2 (GEMM2), K-rows kb*BK.., each
       // atom 64 K rows x 128 B, atom after atom (the MMA's leading-byte offset)
-      if (G == 1 && a.b_atoms) {
+      if (V != 2 && a.b_atoms) {
         // 4-D maps {64 columns, K, atom, expert}: one copy per operand
         const int k0 = kb * BK;
         if (is1) {
@@ -367,7 +389,7 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
         } else {
           tma_load_4d(sb, tm_w2, fb, 0, k0, cur.nt * (BN2 / 64), cur.expert);
         }
-      } else if (G == 1) {
+      } else if (V != 2) {
         if (is1) {
           tma_load_3d(sb, tm_w1, fb, cur.nt * BN1, kb * BK, cur.expert);
           tma_load_3d(sb + B_BOX_BYTES, tm_w1, fb, cur.nt * BN1 + 64, kb * BK, cur.expert);
@@ -415,7 +437,7 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
   for (int s = 0; s < C::NST; ++s) {
     if (!(pending & (1u << s))) continue;
     const uint32_t par = (pend_par >> s) & 1u;
-    if (leader) drained &= wait_bar<G == 2>(&ctl->full[s], par, tmo, nullptr);
+    if (leader) drained &= wait_bar<V == 2>(&ctl->full[s], par, tmo, nullptr);
     else drained &= wait_bar<true>(&ctl->empty[s], par, tmo, abort);
   }
   if (!drained) {
@@ -426,14 +448,18 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
 }
 
 // --------------------------------------------------------------- MMA issuer ---
-// One thread (G == 1: each CTA; G == 2: the pair leader) issues every MMA.
-template <int G>
+// One thread (a single CTA's, or the pair leader's) issues every MMA.
+// V = 1, 2: one accumulator per tile, alternating, so the epilogue of tile i
+// overlaps the main loop of tile i+1.  V = 3: both accumulators per tile, acc b
+// taking band b's 128 rows (A box b) against the same B stage; tile i+1's first
+// MMAs into acc 0 wait only for acc 0 of tile i to be drained, acc 1 for acc 1.
+template <int V>
 __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t tmem_base,
                          const volatile uint32_t* abort) {
-  using C = Cfg<G>;
+  using C = Cfg<V>;
   const uint64_t tmo = a.timeout_ns;
-  constexpr uint32_t idesc_full = idesc_bf16_f32(BM * G, 256, true);
-  constexpr uint32_t idesc_half = idesc_bf16_f32(BM, 256, true);   // G == 2 only
+  constexpr uint32_t idesc_full = idesc_bf16_f32(BM * C::CTAS, 256, true);
+  constexpr uint32_t idesc_half = idesc_bf16_f32(BM, 256, true);   // V == 2 only
   int stage = 0, slot = 0, acc = 0;
   uint32_t ph = 0, sph = 0, aph = 0;
   while (true) {
@@ -442,14 +468,46 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
     mbar_arrive(&ctl->sempty[slot]);
     if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
     if (it.kind == K_END) break;
-    if (!wait_bar<G == 2>(&ctl->tempty[acc], aph ^ 1u, tmo, abort)) { set_error(a.w.status, W_TMEM_EMPTY); break; }
-    tc_fence_after();
-    const uint32_t dt = tmem_base + (uint32_t)(acc * ACC_COLS);
-    const uint32_t idesc = half_tile<G>(it, a) ? idesc_half : idesc_full;
     const int nk = (it.kind == K_G1 ? a.d : a.f) / BK;
     bool ok = true;
+    if (V == 3) {
+      const bool two = it.rows > BM;
+      for (int kb = 0; kb < nk && ok; ++kb) {
+        if (!wait_bar(&ctl->full[stage], ph, tmo, abort)) { set_error(a.w.status, W_STAGE_FULL); ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + (size_t)stage * C::STAGE);
+        const uint32_t sb = sa + C::ABOX * A_STAGE_BYTES;
+        for (int b = 0; b < 2; ++b) {
+          // both accumulators' phases advance every tile, a one-band group's too
+          if (kb == 0) {
+            if (!wait_bar(&ctl->tempty[b], aph ^ 1u, tmo, abort)) { set_error(a.w.status, W_TMEM_EMPTY); ok = false; break; }
+            tc_fence_after();
+          }
+          if (b == 1 && !two) continue;
+          const uint32_t dt = tmem_base + (uint32_t)(b * ACC_COLS);
+#pragma unroll
+          for (int ks = 0; ks < BK / 16; ++ks) {
+            const uint64_t ad = smem_desc_sw128(sa + b * A_STAGE_BYTES + ks * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sb + ks * 2048, B_BOX_BYTES, 1024);
+            tc_mma_f16(dt, ad, bd, idesc_full, (kb | ks) != 0 ? 1u : 0u);
+          }
+        }
+        if (!ok) break;
+        tc_commit(&ctl->empty[stage]);
+        if (++stage == C::NST) { stage = 0; ph ^= 1u; }
+      }
+      if (!ok) break;
+      tc_commit(&ctl->tfull[0]);
+      tc_commit(&ctl->tfull[1]);
+      aph ^= 1u;
+      continue;
+    }
+    if (!wait_bar<V == 2>(&ctl->tempty[acc], aph ^ 1u, tmo, abort)) { set_error(a.w.status, W_TMEM_EMPTY); break; }
+    tc_fence_after();
+    const uint32_t dt = tmem_base + (uint32_t)(acc * ACC_COLS);
+    const uint32_t idesc = half_tile<V>(it, a) ? idesc_half : idesc_full;
     for (int kb = 0; kb < nk; ++kb) {
-      if (!wait_bar<G == 2>(&ctl->full[stage], ph, tmo, abort)) { set_error(a.w.status, W_STAGE_FULL); ok = false; break; }
+      if (!wait_bar<V == 2>(&ctl->full[stage], ph, tmo, abort)) { set_error(a.w.status, W_STAGE_FULL); ok = false; break; }
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + (size_t)stage * C::STAGE);
       const uint32_t sb = sa + A_STAGE_BYTES;
@@ -457,33 +515,86 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
       for (int ks = 0; ks < BK / 16; ++ks) {
         const uint64_t ad = smem_desc_sw128(sa + ks * 32, 16, 1024);
         const uint64_t bd = smem_desc_sw128(sb + ks * 2048, B_BOX_BYTES, 1024);
-        if (G == 1) tc_mma_f16(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+        if (V != 2) tc_mma_f16(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
         else tc_mma_f16_pair(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
       }
       // frees the smem stage (in both CTAs of a pair) once these MMAs finish
-      if (G == 1) tc_commit(&ctl->empty[stage]);
+      if (V != 2) tc_commit(&ctl->empty[stage]);
       else tc_commit_pair(&ctl->empty[stage], (uint16_t)0x3);
       if (++stage == C::NST) { stage = 0; ph ^= 1u; }
     }
     if (!ok) break;
     // accumulator ready for the epilogue (of both CTAs of a pair)
-    if (G == 1) tc_commit(&ctl->tfull[acc]);
+    if (V != 2) tc_commit(&ctl->tfull[acc]);
     else tc_commit_pair(&ctl->tfull[acc], (uint16_t)0x3);
     acc ^= 1;
     if (acc == 0) aph ^= 1u;
   }
   // Wait for every MMA this thread issued before TMEM can be released.
-  if (G == 1) tc_commit(&ctl->mma_done);
+  if (V != 2) tc_commit(&ctl->mma_done);
   else tc_commit_pair(&ctl->mma_done, (uint16_t)0x1);
   wait_bar(&ctl->mma_done, 0u, tmo, nullptr);
 }
 
 // ----------------------------------------------------------------- epilogue ---
+// This warp's 32 TMEM lanes of one accumulator -> registers -> bf16 -> 16-byte
+// global stores (only if `valid`), to destination row `row`:
+//   GEMM1: h[row][col0 + c] = silu(acc[c]) * acc[nc + c] for c < nc (nc = 128 for
+//          a full tile, 64 for a half tile's lane half),
+//   GEMM2: y[row][col0 + c] = acc[c] for c < nc (256, or 128 in a half tile).
+__device__ __forceinline__ void drain_acc(const FfnArgs& a, int kind, uint32_t tb, size_t row,
+                                          bool valid, int nc, int col0) {
+  if (kind == K_G1) {
+    uint4* dst = reinterpret_cast<uint4*>(a.h + row * a.f + col0);
+#pragma unroll 1
+    for (int c = 0; c < nc / 32; ++c) {
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tb + c * 32, ra);
+      tmem_ld32(tb + nc + c * 32, rb);
+      tmem_ld_wait();
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        pk[i] = pack_bf16x2(silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i])),
+                            silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1])));
+      if (valid) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      }
+    }
+    fence_proxy_async_global();   // h is read back by TMA in other CTAs
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(a.y + row * a.d + col0);
+#pragma unroll 1
+    for (int c = 0; c < nc / 32; ++c) {
+      uint32_t rr[32];
+      tmem_ld32(tb + c * 32, rr);
+      tmem_ld_wait();
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
+      if (valid) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      }
+    }
+  }
+}
+
+// Publish a stored band tile: fence, then add `units` to the band's counter with
+// release semantics (skipped for band 0's GEMM1 tiles under MOE_DBG_SKIP_FLAG_BAND).
+__device__ __forceinline__ void publish_band(const FfnArgs& a, int kind, int band, uint32_t units) {
+  if ((a.flags & MOE_DBG_SKIP_FLAG_BAND) && kind == K_G1 && band == 0) return;
+  __threadfence();
+  red_release_add(kind == K_G1 ? &a.w.band_done1[band] : &a.w.band_done2[band], units);
+}
+
 // Four warps per CTA; warp q (= warp id mod 4) owns TMEM lanes [32q, 32q+32), i.e.
-// rows 32q.. of this CTA's 128 rows.  TMEM -> registers -> bf16 -> 16-byte global
-// stores, masked to the band's valid rows; then the tile is published on the
-// band's counter.
-template <int G>
+// rows 32q.. of each accumulator's 128 rows.  Stores are masked to the band's
+// valid rows; then the tile is published on the band's counter.
+template <int V>
 __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base, uint32_t rank,
                               int warp, int lane, const volatile uint32_t* abort) {
   const Work& w = a.w;
@@ -495,71 +606,66 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
   while (true) {
     // Every lane waits; the warp proceeds only if all lanes saw the phase, so a
     // timeout never splits the warp before the .sync.aligned TMEM loads.
-    bool ok = __all_sync(0xffffffffu, wait_bar<G == 2>(&ctl->sfull[slot], sph, tmo, abort));
+    bool ok = __all_sync(0xffffffffu, wait_bar<V == 2>(&ctl->sfull[slot], sph, tmo, abort));
     if (!ok) { if (lane == 0) set_error(w.status, W_SCHED_FULL); break; }
     const Item it = ctl->ring[slot];
     __syncwarp();
-    if (lane == 0) arrive_leader<G>(&ctl->sempty[slot], rank);
+    if (lane == 0) arrive_leader<V>(&ctl->sempty[slot], rank);
     if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
     if (it.kind == K_END) break;
-    ok = __all_sync(0xffffffffu, wait_bar<G == 2>(&ctl->tfull[acc], aph, tmo, abort));
+    const int col0 = it.kind == K_G1 ? it.nt * BN1 : it.nt * BN2;
+    const int ncf = it.kind == K_G1 ? BN1 : BN2;   // columns a full tile stores
+    if (V == 3) {
+      // acc b holds band0+b: rows it.row0 + 128 b + row
+      for (int b = 0; b < 2 && ok; ++b) {
+        ok = __all_sync(0xffffffffu, wait_bar(&ctl->tfull[b], aph, tmo, abort));
+        if (!ok) { if (lane == 0) set_error(w.status, W_TMEM_FULL); break; }
+        tc_fence_after();
+        const int rb = min(BM, max(0, it.rows - b * BM));
+        if (rb > 0)
+          drain_acc(a, it.kind, tmem_base + (uint32_t)(b * ACC_COLS) + ((uint32_t)(q * 32) << 16),
+                    (size_t)(it.row0 + b * BM + row), row < rb, ncf, col0);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&ctl->tempty[b]);     // accumulator may be overwritten
+          mbar_arrive(&ctl->epi_done[b]);   // this warp's rows of band b are stored
+        }
+      }
+      if (!ok) break;
+      aph ^= 1u;
+      // publish both bands once the four warps stored them (each epi_done phase
+      // holds one tile's arrivals: a warp can run at most one tile ahead)
+      if (warp == 2 && lane == 0) {
+        for (int b = 0; b < 2; ++b) {
+          const bool stored = wait_bar(&ctl->epi_done[b], (eph >> b) & 1u, tmo, abort);
+          if (!stored) { set_error(w.status, W_DRAIN); break; }
+          if (it.rows > b * BM) publish_band(a, it.kind, it.band0 + b, BAND_UNIT);
+        }
+      }
+      eph ^= 3u;
+      __syncwarp();
+      continue;
+    }
+    ok = __all_sync(0xffffffffu, wait_bar<V == 2>(&ctl->tfull[acc], aph, tmo, abort));
     if (!ok) { if (lane == 0) set_error(w.status, W_TMEM_FULL); break; }
     tc_fence_after();
-    const bool half = half_tile<G>(it, a);
-    const MyRows m = my_rows<G>(it, rank, half);
+    const bool half = half_tile<V>(it, a);
+    const MyRows m = my_rows<V>(it, rank, half);
     const uint32_t tb = tmem_base + (uint32_t)(acc * ACC_COLS) + ((uint32_t)(q * 32) << 16);
     // full tile: lane `row` is row `row`, all N columns; half tile: lane `row` is
-    // row row % 64, and the N/2 columns of the B half row / 64 supplied
+    // row row % 64, and the N/2 columns of the B half row / 64 supplied (GEMM1:
+    // h columns nt*128 + 64*ch + [0,64) from accumulator columns [0,64) and
+    // [64,128); GEMM2: y columns nt*256 + 128*ch + [0,128))
     const int r = half ? (row & (BM / 2 - 1)) : row;
     const int ch = half ? (row >> 6) : 0;
-    const bool valid = r < m.rows;
-    if (it.kind == K_G1) {
-      // h columns: full tile nt*128 + [0,128) from W1 columns [0,128) and W3
-      // columns [128,256); half tile nt*128 + 64*ch + [0,64) from [0,64) and [64,128)
-      const int nh = half ? BN1 / 2 : BN1;
-      uint4* dst = reinterpret_cast<uint4*>(a.h + (size_t)(m.row0 + r) * a.f + it.nt * BN1 + ch * (BN1 / 2));
-#pragma unroll 1
-      for (int c = 0; c < nh / 32; ++c) {
-        uint32_t ra[32], rb[32];
-        tmem_ld32(tb + c * 32, ra);
-        tmem_ld32(tb + nh + c * 32, rb);
-        tmem_ld_wait();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i])),
-                              silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1])));
-        if (valid) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
-      }
-      fence_proxy_async_global();   // h is read back by TMA in other CTAs
-    } else {
-      // y columns: full tile nt*256 + [0,256); half tile nt*256 + 128*ch + [0,128)
-      const int ny = half ? BN2 / 2 : BN2;
-      uint4* dst = reinterpret_cast<uint4*>(a.y + (size_t)(m.row0 + r) * a.d + it.nt * BN2 + ch * (BN2 / 2));
-#pragma unroll 1
-      for (int c = 0; c < ny / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tb + c * 32, rr);
-        tmem_ld_wait();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
-        if (valid) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-        }
-      }
-    }
+    const int nc = half ? ncf / 2 : ncf;
+    drain_acc(a, it.kind, tb, (size_t)(m.row0 + r), r < m.rows, nc, col0 + ch * nc);
     tc_fence_before();
     __syncwarp();
     const int my_acc = acc;
     if (lane == 0) {
-      arrive_leader<G>(&ctl->tempty[my_acc], rank);   // accumulator may be overwritten
+      arrive_leader<V>(&ctl->tempty[my_acc], rank);   // accumulator may be overwritten
       mbar_arrive(&ctl->epi_done[my_acc]);             // this warp's rows of the tile are stored
     }
     acc ^= 1;
@@ -568,17 +674,12 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
     // warps' stores of the tile, then fences and bumps its band's counter with
     // release semantics.  A warp can run at most one tile ahead, and consecutive
     // tiles use different accumulators, so each epi_done phase holds one tile's
-    // arrivals only.
+    // arrivals only.  A half tile's band is published by both CTAs (even one with
+    // no valid rows), one unit each.
     if (warp == 2 && lane == 0) {
       const bool stored = wait_bar(&ctl->epi_done[my_acc], (eph >> my_acc) & 1u, tmo, abort);
-      const bool skip = (a.flags & MOE_DBG_SKIP_FLAG_BAND) && it.kind == K_G1 && m.band == 0;
       if (!stored) set_error(w.status, W_DRAIN);
-      else if ((half || m.rows > 0) && !skip) {
-        // a half tile's band is published by both CTAs (even one with no valid rows)
-        __threadfence();
-        red_release_add(it.kind == K_G1 ? &w.band_done1[m.band] : &w.band_done2[m.band],
-                        half ? BAND_UNIT / 2 : BAND_UNIT);
-      }
+      else if (half || m.rows > 0) publish_band(a, it.kind, m.band, half ? BAND_UNIT / 2 : BAND_UNIT);
     }
     eph ^= 1u << my_acc;
     __syncwarp();
@@ -812,7 +913,7 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
 }
 
 // ------------------------------------------------------------------- kernel ---
-template <int G>
+template <int V>
 __global__ void __launch_bounds__(FFN_THREADS, 1)
 ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_w1,
            const __grid_constant__ CUtensorMap tm_w3, const __grid_constant__ CUtensorMap tm_a2,
@@ -822,15 +923,16 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + (size_t)STAGE_AREA);
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = G == 2 ? cluster_ctarank() : 0u;
+  constexpr int CTAS = Cfg<V>::CTAS;
+  const uint32_t rank = V == 2 ? cluster_ctarank() : 0u;
 
   // prologue (touches nothing the previous kernel writes): barriers, TMEM, descriptors
   if (threadIdx.x == 0) {
     for (int i = 0; i < MAX_NST; ++i) { mbar_init(&ctl->full[i], 1); mbar_init(&ctl->empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&ctl->tfull[i], 1); mbar_init(&ctl->tempty[i], 4 * G); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&ctl->tfull[i], 1); mbar_init(&ctl->tempty[i], 4 * CTAS); }
     for (int i = 0; i < SCHED_DEPTH; ++i) {
       mbar_init(&ctl->sfull[i], 1);
-      mbar_init(&ctl->sempty[i], G == 1 ? 5 : 10);   // pair: leader MMA + 4 epi, peer TMA + 4 epi
+      mbar_init(&ctl->sempty[i], 5 * CTAS);   // MMA + 4 epi; a pair adds the peer's TMA + 4 epi
     }
     mbar_init(&ctl->epi_done[0], 4);
     mbar_init(&ctl->epi_done[1], 4);
@@ -846,12 +948,12 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
     tma_prefetch_desc(&tm_a2); tma_prefetch_desc(&tm_w2);
   }
   if (warp == 1) {
-    if (G == 1) tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+    if (V != 2) tmem_alloc(&ctl->tmem_base, TMEM_COLS);
     else tmem_alloc_pair(&ctl->tmem_base, TMEM_COLS);
     tc_fence_before();
   }
   __syncthreads();
-  if (G == 2) cluster_sync();   // both CTAs' barriers exist before any remote arrive
+  if (V == 2) cluster_sync();   // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
 
@@ -876,11 +978,11 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   if (run_g1 || run_g2) {
     if (warp == 0) {
       if (lane == 0)
-        role_tma<G>(&tm_a1, &tm_w1, &tm_w3, &tm_a2, &tm_w2, a, ctl, smem, rank, run_g1, run_g2, n1, n2, abort);
+        role_tma<V>(&tm_a1, &tm_w1, &tm_w3, &tm_a2, &tm_w2, a, ctl, smem, rank, run_g1, run_g2, n1, n2, abort);
     } else if (warp == 1) {
-      if (lane == 0 && rank == 0) role_mma<G>(a, ctl, smem, tmem_base, abort);
+      if (lane == 0 && rank == 0) role_mma<V>(a, ctl, smem, tmem_base, abort);
     } else {
-      role_epilogue<G>(a, ctl, tmem_base, rank, warp, lane, abort);
+      role_epilogue<V>(a, ctl, tmem_base, rank, warp, lane, abort);
     }
     __syncwarp();
   }
@@ -889,14 +991,14 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   if (threadIdx.x == 0 && (a.phase & PH_CONS)) atomicAdd(&a.w.sync->prod_done, 1u);
   // A pair's peer may still be read by the leader's MMAs until the leader is
   // done; nobody reuses the operand ring before both CTAs finished producing.
-  if (G == 2) cluster_sync();
+  if (V == 2) cluster_sync();
   if (do_consume) role_consumer(a, ctl, smem, nb, n_items, abort);
   __syncthreads();
   if (stamp && threadIdx.x == 0) my_stamps[3] = globaltimer();
-  if (G == 2) cluster_sync();
+  if (V == 2) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    if (G == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+    if (V != 2) tmem_dealloc(tmem_base, TMEM_COLS);
     else tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
@@ -945,21 +1047,21 @@ static bool encode4(CUtensorMap* m, const void* base, const cuuint64_t* dims,
 
 namespace {
 constexpr int MAX_DEV = 64;
-int g_configured[2][MAX_DEV] = {{0}};
-int g_grid[2][MAX_DEV] = {{0}};
+int g_configured[3][MAX_DEV] = {{0}};
+int g_grid[3][MAX_DEV] = {{0}};
 
-template <int G>
+template <int V>
 cudaError_t configure(int dev) {
   if (dev < 0 || dev >= MAX_DEV) return cudaErrorInvalidDevice;
-  if (g_configured[G - 1][dev]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(ffn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (g_configured[V - 1][dev]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(ffn_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)ffn_smem_bytes());
   if (e != cudaSuccess) return e;
   int nsm = 0;
   e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   int grid = nsm;
-  if (G == 2) {
+  if (V == 2) {
     // as many CTA pairs as can be resident at once (one CTA per SM)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(nsm & ~1));
@@ -978,20 +1080,29 @@ cudaError_t configure(int dev) {
     if (clusters < 1) return cudaErrorInvalidConfiguration;
     grid = 2 * min(clusters, nsm / 2);
   }
-  g_grid[G - 1][dev] = grid;
-  g_configured[G - 1][dev] = 1;
+  g_grid[V - 1][dev] = grid;
+  g_configured[V - 1][dev] = 1;
   return cudaSuccess;
+}
+
+cudaError_t configure_variant(int V, int dev) {
+  switch (V) {
+    case 1: return configure<1>(dev);
+    case 2: return configure<2>(dev);
+    case 3: return configure<3>(dev);
+  }
+  return cudaErrorInvalidValue;
 }
 }  // namespace
 
-cudaError_t ffn_grid(int G, int* grid) {
+cudaError_t ffn_grid(int V, int* grid) {
   *grid = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  e = G == 2 ? configure<2>(dev) : configure<1>(dev);
+  e = configure_variant(V, dev);
   if (e != cudaSuccess) return e;
-  *grid = g_grid[G - 1][dev];
+  *grid = g_grid[V - 1][dev];
   return cudaSuccess;
 }
 
@@ -999,7 +1110,8 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  e = a.G == 2 ? configure<2>(dev) : configure<1>(dev);
+  if (a.V == 3 && a.gather) return cudaErrorInvalidValue;   // gathered A rows: 128-row tiles only
+  e = configure_variant(a.V, dev);
   if (e != cudaSuccess) return e;
   CUtensorMap tm_a1, tm_w1, tm_w3, tm_a2, tm_w2;
   const cuuint64_t R = (cuuint64_t)a.R, d = (cuuint64_t)a.d, f = (cuuint64_t)a.f, E = (cuuint64_t)a.E;
@@ -1015,15 +1127,15 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
     const cuuint64_t dims[2] = {f, R}, st[1] = {f * 2};
     if (!encode(&tm_a2, a.h, 2, dims, st, BM)) return cudaErrorInvalidValue;
   }
-  // Single CTAs read the weights through 4-D maps {64 columns, K, 64-column
-  // atom, expert} with the atom stride 128 B, so that one box holds all the
-  // atoms of the CTA's tile, atom after atom: 2-3 copies per k-block instead of
-  // 5 (measured faster).  CTA pairs take 2 atoms per CTA and per operand through
+  // Single CTAs (V = 1, 3) read the weights through 4-D maps {64 columns, K,
+  // 64-column atom, expert} with the atom stride 128 B, so that one box holds
+  // all the atoms of the CTA's tile, atom after atom: 2-3 copies per k-block
+  // instead of 5 (measured faster).  CTA pairs take 2 atoms per CTA and per operand through
   // the 3-D maps {columns, K, expert}, one box per atom (a 4-D copy there
   // measured slower), as do single CTAs if the driver refuses the 4-D maps.
   FfnArgs args = a;
   args.b_atoms = 0;
-  if (a.G == 1 && !(a.flags & MOE_SCHED_B_PER_ATOM)) {
+  if (a.V != 2 && !(a.flags & MOE_SCHED_B_PER_ATOM)) {
     const cuuint64_t d1[4] = {64, d, f / 64, E}, s1[3] = {f * 2, 128, d * f * 2};
     const cuuint64_t d2[4] = {64, f, d / 64, E}, s2[3] = {d * 2, 128, f * d * 2};
     args.b_atoms = encode4(&tm_w1, a.W1, d1, s1, 2) && encode4(&tm_w3, a.W3, d1, s1, 2) &&
@@ -1042,7 +1154,7 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   cfg.dynamicSmemBytes = ffn_smem_bytes();
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
-  if (a.G == 2) {
+  if (a.V == 2) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
@@ -1057,7 +1169,8 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
     cfg.numAttrs = 1;
   }
   cfg.attrs = attr;
-  if (a.G == 2) return cudaLaunchKernelEx(&cfg, ffn_kernel<2>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+  if (a.V == 2) return cudaLaunchKernelEx(&cfg, ffn_kernel<2>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+  if (a.V == 3) return cudaLaunchKernelEx(&cfg, ffn_kernel<3>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
   return cudaLaunchKernelEx(&cfg, ffn_kernel<1>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
 }
 

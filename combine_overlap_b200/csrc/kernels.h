@@ -39,10 +39,11 @@ cudaError_t launch_colsum(const int32_t* blk_hist, int nblk, int E, int32_t* cou
 // Plan: counts/offsets (from blk_hist when nblk > 0, else from `offsets_in`),
 // per-block scatter bases, expert priority order, band table, tile counts,
 // zeroed sync counters and the producer/consumer split.
-// G = CTAs per MMA tile (1: 128-row tiles, 2: CTA pairs with 256-row tiles).
+// G = row bands per MMA tile (1: 128-row tiles; 2: 256-row tiles), cg = CTAs per
+// tile (consumer CTAs come in whole tiles' CTAs).
 cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
-                        int E, int k, int num_sms, int consumer_hint, int mgb, int G, int join,
-                        const CostModel& cm, cudaStream_t s);
+                        int E, int k, int num_sms, int consumer_hint, int mgb, int G, int cg,
+                        int join, const CostModel& cm, cudaStream_t s);
 // With a plan (w.bands etc. set), also fills w.tok_band, GEMM1's gather indices.
 cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const int32_t* blk_base,
                            int32_t* perm, int32_t* row_of, const Work* plan, cudaStream_t s);
@@ -71,7 +72,8 @@ struct FfnArgs {
   const float* gate;             // [T][k] (consumer role)
   __nv_bfloat16* out;            // [T][d] (consumer role)
   int R, T, d, f, E, k;
-  int G;                         // CTAs per MMA tile: 1 or 2 (cluster pair, cta_group::2)
+  int V;                         // tile variant: 1 one CTA per 128-row tile, 2 a CTA pair per
+                                 // 256-row tile (cta_group::2), 3 one CTA per 256-row tile
   int phase;                     // PH_* bits
   int join;                      // producers join the combine when the tile queue drains
   int mgb;
@@ -81,9 +83,9 @@ struct FfnArgs {
 };
 
 size_t ffn_smem_bytes();
-// CTAs the persistent kernel runs with for group size G; also sets the kernel's
-// shared-memory attribute for the current device.
-cudaError_t ffn_grid(int G, int* grid);
+// CTAs the persistent kernel runs with for tile variant V; also sets the
+// kernel's shared-memory attribute for the current device.
+cudaError_t ffn_grid(int V, int* grid);
 
 // The CUDA error behind the calling thread's latest MOE_ERR_CUDA (api.cu).
 void record_cuda_error(cudaError_t e);

@@ -111,7 +111,7 @@ extern "C" moe_status moe_permute_noalloc(const void* x, int T, int d, int E, in
   cm.max_consumers = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_hist(topk_idx, T, E, k, w.blk_hist, st);
-  if (e == cudaSuccess) e = launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, cm, st);
+  if (e == cudaSuccess) e = launch_plan(w, nblk, nullptr, T, BN2, BN1, E, k, nsm, 1, 1, 1, 1, 1, cm, st);
   if (e == cudaSuccess) e = launch_scatter(topk_idx, T, E, k, w.blk_base, perm, row_of, nullptr, st);
   if (e == cudaSuccess)
     e = launch_gather(static_cast<const __nv_bfloat16*>(x), row_of, T, d, k,

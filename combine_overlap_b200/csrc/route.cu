@@ -168,15 +168,15 @@ cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int32_t* b
 // routed row read once, every output row written once): C dedicated consumers
 // combine during GEMM2, and whatever is left is combined by all S CTAs once the
 // GEMM queue is empty (producers join).  Deterministic: same counts, same C.
-__device__ int choose_consumers(int S, int G, int cmin, long long R, int T, int d, int f,
+__device__ int choose_consumers(int S, int cg, int cmin, long long R, int T, int d, int f,
                                 const CostModel& cm) {
   const double F2 = 2.0 * (double)R * f * d;
   const double Bc = 2.0 * (double)R * d + 2.0 * (double)T * d;
   const double drain = fmin((double)S * cm.copy_bytes_per_sm, (double)cm.hbm_bytes);
   int best = cmin;
   double best_t = 1e300;
-  const int cmax = min(cm.max_consumers, S - G);
-  for (int C = cmin; C <= cmax; C += G) {
+  const int cmax = min(cm.max_consumers, S - cg);
+  for (int C = cmin; C <= cmax; C += cg) {
     const double t2 = F2 / ((double)(S - C) * cm.mma_flops_per_sm);
     const double left = fmax(0.0, Bc - (double)C * cm.copy_bytes_per_sm * t2);
     const double t = t2 + left / drain;
@@ -219,8 +219,8 @@ __device__ int warp_scan_smem(int* a, int n, int lane) {
 
 __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int32_t* offsets_in,
                                                     int T, int d, int f, int E, int k, int num_sms,
-                                                    int consumer_hint, int mgb, int G, int join,
-                                                    CostModel cm) {
+                                                    int consumer_hint, int mgb, int G, int cg,
+                                                    int join, CostModel cm) {
   pdl_trigger();
   pdl_wait();
   __shared__ int cnt[MAX_E];
@@ -330,10 +330,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
   if (tid == 0) {
     const long long R = offs[E];
     // without producers joining, at least one CTA group must consume from the start
-    const int cmin = join ? 0 : G;
-    int C = consumer_hint > 0 ? consumer_hint : choose_consumers(num_sms, G, cmin, R, T, d, f, cm);
-    C = G * cdiv(C, G);                         // consumers come in whole CTA groups
-    C = max(cmin, min(C, num_sms - G));         // and leave at least one producer group
+    const int cmin = join ? 0 : cg;
+    int C = consumer_hint > 0 ? consumer_hint : choose_consumers(num_sms, cg, cmin, R, T, d, f, cm);
+    C = cg * cdiv(C, cg);                       // consumers come in whole CTA groups
+    C = max(cmin, min(C, num_sms - cg));        // and leave at least one producer group
     Status st;
     st.code = ST_OK;
     st.consumer_sms = C;
@@ -385,10 +385,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
 }
 
 cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
-                        int E, int k, int num_sms, int consumer_hint, int mgb, int G, int join,
-                        const CostModel& cm, cudaStream_t s) {
+                        int E, int k, int num_sms, int consumer_hint, int mgb, int G, int cg,
+                        int join, const CostModel& cm, cudaStream_t s) {
   return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, w, nblk, offsets_in, T, d, f, E, k, num_sms,
-                    consumer_hint, mgb, G, join, cm);
+                    consumer_hint, mgb, G, cg, join, cm);
 }
 
 // ---------------------------------------------------------------- scatter ---

@@ -33,6 +33,7 @@ SCHED_GATHER_A = 0x10
 SCHED_CTA_PAIR = 0x20
 SCHED_B_PER_ATOM = 0x40
 SCHED_FULL_TILES = 0x80
+SCHED_WIDE_CTA = 0x100
 
 
 class MoEError(RuntimeError):
@@ -72,6 +73,8 @@ _lib.moe_get_status.argtypes = [_P, _P, ctypes.POINTER(_I), ctypes.POINTER(_I)]
 _lib.moe_status_string.argtypes = [_I]
 _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_num_sms.restype = _I
+_lib.moe_tile_variant.argtypes = [_I, _I, _I, _I, ctypes.c_uint]
+_lib.moe_tile_variant.restype = _I
 _lib.moe_last_cuda_error.restype = _I
 _lib.moe_cuda_error_string.argtypes = [_I]
 _lib.moe_cuda_error_string.restype = ctypes.c_char_p
@@ -96,6 +99,15 @@ def declared_symbols() -> list[str]:
 
 def status_string(code: int) -> str:
     return _lib.moe_status_string(int(code)).decode()
+
+
+TILE_VARIANTS = {1: "128x256 per CTA", 2: "256x256 per CTA pair (cta_group::2)",
+                 3: "256x256 per CTA (two 128-row MMAs)"}
+
+
+def tile_variant(T: int, f: int, E: int, k: int, flags: int = 0) -> int:
+    """The MMA tile variant the library picks for this shape and flags (1, 2, 3)."""
+    return int(_lib.moe_tile_variant(T, f, E, k, int(flags)))
 
 
 def last_cuda_error() -> int:

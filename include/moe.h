@@ -76,10 +76,11 @@ typedef enum {
 #define MOE_SCHED_ONE_CTA      0x4u  /* force 128-row MMA tiles on single CTAs          */
 #define MOE_SCHED_CTA_PAIR     0x20u /* force 256-row MMA tiles on CTA pairs (tcgen05
                                         cta_group::2); an expert's odd last row band runs
-                                        as a 128-row half tile.  Without either flag the
-                                        call picks pairs when T*k/E >= 512 and f >= 8192,
-                                        else single CTAs (measured on B200).  ONE_CTA
-                                        wins if both are set */
+                                        as a 128-row half tile.  Without a tile flag the
+                                        call picks 256-row tiles on single CTAs
+                                        (MOE_SCHED_WIDE_CTA) when T*k/E >= 256, else
+                                        128-row tiles (measured on B200).  ONE_CTA wins
+                                        over CTA_PAIR, CTA_PAIR over WIDE_CTA */
 #define MOE_SCHED_B_PER_ATOM   0x40u /* single-CTA tiles load each 64-column atom of the
                                         weight tiles with a TMA copy of its own (3-D maps),
                                         as CTA pairs always do, instead of one 4-D copy
@@ -87,6 +88,11 @@ typedef enum {
 #define MOE_SCHED_FULL_TILES   0x80u /* CTA pairs run an expert's odd last row band as a
                                         full 256-row tile (half of it masked) instead of a
                                         128-row half tile (M=128 cta_group::2 MMA) */
+#define MOE_SCHED_WIDE_CTA     0x100u /* force 256-row MMA tiles on single CTAs: two
+                                        128-row MMAs per K step share one B stage and
+                                        fill the CTA's two accumulators (an expert's odd
+                                        last band uses the first only).  Not with
+                                        MOE_SCHED_GATHER_A (MOE_ERR_UNSUPPORTED) */
 
 typedef struct {
   int T, d, f, E, k;        /* tokens, d_model, d_ff, experts, top-k                */
@@ -212,6 +218,12 @@ moe_status moe_debug_band_stamps(void* ws, void* stream, uint64_t* host_out, int
 
 /* Static English description of a status code. */
 const char* moe_status_string(moe_status s);
+
+/* The MMA tile variant moe_layer_forward and moe_grouped_ffn use for this
+ * shape and these flags (a host query, no device work): 1 = 128-row tiles on
+ * single CTAs, 2 = 256-row tiles on CTA pairs (cta_group::2), 3 = 256-row tiles
+ * on single CTAs; 0 for a non-positive size. */
+int moe_tile_variant(int T, int f, int E, int k, unsigned flags);
 
 /* The cudaError_t value behind the calling thread's most recent MOE_ERR_CUDA
  * from any entry point (a launch refused, a device fault surfacing at a launch

@@ -1,8 +1,9 @@
 """Steps (c1)+(c2), the grouped SwiGLU expert FFN on tcgen05, against the oracle
 on the same permuted rows: y within 2e-2 * max|ref|.  Shapes span several
 row bands per expert, ragged last bands, near-empty and empty experts, a single
-row, and several column tiles of both GEMMs -- each in both tile variants:
-single CTAs and CTA pairs with half tiles."""
+row, and several column tiles of both GEMMs -- each in every tile variant:
+128-row tiles on single CTAs, 256-row tiles on CTA pairs (with half tiles) and
+256-row tiles on single CTAs."""
 import numpy as np
 import pytest
 import torch
@@ -24,7 +25,7 @@ CASES = [
     synth.small("many_bands", 1100, 256, 256, 4, 2, "zipf"),   # several full pair groups per expert
 ]
 
-VARIANTS = {"one_cta": moe.SCHED_ONE_CTA, "cta_pair": moe.SCHED_CTA_PAIR}
+VARIANTS = {"one_cta": moe.SCHED_ONE_CTA, "cta_pair": moe.SCHED_CTA_PAIR, "wide_cta": moe.SCHED_WIDE_CTA}
 
 
 def _run(orc, wl, w_std=0.02, flags=0):

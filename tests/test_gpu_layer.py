@@ -71,10 +71,18 @@ def test_layer_small(orc, wl):
     for kw in (dict(), dict(consumer_sms=1), dict(consumer_sms=5, mgb=2)):
         ovl1, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=one | kw.pop("flags", 0), **kw)
         assert np.array_equal(gu.host(ovl1), gu.host(seq1)), f"one-CTA overlapped {kw} differs"
-    # the default picks pairs when T*k/E >= 512 and d_ff >= 8192, else single CTAs
+    # 256-row tiles on single CTAs: per band the same MMA shape and K order as the
+    # 128-row tiles, so the same bits, in both modes
+    wide = moe.SCHED_WIDE_CTA
+    for mode, kw in ((moe.MODE_SEQUENTIAL, dict()), (moe.MODE_OVERLAPPED, dict()),
+                     (moe.MODE_OVERLAPPED, dict(consumer_sms=3, mgb=2))):
+        out3, _, _ = _forward(inp, wl, ws, mode, flags=wide, **kw)
+        assert np.array_equal(gu.host(out3), gu.host(seq1)), f"wide-CTA tiles {mode} {kw} differ"
+    # the default picks single-CTA tiles of 256 rows (T*k/E >= 256) or 128 rows:
+    # either way the bits of the 128-row variant
     dflt, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED)
-    expect = seq_bits if wl.T * wl.k >= 512 * wl.E and wl.f >= 8192 else gu.host(seq1)
-    assert np.array_equal(gu.host(dflt), expect)
+    assert moe.tile_variant(wl.T, wl.f, wl.E, wl.k) == (3 if wl.T * wl.k >= 256 * wl.E else 1)
+    assert np.array_equal(gu.host(dflt), gu.host(seq1))
     # GEMM1 reading its A rows with TMA gather4 from x instead of x_perm: same
     # arithmetic on the same rows, so the same bits, in both tile variants;
     # and single CTAs loading the weight tiles one 64-column atom per copy (3-D
@@ -100,15 +108,18 @@ def test_layer_repeat_bitwise():
 
 FULL = ["mixtral", "fine_grained", "imbalanced", "sweep_T512_hot", "sweep_T2048_uniform",
         "sweep_T8192_zipf", "sweep_T32768_uniform"]
-# (workload, flags): every layer in its default variant (CTA pairs on the
-# Mixtral-shaped layer, single CTAs elsewhere), and the other variant on two
-FULL_CASES = [(n, 0) for n in FULL] + [("mixtral", 0x4), ("fine_grained", 0x20)]
+# (workload, flags): every layer in its default variant (256-row single-CTA
+# tiles from 256 rows per expert up, 128-row tiles below), and the other variants
+# on a few
+FULL_CASES = [(n, 0) for n in FULL] + [("mixtral", 0x4), ("mixtral", 0x20), ("fine_grained", 0x20),
+                                        ("sweep_T512_hot", 0x100)]
 
 
 @pytest.mark.parametrize("name,flags", FULL_CASES,
-                         ids=[f"{n}-{ {0: 'default', 0x4: 'one', 0x20: 'pair'}[f]}" for n, f in FULL_CASES])
+                         ids=[f"{n}-{ {0: 'default', 0x4: 'one', 0x20: 'pair', 0x100: 'wide'}[f]}"
+                              for n, f in FULL_CASES])
 def test_layer_full_size_sampled(orc, name, flags):
-    assert flags in (0, moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR)
+    assert flags in (0, moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR, moe.SCHED_WIDE_CTA)
     wl = synth.WORKLOADS[name]
     orc.set_threads(os.cpu_count() or 1)
     inp = gu.inputs(wl)
@@ -135,11 +146,11 @@ def test_layer_full_size_sampled(orc, name, flags):
 
 
 def _check_variants(orc, wl, inp):
-    """Both tile variants against the oracle, and overlapped == sequential in each."""
+    """Every tile variant against the oracle, and overlapped == sequential in each."""
     ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
     ref = orc.forward(gu.host(inp["x"]), gu.host(inp["logits"]), gu.host(inp["W1"]),
                       gu.host(inp["W3"]), gu.host(inp["W2"]), wl.k)
-    for fl in (moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR):
+    for fl in (moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR, moe.SCHED_WIDE_CTA):
         seq, extra, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL, flags=fl)
         assert np.array_equal(gu.host(extra["topk_idx"]), ref["topk_idx"])
         assert np.array_equal(gu.host(extra["counts"]), ref["counts"])
@@ -165,3 +176,13 @@ def test_layer_every_token_one_expert(orc, k):
     inp = gu.inputs(wl)
     inp["logits"][:, 3] += 50.0
     _check_variants(orc, wl, inp)
+
+
+def test_wide_tiles_refuse_gathered_rows():
+    # GEMM1's gathered-row path loads 128-row tiles only
+    wl = synth.WORKLOADS["tiny"]
+    inp = gu.inputs(wl)
+    ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
+    with pytest.raises(moe.MoEError) as e:
+        _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=moe.SCHED_WIDE_CTA | moe.SCHED_GATHER_A)
+    assert e.value.code == moe.MOE_ERR_UNSUPPORTED
