@@ -22,7 +22,7 @@ constexpr int A_STAGE_BYTES = BM * BK * 2;          // 16 KiB
 constexpr int B_BOX_BYTES = BK * 64 * 2;            // one 64x64 bf16 box, 8 KiB
 constexpr int B_STAGE_BYTES = 4 * B_BOX_BYTES;      // 32 KiB
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-constexpr int FFN_THREADS = 192;                    // warp0 TMA, warp1 MMA, warps2-5 epilogue
+constexpr int FFN_THREADS = 320;                    // warp0 TMA, warp1 MMA, warps2-9 epilogue
 constexpr int SCHED_DEPTH = 4;
 
 constexpr int ROUTE_TOK = 32;   // tokens per route / scatter block

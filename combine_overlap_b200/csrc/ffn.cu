@@ -19,23 +19,27 @@
 // once the GEMM tile queue is empty.
 //
 // B200 mapping (differs from the paper's A100 CUTLASS/NVSHMEM kernels):
-//   * one launch of one CTA per SM (G = 1: a cooperative launch; G = 2: a
+//   * one launch of one CTA per SM (V = 1, 3: a cooperative launch; V = 2: a
 //     cluster launch of as many pairs as can be resident at once), each CTA
 //     taking tiles from an atomic work queue in priority order instead of a
 //     fixed stride;
 //   * per CTA: warp 0 = tile scheduler + TMA producer, warp 1 = TMEM allocator
-//     + single-thread tcgen05.mma issuer, warps 2-5 = epilogue (TMEM -> registers
-//     -> bf16 -> global), a 192 KB smem operand ring, two 256-column TMEM
-//     accumulators so the epilogue of one tile overlaps the main loop of the next;
-//   * two variants, G = CTAs per MMA, chosen per call by the host: G = 1, one
-//     CTA per 128-row tile (weight tiles in one 4-D TMA copy per operand); G = 2,
-//     a cluster pair per 256-row tile with tcgen05 cta_group::2 -- the leader
-//     issues the MMAs, each CTA loads its 128 rows of A and half of B (no
-//     multicast), work items are mirrored into the peer over DSMEM, and an
-//     expert's odd last band runs as an M=128 half tile;
-//   * GEMM1 tile: 128*G rows x 128 h-columns; one N=256 MMA accumulates x*W1 and
-//     x*W3 side by side (the B tile holds the W1 and W3 column blocks), and the
-//     epilogue applies silu(a)*b;  GEMM2 tile: 128*G rows x 256 y-columns;
+//     + single-thread tcgen05.mma issuer, warps 2-9 = epilogue (TMEM -> registers
+//     -> bf16 -> global, two warps per TMEM lane quadrant), a 192 KB smem operand
+//     ring and two 256-column TMEM accumulators;
+//   * three tile variants V, chosen per call by the host: V = 1, one CTA per
+//     128-row tile; V = 2, a cluster pair per 256-row tile with tcgen05
+//     cta_group::2 -- the leader issues the MMAs, each CTA loads its 128 rows of
+//     A and half of B (no multicast), work items are mirrored into the peer over
+//     DSMEM, and an expert's odd last band runs as an M=128 half tile; V = 3, one
+//     CTA per 256-row tile as two 128-row MMAs per K step into its two
+//     accumulators.  V = 1 and 2 alternate the accumulators between tiles, so the
+//     epilogue of one tile overlaps the main loop of the next; single CTAs read
+//     their weight tiles with one 4-D TMA copy per operand;
+//   * GEMM1 tile: 128 or 256 rows x 128 h-columns; one N=256 MMA accumulates
+//     x*W1 and x*W3 side by side (the B tile holds the W1 and W3 column blocks),
+//     and the epilogue applies silu(a)*b;  GEMM2 tile: 128 or 256 rows x 256
+//     y-columns;
 //   * A (x_perm or h) is K-major, W is stored [K][N] (N-major): both are read
 //     by TMA with 128-byte swizzle and fed to tcgen05 as K-major / MN-major
 //     operands, so the weights need no repacking;
@@ -89,7 +93,7 @@ struct SmemCtl {
   uint64_t tempty[2];            // accumulator drained by every epilogue warp (pair: on the leader)
   uint64_t sfull[SCHED_DEPTH];   // a work item is in the ring slot
   uint64_t sempty[SCHED_DEPTH];  // every role read the slot (pair: on the leader)
-  uint64_t epi_done[2];          // per accumulator: this CTA's four epilogue warps stored the tile
+  uint64_t epi_done[2];          // per accumulator: this CTA's epilogue warps stored the tile
   uint64_t mma_done;
   uint64_t cfull[CONS_SLOTS];    // consumer ring: a token's k expert rows landed in the slot
   uint64_t cempty[CONS_SLOTS];   // consumer ring: the slot's token is reduced and stored
@@ -537,17 +541,24 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
 }
 
 // ----------------------------------------------------------------- epilogue ---
-// This warp's 32 TMEM lanes of one accumulator -> registers -> bf16 -> 16-byte
-// global stores (only if `valid`), to destination row `row`:
-//   GEMM1: h[row][col0 + c] = silu(acc[c]) * acc[nc + c] for c < nc (nc = 128 for
-//          a full tile, 64 for a half tile's lane half),
-//   GEMM2: y[row][col0 + c] = acc[c] for c < nc (256, or 128 in a half tile).
+constexpr int EPI_WARPS = FFN_THREADS / 32 - 2;   // warps 2.. : two per TMEM lane quadrant
+static_assert(EPI_WARPS == 8, "the epilogue splits each accumulator's columns between two warps");
+
+// This warp's 32 TMEM lanes of one accumulator, columns [c0, c1) (multiples of
+// 32) -> registers -> bf16 -> 16-byte global stores (only if `valid`), to
+// destination row `row`:
+//   GEMM1: h[row][col0 + c] = silu(acc[c]) * acc[nc + c] (nc = 128 for a full
+//          tile, 64 for a half tile's lane half),
+//   GEMM2: y[row][col0 + c] = acc[c] (nc = 256, or 128 in a half tile).
+// GEMM1's h rows are read back by TMA (async proxy) in other CTAs: the caller
+// fences them (fence.proxy.async) after releasing the accumulator and before
+// the tile is published.
 __device__ __forceinline__ void drain_acc(const FfnArgs& a, int kind, uint32_t tb, size_t row,
-                                          bool valid, int nc, int col0) {
+                                          bool valid, int nc, int col0, int c0, int c1) {
   if (kind == K_G1) {
     uint4* dst = reinterpret_cast<uint4*>(a.h + row * a.f + col0);
 #pragma unroll 1
-    for (int c = 0; c < nc / 32; ++c) {
+    for (int c = c0 / 32; c < c1 / 32; ++c) {
       uint32_t ra[32], rb[32];
       tmem_ld32(tb + c * 32, ra);
       tmem_ld32(tb + nc + c * 32, rb);
@@ -563,11 +574,10 @@ __device__ __forceinline__ void drain_acc(const FfnArgs& a, int kind, uint32_t t
           dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
     }
-    fence_proxy_async_global();   // h is read back by TMA in other CTAs
   } else {
     uint4* dst = reinterpret_cast<uint4*>(a.y + row * a.d + col0);
 #pragma unroll 1
-    for (int c = 0; c < nc / 32; ++c) {
+    for (int c = c0 / 32; c < c1 / 32; ++c) {
       uint32_t rr[32];
       tmem_ld32(tb + c * 32, rr);
       tmem_ld_wait();
@@ -591,15 +601,17 @@ __device__ __forceinline__ void publish_band(const FfnArgs& a, int kind, int ban
   red_release_add(kind == K_G1 ? &a.w.band_done1[band] : &a.w.band_done2[band], units);
 }
 
-// Four warps per CTA; warp q (= warp id mod 4) owns TMEM lanes [32q, 32q+32), i.e.
-// rows 32q.. of each accumulator's 128 rows.  Stores are masked to the band's
-// valid rows; then the tile is published on the band's counter.
+// Eight warps per CTA; warp w reads TMEM lanes [32q, 32q+32) with q = w mod 4,
+// i.e. rows 32q.. of each accumulator's 128 rows, and half of the accumulator's
+// columns, hc = (w - 2) / 4.  Stores are masked to the band's valid rows; then
+// the tile is published on the band's counter.
 template <int V>
 __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base, uint32_t rank,
                               int warp, int lane, const volatile uint32_t* abort) {
   const Work& w = a.w;
   const uint64_t tmo = a.timeout_ns;
   const int q = warp & 3;                 // TMEM lane quadrant this warp may read
+  const int hc = (warp - 2) >> 2;         // which half of the columns
   const int row = q * 32 + lane;
   int slot = 0, acc = 0;
   uint32_t sph = 0, aph = 0, eph = 0;   // eph: one parity bit per accumulator
@@ -624,17 +636,18 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
         const int rb = min(BM, max(0, it.rows - b * BM));
         if (rb > 0)
           drain_acc(a, it.kind, tmem_base + (uint32_t)(b * ACC_COLS) + ((uint32_t)(q * 32) << 16),
-                    (size_t)(it.row0 + b * BM + row), row < rb, ncf, col0);
+                    (size_t)(it.row0 + b * BM + row), row < rb, ncf, col0, hc * ncf / 2,
+                    (hc + 1) * ncf / 2);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&ctl->tempty[b]);     // accumulator may be overwritten
-          mbar_arrive(&ctl->epi_done[b]);   // this warp's rows of band b are stored
-        }
+        if (lane == 0) mbar_arrive(&ctl->tempty[b]);   // accumulator may be overwritten
+        if (it.kind == K_G1) fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->epi_done[b]);  // this warp's rows of band b are stored
       }
       if (!ok) break;
       aph ^= 1u;
-      // publish both bands once the four warps stored them (each epi_done phase
+      // publish both bands once the epilogue warps stored them (each epi_done phase
       // holds one tile's arrivals: a warp can run at most one tile ahead)
       if (warp == 2 && lane == 0) {
         for (int b = 0; b < 2; ++b) {
@@ -660,17 +673,18 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
     const int r = half ? (row & (BM / 2 - 1)) : row;
     const int ch = half ? (row >> 6) : 0;
     const int nc = half ? ncf / 2 : ncf;
-    drain_acc(a, it.kind, tb, (size_t)(m.row0 + r), r < m.rows, nc, col0 + ch * nc);
+    drain_acc(a, it.kind, tb, (size_t)(m.row0 + r), r < m.rows, nc, col0 + ch * nc, hc * nc / 2,
+              (hc + 1) * nc / 2);
     tc_fence_before();
     __syncwarp();
     const int my_acc = acc;
-    if (lane == 0) {
-      arrive_leader<V>(&ctl->tempty[my_acc], rank);   // accumulator may be overwritten
-      mbar_arrive(&ctl->epi_done[my_acc]);             // this warp's rows of the tile are stored
-    }
+    if (lane == 0) arrive_leader<V>(&ctl->tempty[my_acc], rank);   // accumulator may be overwritten
+    if (it.kind == K_G1) fence_proxy_async_global();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->epi_done[my_acc]);            // this warp's rows are stored
     acc ^= 1;
     if (acc == 0) aph ^= 1u;
-    // Publish the tile: one thread waits (bounded) for this CTA's four epilogue
+    // Publish the tile: one thread waits (bounded) for this CTA's epilogue
     // warps' stores of the tile, then fences and bumps its band's counter with
     // release semantics.  A warp can run at most one tile ahead, and consecutive
     // tiles use different accumulators, so each epi_done phase holds one tile's
@@ -695,7 +709,7 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
 //    (st.release of t+1 into an allocated entry).
 //  * COMBINE: up to S ready tokens from the queue.  Their k expert rows are
 //    streamed into a shared-memory slot ring with cp.async.bulk by one thread,
-//    and warps 1-5 each reduce a column slice of every token in fp32, slot order
+//    and warps 1.. each reduce a column slice of every token in fp32, slot order
 //    (the arithmetic of combine_token_warp, so both modes agree bit for bit),
 //    storing out[t] with 16-byte stores.
 // Splitting arrival from reduction lets every consuming CTA share the tokens
@@ -929,13 +943,13 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   // prologue (touches nothing the previous kernel writes): barriers, TMEM, descriptors
   if (threadIdx.x == 0) {
     for (int i = 0; i < MAX_NST; ++i) { mbar_init(&ctl->full[i], 1); mbar_init(&ctl->empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&ctl->tfull[i], 1); mbar_init(&ctl->tempty[i], 4 * CTAS); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&ctl->tfull[i], 1); mbar_init(&ctl->tempty[i], EPI_WARPS * CTAS); }
     for (int i = 0; i < SCHED_DEPTH; ++i) {
       mbar_init(&ctl->sfull[i], 1);
-      mbar_init(&ctl->sempty[i], 5 * CTAS);   // MMA + 4 epi; a pair adds the peer's TMA + 4 epi
+      mbar_init(&ctl->sempty[i], (1 + EPI_WARPS) * CTAS);   // MMA + epilogue; a pair adds the peer's TMA + epilogue
     }
-    mbar_init(&ctl->epi_done[0], 4);
-    mbar_init(&ctl->epi_done[1], 4);
+    mbar_init(&ctl->epi_done[0], EPI_WARPS);
+    mbar_init(&ctl->epi_done[1], EPI_WARPS);
     mbar_init(&ctl->mma_done, 1);
     mbar_init(&ctl->gbar[0], 1);
     mbar_init(&ctl->gbar[1], 1);
