@@ -86,6 +86,9 @@ struct __align__(16) Item {
   int kind, group, nt, expert, row0, rows, band0, pad;   // rows: valid rows of the whole group
 };
 
+constexpr int EPI_WARPS = FFN_THREADS / 32 - 2;   // warps 2.. : two per TMEM lane quadrant
+constexpr int OSTAGE_ROW = 80;                    // staged bytes per row: 64 of data + 16 of pad
+
 struct SmemCtl {
   uint64_t full[MAX_NST];        // operands of a stage landed (pair: counted on the leader)
   uint64_t empty[MAX_NST];       // the MMAs reading a stage finished
@@ -107,12 +110,15 @@ struct SmemCtl {
   int ctok[BM];                  // ... and which,
   int crow[BM][MAX_K];           // ... their k expert rows
   float cgate[BM][MAX_K];        // ... and their k gates (staged once, read by every warp)
+  // epilogue: per warp, 32 rows x 32 bf16 columns on their way to global memory
+  alignas(16) uint8_t ostage[EPI_WARPS][32 * OSTAGE_ROW];
 };
 
 static_assert(offsetof(SmemCtl, ring) % 16 == 0, "ring items must be 16-byte aligned");
 static_assert(sizeof(Item) == 32, "an item is two 16-byte stores");
 
 size_t ffn_smem_bytes() { return 1024 + (size_t)STAGE_AREA + sizeof(SmemCtl); }
+static_assert(1024 + STAGE_AREA + sizeof(SmemCtl) <= 227 * 1024, "over the 227 KB per-CTA limit");
 
 __device__ __forceinline__ void set_error(Status* st, uint32_t where) {
   if (atomicCAS(&st->code, (uint32_t)ST_OK, (uint32_t)ST_TIMEOUT) == (uint32_t)ST_OK) {
@@ -541,22 +547,46 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
 }
 
 // ----------------------------------------------------------------- epilogue ---
-constexpr int EPI_WARPS = FFN_THREADS / 32 - 2;   // warps 2.. : two per TMEM lane quadrant
 static_assert(EPI_WARPS == 8, "the epilogue splits each accumulator's columns between two warps");
 
 // This warp's 32 TMEM lanes of one accumulator, columns [c0, c1) (multiples of
-// 32) -> registers -> bf16 -> 16-byte global stores (only if `valid`), to
-// destination row `row`:
+// 32) -> registers -> bf16 -> global memory, rows `row` of the lanes whose
+// `valid` is set (the warp's lanes hold consecutive rows):
 //   GEMM1: h[row][col0 + c] = silu(acc[c]) * acc[nc + c] (nc = 128 for a full
 //          tile, 64 for a half tile's lane half),
 //   GEMM2: y[row][col0 + c] = acc[c] (nc = 256, or 128 in a half tile).
+// Each 32-column chunk (64 bytes per row) goes through the warp's staging tile
+// in shared memory, so that a store instruction writes 8 rows x 64 contiguous
+// bytes instead of 32 rows x 16.
 // GEMM1's h rows are read back by TMA (async proxy) in other CTAs: the caller
 // fences them (fence.proxy.async) after releasing the accumulator and before
 // the tile is published.
+__device__ __forceinline__ void store_chunk(uint8_t* ost, const uint32_t (&pk)[16], int lane,
+                                            unsigned vmask, __nv_bfloat16* base_row0,
+                                            size_t ld, int col) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    *reinterpret_cast<uint4*>(ost + lane * OSTAGE_ROW + v * 16) =
+        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int r = (lane >> 2) + 8 * v;            // row of the warp this lane writes
+    const uint4 val = *reinterpret_cast<const uint4*>(ost + r * OSTAGE_ROW + (lane & 3) * 16);
+    if ((vmask >> r) & 1u)
+      *reinterpret_cast<uint4*>(base_row0 + (size_t)r * ld + col + (lane & 3) * 8) = val;
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ void drain_acc(const FfnArgs& a, int kind, uint32_t tb, size_t row,
-                                          bool valid, int nc, int col0, int c0, int c1) {
+                                          bool valid, int nc, int col0, int c0, int c1,
+                                          uint8_t* ost) {
+  const int lane = threadIdx.x & 31;
+  const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+  const size_t row0 = row - (size_t)lane;         // the warp's first row
   if (kind == K_G1) {
-    uint4* dst = reinterpret_cast<uint4*>(a.h + row * a.f + col0);
+    __nv_bfloat16* base = a.h + row0 * a.f + col0;
 #pragma unroll 1
     for (int c = c0 / 32; c < c1 / 32; ++c) {
       uint32_t ra[32], rb[32];
@@ -568,14 +598,10 @@ __device__ __forceinline__ void drain_acc(const FfnArgs& a, int kind, uint32_t t
       for (int i = 0; i < 16; ++i)
         pk[i] = pack_bf16x2(silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i])),
                             silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1])));
-      if (valid) {
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-      }
+      store_chunk(ost, pk, lane, vmask, base, (size_t)a.f, c * 32);
     }
   } else {
-    uint4* dst = reinterpret_cast<uint4*>(a.y + row * a.d + col0);
+    __nv_bfloat16* base = a.y + row0 * a.d + col0;
 #pragma unroll 1
     for (int c = c0 / 32; c < c1 / 32; ++c) {
       uint32_t rr[32];
@@ -584,11 +610,7 @@ __device__ __forceinline__ void drain_acc(const FfnArgs& a, int kind, uint32_t t
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
-      if (valid) {
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          dst[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-      }
+      store_chunk(ost, pk, lane, vmask, base, (size_t)a.d, c * 32);
     }
   }
 }
@@ -637,7 +659,7 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
         if (rb > 0)
           drain_acc(a, it.kind, tmem_base + (uint32_t)(b * ACC_COLS) + ((uint32_t)(q * 32) << 16),
                     (size_t)(it.row0 + b * BM + row), row < rb, ncf, col0, hc * ncf / 2,
-                    (hc + 1) * ncf / 2);
+                    (hc + 1) * ncf / 2, ctl->ostage[warp - 2]);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->tempty[b]);   // accumulator may be overwritten
@@ -674,7 +696,7 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
     const int ch = half ? (row >> 6) : 0;
     const int nc = half ? ncf / 2 : ncf;
     drain_acc(a, it.kind, tb, (size_t)(m.row0 + r), r < m.rows, nc, col0 + ch * nc, hc * nc / 2,
-              (hc + 1) * nc / 2);
+              (hc + 1) * nc / 2, ctl->ostage[warp - 2]);
     tc_fence_before();
     __syncwarp();
     const int my_acc = acc;
