@@ -42,7 +42,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the persistent FFN kernel, keyed by workload, valid only for the kernel sources
 # whose hash is recorded with it (see profiles/).
-TRAFFIC = {"mixtral": {"bytes": 4695493000 + 316746240, "kernel_hash": "e312b2838377"}}
+TRAFFIC = {"mixtral": {"bytes": 4156785000 + 314484480, "kernel_hash": "bdecdd82a1a6"}}
 
 
 def kernel_source_hash() -> str:
