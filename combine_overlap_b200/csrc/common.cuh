@@ -50,7 +50,7 @@ struct Status {
   int32_t n_tiles2;
   uint32_t where;
   int32_t n_items;
-  int32_t n_groups;    // producer tile rows: groups of G consecutive bands of one expert
+  int32_t n_groups;    // producer tile rows: groups of 1 or 2 consecutive bands of one expert
 };
 
 struct Sync {          // zeroed by the plan kernel on every call
@@ -65,7 +65,8 @@ struct Band {          // one row band: up to BM rows of one expert
   int32_t expert, row0, rows, pad;
 };
 
-// A producer row group: G consecutive bands of one expert (G = CTAs per MMA).
+// A producer row group: the 1 or 2 consecutive bands of one expert that one MMA
+// tile covers (128-row or 256-row tiles).
 struct Group {
   int32_t expert, band0, row0, rows;   // rows: valid rows over the whole group
 };

@@ -997,7 +997,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   Status* st = a.w.status;
   const volatile uint32_t* abort = &st->code;
   const int n1 = st->n_tiles1, n2 = st->n_tiles2, nb = st->n_bands, n_items = st->n_items;
-  // consumer CTAs come in whole groups (the plan rounds C to a multiple of G)
+  // consumer CTAs come in whole tiles' CTAs (the plan rounds C to a multiple of cg)
   const bool consumer_cta = (a.phase & PH_CONS) && (int)blockIdx.x < st->consumer_sms;
   const bool run_g1 = (a.phase & PH_G1) != 0;
   const bool run_g2 = (a.phase & PH_G2) && !consumer_cta;

@@ -160,8 +160,8 @@ cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int32_t* b
 
 // ------------------------------------------------------------------- plan ---
 // Producer/consumer split (the Weave-style spatial scheduler): choose the number
-// C of CTAs (a multiple of G, from `cmin`) that consume from the start instead of
-// running GEMM2, minimising the modelled layer tail
+// C of CTAs (a multiple of cg, the CTAs per tile, from `cmin`) that consume from
+// the start instead of running GEMM2, minimising the modelled layer tail
 //   t(C) = t2 + max(0, Bc - C * beta * t2) / min(S * beta, beta_hbm),
 //   t2   = F2 / ((S - C) * phi)
 // F2 = GEMM2 FLOPs (the part the combine can overlap), Bc = combine bytes (every

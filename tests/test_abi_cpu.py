@@ -81,3 +81,23 @@ def test_host_side_argument_errors():
                               None) == moe.MOE_ERR_WORKSPACE
     assert moe._lib.moe_combine(P(0x1000), P(0x2000), P(0x3000), 16, 512, 9, P(0x4000),
                                 None) == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_tile_variant_rule():
+    tv = moe.tile_variant
+    # 256-row tiles on single CTAs from 256 rows per expert (T*k/E) up, else 128-row tiles
+    assert tv(4096, 14336, 8, 2) == 3          # Mixtral-shaped: 1024 rows per expert
+    assert tv(8192, 1408, 64, 6) == 3          # fine-grained: 768
+    assert tv(1024, 2048, 8, 2) == 3           # exactly 256
+    assert tv(1023, 2048, 8, 2) == 1           # just below
+    assert tv(512, 2048, 32, 4) == 1           # 64
+    # flags force a variant; ONE_CTA before CTA_PAIR before WIDE_CTA
+    assert tv(4096, 14336, 8, 2, moe.SCHED_ONE_CTA) == 1
+    assert tv(512, 2048, 32, 4, moe.SCHED_CTA_PAIR) == 2
+    assert tv(512, 2048, 32, 4, moe.SCHED_WIDE_CTA) == 3
+    assert tv(512, 2048, 32, 4, moe.SCHED_ONE_CTA | moe.SCHED_CTA_PAIR) == 1
+    assert tv(512, 2048, 32, 4, moe.SCHED_CTA_PAIR | moe.SCHED_WIDE_CTA) == 2
+    # other flags do not change the choice
+    assert tv(4096, 14336, 8, 2, moe.SCHED_NO_JOIN | moe.SCHED_B_PER_ATOM) == 3
+    assert tv(0, 14336, 8, 2) == 0
+    assert set(moe.TILE_VARIANTS) == {1, 2, 3}
