@@ -137,6 +137,27 @@ def _need(t: torch.Tensor, dtype, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _shape(t: torch.Tensor, shape: tuple, name: str):
+    """The library sees pointers only: a tensor of another shape would be read or
+    written out of bounds on the device, so sizes are checked here."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _weights(W1, W3, W2, d=None):
+    """Checks W1, W3 [E][d][f] and W2 [E][f][d]; returns (E, d, f)."""
+    for n, w in (("W1", W1), ("W3", W3), ("W2", W2)):
+        _need(w, torch.bfloat16, n)
+        if w.dim() != 3:
+            raise ValueError(f"{n} must be 3-D, got shape {tuple(w.shape)}")
+    E, dw, f = W1.shape
+    if d is not None and dw != d:
+        raise ValueError(f"W1 is [E][{dw}][f] but the rows have d = {d}")
+    _shape(W3, (E, dw, f), "W3")
+    _shape(W2, (E, f, dw), "W2")
+    return E, dw, f
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
@@ -173,6 +194,7 @@ def permute(x: torch.Tensor, topk_idx: torch.Tensor, E: int, ws: torch.Tensor):
     _need(topk_idx, torch.int32, "topk_idx")
     T, d = x.shape
     k = topk_idx.shape[1]
+    _shape(topk_idx, (T, k), "topk_idx")
     dev = x.device
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
@@ -192,6 +214,7 @@ def permute_noalloc(x: torch.Tensor, topk_idx: torch.Tensor, E: int):
     _need(topk_idx, torch.int32, "topk_idx")
     T, d = x.shape
     k = topk_idx.shape[1]
+    _shape(topk_idx, (T, k), "topk_idx")
     dev = x.device
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
@@ -210,9 +233,9 @@ def grouped_ffn(x_perm: torch.Tensor, offsets: torch.Tensor, W1, W3, W2, T: int,
     SCHED_CTA_PAIR, SCHED_B_PER_ATOM, SCHED_FULL_TILES."""
     _need(x_perm, torch.bfloat16, "x_perm")
     _need(offsets, torch.int32, "offsets")
-    for n, w in (("W1", W1), ("W3", W3), ("W2", W2)):
-        _need(w, torch.bfloat16, n)
-    E, d, f = W1.shape
+    E, d, f = _weights(W1, W3, W2, x_perm.shape[1])
+    _shape(x_perm, (T * k, d), "x_perm")
+    _shape(offsets, (E + 1,), "offsets")
     dev = x_perm.device
     y = torch.empty((T * k, d), dtype=torch.bfloat16, device=dev)
     h = torch.empty((T * k, f), dtype=torch.bfloat16, device=dev) if want_h else None
@@ -229,8 +252,12 @@ def combine(y: torch.Tensor, row_of: torch.Tensor, topk_gate: torch.Tensor, out=
     _need(topk_gate, torch.float32, "topk_gate")
     T, k = topk_gate.shape
     d = y.shape[1]
+    _shape(y, (T * k, d), "y")
+    _shape(row_of, (T * k,), "row_of")
     if out is None:
         out = torch.empty((T, d), dtype=torch.bfloat16, device=y.device)
+    _need(out, torch.bfloat16, "out")
+    _shape(out, (T, d), "out")
     _check(_lib.moe_combine(_ptr(y), _ptr(row_of), _ptr(topk_gate), T, d, k, _ptr(out), _stream()),
            "moe_combine")
     return out
@@ -255,13 +282,14 @@ def layer_forward(x, logits, W1, W3, W2, k, ws, mode=MODE_OVERLAPPED, out=None, 
     """One MoE layer.  Returns out, or (out, dict of routing outputs) if outputs."""
     _need(x, torch.bfloat16, "x")
     _need(logits, torch.float32, "logits")
-    for n, w in (("W1", W1), ("W3", W3), ("W2", W2)):
-        _need(w, torch.bfloat16, n)
     T, d = x.shape
-    E = logits.shape[1]
+    E, _, f = _weights(W1, W3, W2, d)
+    _shape(logits, (T, E), "logits")
     dev = x.device
     if out is None:
         out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    _need(out, torch.bfloat16, "out")
+    _shape(out, (T, d), "out")
     extra = {}
     if outputs:
         extra = dict(topk_idx=torch.empty((T, k), dtype=torch.int32, device=dev),

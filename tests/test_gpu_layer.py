@@ -186,3 +186,21 @@ def test_wide_tiles_refuse_gathered_rows():
     with pytest.raises(moe.MoEError) as e:
         _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=moe.SCHED_WIDE_CTA | moe.SCHED_GATHER_A)
     assert e.value.code == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_binding_rejects_mismatched_shapes():
+    # the library sees pointers only; the binding refuses shapes that would make it
+    # read or write out of bounds, before anything is launched
+    wl = synth.WORKLOADS["tiny"]
+    inp = gu.inputs(wl)
+    ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
+    x, logits, W1, W3, W2 = (inp[n] for n in ("x", "logits", "W1", "W3", "W2"))
+    with pytest.raises(ValueError):      # W2 given as [E][d][f]
+        moe.layer_forward(x, logits, W1, W3, W1, wl.k, ws)
+    with pytest.raises(ValueError):      # logits for another expert count
+        moe.layer_forward(x, logits[:, :wl.E - 1].contiguous(), W1, W3, W2, wl.k, ws)
+    with pytest.raises(ValueError):      # output rows short
+        moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, out=x[:-1].clone())
+    with pytest.raises(ValueError):      # combine: gates for more tokens than y rows
+        moe.combine(x, torch.zeros(wl.T, dtype=torch.int32, device="cuda"),
+                    torch.zeros((wl.T, wl.k), dtype=torch.float32, device="cuda"))
