@@ -22,9 +22,13 @@
  *    Every device pointer must be 16-byte aligned.
  *  - `stream` is a cudaStream_t passed as void*.  Calls are asynchronous on it
  *    and never synchronise the host, except moe_get_status.
+ *  - Buffers must hold the sizes each entry point states: the library sees
+ *    pointers only and cannot check them (the Python binding checks tensor
+ *    shapes before calling).
  *  - Argument errors return at once, before any launch, with MOE_ERR_INVALID or
- *    MOE_ERR_UNSUPPORTED; a launch failure returns MOE_ERR_CUDA.  Errors found on
- *    the device (a bounded wait that ran out) are written to the status block in
+ *    MOE_ERR_UNSUPPORTED; a launch failure returns MOE_ERR_CUDA, and
+ *    moe_last_cuda_error names the CUDA error behind it.  Errors found on the
+ *    device (a bounded wait that ran out) are written to the status block in
  *    the workspace and read back by moe_get_status.  Kernels never trap and
  *    every wait inside them is bounded.
  *  - Preconditions: 1 <= T; 1 <= k <= min(E, 8); E <= 256; d % 256 == 0;
