@@ -625,6 +625,7 @@ def run_sweep(args):
                 "tokens_per_s": wl.T / (med["ovl"] * 1e-3), "tflops": F / (med["ovl"] * 1e-3) / 1e12,
                 "roofline_frac_layer": t_roof / med["ovl"],
                 "roofline_bound": "tensor" if F / (peak_tf * 1e12) >= B / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                "mma_tile": moe.TILE_VARIANTS[moe.tile_variant(wl.T, wl.f, wl.E, wl.k)],
             }), flush=True)
         del x, logits, W1, W3, W2, ws, out
         torch.cuda.empty_cache()
