@@ -93,6 +93,10 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="d=4096/E=32/top-4 sweep: T x router x consumer SMs, overlapped vs "
                          "sequential; one JSON line per cell (not the benchmark line)")
+    ap.add_argument("--sweep-layers", default="",
+                    help="comma-separated workloads for --sweep (default: the d=4096/E=32 grid)")
+    ap.add_argument("--sweep-cells", default="seq,0,2,4,8,16",
+                    help="--sweep cells: 'seq' or 'C[/mgb]' (overlapped, C consumer SMs, 0 = cost model)")
     ap.add_argument("--oracle-timings", action="store_true",
                     help="time the CPU oracle on each benchmark configuration; one JSON line "
                          "per configuration (not the benchmark line)")
@@ -101,56 +105,85 @@ def parse():
 
 # ----------------------------------------------------------------- clocks ---
 class Clocks:
+    """nvidia-smi samples of the SM clock, power and throttle reasons, every 50 ms,
+    from before the warm-up to the end of the GPU work; each sample is stamped with
+    the host's monotonic clock so that a timed region can take the samples that fall
+    inside it."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, device: int, enabled: bool = True):
+    def __init__(self, device: int, enabled: bool = True, period_ms: int = 50):
+        import threading
         self.proc = None
-        self.path = None
+        self.samples = []          # (t_monotonic, sm_mhz, max_mhz, power_w, reasons)
+        self.windows = {}
         if not enabled:
             return
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", sel], stdout=self.fh, stderr=subprocess.DEVNULL)
+                 "-lms", str(period_ms), "-i", sel], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
         except (OSError, RuntimeError):
             self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        import atexit
+        atexit.register(self.stop)   # never leave the sampler running after an error
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, smax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            try:
+                pw = float(parts[3])
+            except ValueError:
+                pw = None
+            reasons = {n for n, v in zip(self.REASONS, parts[5:9]) if v.lower().startswith("active")}
+            self.samples.append((time.monotonic(), sm, smax, pw, reasons))
+
+    def mark(self, name: str, t0: float, t1: float):
+        """Record the host-clock window [t0, t1] of a timed region."""
+        self.windows[name] = (t0, t1)
 
     def stop(self):
-        if self.proc is None:
-            return None
-        time.sleep(0.25)
+        if self.proc is None or self.proc.returncode is not None:
+            return
+        time.sleep(0.2)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        self.fh.close()
-        sm, smax, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        with open(self.path) as fh:
-            for line in fh:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smax.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(n)
-        os.unlink(self.path)
-        if not sm:
+        self.thread.join(timeout=5)
+
+    def summary(self, name: str | None = None, pad_s: float = 0.06):
+        """Median SM clock, max clock and the throttle reasons seen, over the samples
+        inside region `name` (widened by one sampling period on each side, so a region
+        shorter than the period still gets its neighbours), or over every sample."""
+        if name is not None and name in self.windows:
+            t0, t1 = self.windows[name]
+            sel = [s for s in self.samples if t0 - pad_s <= s[0] <= t1 + pad_s]
+        else:
+            sel = list(self.samples)
+        if not sel:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+        reasons = set()
+        for s in sel:
+            reasons |= s[4]
+        pw = [s[3] for s in sel if s[3] is not None]
+        return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": max(s[2] for s in sel),
+                "samples": len(sel), "power_w_max": max(pw) if pw else None,
                 "reasons": sorted(reasons)}
 
 
@@ -234,6 +267,9 @@ def run_ours(args):
             torch.distributed.barrier()
 
     stream = torch.cuda.current_stream()
+    # the clock sampler starts before the warm-up, so starting it costs the timed
+    # regions nothing; each region marks its host-clock window
+    clk = Clocks(local, not args.no_clocks)
     for _ in range(args.warmup):
         step(moe.MODE_OVERLAPPED)
         step(moe.MODE_SEQUENTIAL)
@@ -244,32 +280,36 @@ def run_ours(args):
     counts = moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, moe.MODE_OVERLAPPED, outputs=True,
                                **kw)[1]["counts"].cpu().tolist()
 
-    def timed(mode, clocks=False, hooks=False):
+    def timed(mode, name, hooks=False):
         K = args.steps
         evb = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if hooks else [None] * K
         eve = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if hooks else [None] * K
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # a few untimed steps right before the region, so it starts in the steady
+        # state rather than after the host-side pause above
+        for _ in range(3):
+            step(mode)
         barrier()
         torch.cuda.synchronize()
-        clk = Clocks(local, clocks and not args.no_clocks) if clocks else None
+        h0 = time.monotonic()
         e0.record(stream)
         for i in range(K):
             step(mode, evb[i], eve[i])
         e1.record(stream)
         torch.cuda.synchronize()
+        clk.mark(name, h0, time.monotonic())
         barrier()
-        c = clk.stop() if clk else None
         total = e0.elapsed_time(e1) / K
         ffn = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / K if hooks else None
-        return total, ffn, c
+        return total, ffn
 
-    # The contract's timed region: K overlapped steps, clocks sampled meanwhile.
-    # It runs without the library's timing hooks: a recorded event between two
-    # launches costs them their programmatic overlap.
-    t_ovl, _, clocks = timed(moe.MODE_OVERLAPPED, clocks=True)
+    # The contract's timed region: K overlapped steps.  It runs without the
+    # library's timing hooks: a recorded event between two launches costs them
+    # their programmatic overlap.
+    t_ovl, _ = timed(moe.MODE_OVERLAPPED, "contract")
     # The persistent FFN kernel's average launch duration, from K more overlapped
     # steps with the hooks (events recorded on the launching stream around it).
-    t_ovl_hooked, ffn_ovl, _ = timed(moe.MODE_OVERLAPPED, hooks=True)
+    t_ovl_hooked, ffn_ovl = timed(moe.MODE_OVERLAPPED, "hooked", hooks=True)
     # overlapped vs sequential: the two modes alternate step by step (paired
     # samples under the same clock and power state), each step timed with events
     # on the stream; medians per mode
@@ -279,13 +319,17 @@ def run_ours(args):
               for _ in range(K)] for m in ("seq", "ovl")}
     barrier()
     torch.cuda.synchronize()
+    h0 = time.monotonic()
     for i in range(K):
-        for m, mode in (("seq", moe.MODE_SEQUENTIAL), ("ovl", moe.MODE_OVERLAPPED)):
+        # alternate which mode goes first, so neither always follows the other
+        order = (("seq", moe.MODE_SEQUENTIAL), ("ovl", moe.MODE_OVERLAPPED))
+        for m, mode in (order if i % 2 == 0 else order[::-1]):
             e0, e1, fb, fe = ev[m][i]
             e0.record(stream)
             step(mode, fb, fe)
             e1.record(stream)
     torch.cuda.synchronize()
+    clk.mark("paired", h0, time.monotonic())
     barrier()
     step_ms = {m: [e0.elapsed_time(e1) for e0, e1, _, _ in ev[m]] for m in ev}
     ffn_ms = {m: [fb.elapsed_time(fe) for _, _, fb, fe in ev[m]] for m in ev}
@@ -308,11 +352,13 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0 = time.monotonic()
     e0.record(stream)
     for _ in range(args.steps):
         g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
+    clk.mark("graph", h0, time.monotonic())
     barrier()
     t_graph = e0.elapsed_time(e1) / args.steps
     del g
@@ -359,13 +405,19 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0 = time.monotonic()
     e0.record(stream)
     h2d.wait_event(e0)
     e2e_steps(args.steps)
     e1.record(stream)
     torch.cuda.synchronize()
+    clk.mark("e2e", h0, time.monotonic())
     barrier()
     t_e2e = e0.elapsed_time(e1) / args.steps
+    clk.stop()
+    clocks = clk.summary("contract")
+    clocks_by_region = {n: clk.summary(n) for n in ("contract", "hooked", "paired", "graph", "e2e")}
+    clocks_run = clk.summary()
     if not torch.equal(out_h[(args.steps - 1) & 1].to(out.device), out):
         raise RuntimeError("end-to-end output differs from the device-resident run")
     code, _, _ = moe.get_status(ws)
@@ -384,7 +436,11 @@ def run_ours(args):
     if rank == 0:
         peaks, src = load_peaks()
         F, B = flops_and_bytes(wl, counts)
-        peak_tf = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+        # the FFN launch and the layer step last milliseconds: the burst cuBLAS
+        # figure is their peak (the sustained one, under the power cap after
+        # seconds of back-to-back GEMMs, is reported beside it)
+        peak_tf = peaks["bf16_tflops"]
+        peak_tf_sus = peaks.get("bf16_tflops_sustained")
         hbm = peaks["hbm_gbs"]
         t_roof_ms = max(F / (peak_tf * 1e12), B / (hbm * 1e9)) * 1e3
         ach = F / (ffn_ovl * 1e-3) / 1e12
@@ -415,7 +471,10 @@ def run_ours(args):
             "roofline_frac_layer": t_roof_ms / t_ovl,
             "roofline_layer": {"bound": "tensor" if F / (peak_tf * 1e12) >= B / (hbm * 1e9) else "hbm",
                                "time_ms": t_roof_ms, "flops": F, "min_bytes": B,
-                               "peak_tflops": peak_tf, "peak_hbm_gbs": hbm, "peaks": src},
+                               "peak_tflops": peak_tf, "peak_hbm_gbs": hbm,
+                               "peaks": f"{src} (bf16 burst, HBM copy)",
+                               "frac_vs_sustained_peak": (max(F / (peak_tf_sus * 1e12), B / (hbm * 1e9)) * 1e3
+                                                          / t_ovl) if peak_tf_sus else None},
             "sequential": {"value": T_all / (t_seq * 1e-3), "ms_per_step": t_seq,
                            "ffn_ms": ffn_seq, "tflops": world * F / (t_seq * 1e-3) / 1e12,
                            "overlapped_ms_per_step": t_ovl_med, "overlapped_ffn_ms": ffn_ovl_med,
@@ -443,13 +502,17 @@ def run_ours(args):
                          "launch_timing": "CUDA events on the launching stream around the "
                                           "persistent kernel, K overlapped steps after the "
                                           "contract region (%.4f ms per step there)" % t_ovl_hooked,
-                         "peak_kind": f"{src} sustained bf16 (cuBLAS 8192^3 under the power cap)"},
+                         "peak_kind": f"{src} burst bf16 (cuBLAS 8192^3, best of 10): the kernel is "
+                                      "a ms-long launch",
+                         "frac_vs_sustained_peak": ach / peak_tf_sus if peak_tf_sus else None},
             "e2e": {"value": job_tokens_per_s(wl.T, world, t_e2e), "unit": "tokens/s", "ms_per_step": t_e2e,
                     "h2d_bytes_per_step": x.numel() * 2 + logits.numel() * 4,
                     "d2h_bytes_per_step": out.numel() * 2,
                     "method": "pinned host buffers; double-buffered device buffers; H2D and D2H on their own streams, overlapping the neighbouring steps' compute"},
             "gpu_launches": 6 * args.steps,   # route, plan, scatter, gather, persistent FFN, combine
             "clocks": clocks,
+            "clocks_by_region": clocks_by_region,
+            "clocks_whole_run": clocks_run,
             "kernel_hash": h,
         }
         if cpu is not None:
@@ -519,7 +582,11 @@ def run_reference(args):
     res = {
         "impl": "reference",
         "metric": "MoE-layer tokens/s", "value": v, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.T / v * 1e3,
+        # a step is the timed token sample, not the whole layer (which would take
+        # layer_ms_extrapolated below)
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "tokens_per_step": tot_n / args.steps,
+        "layer_ms_extrapolated": wl.T / v * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic: seeded counter-based inputs, random-init weights",
         "config": {"workload": wl.name, "T": wl.T, "d_model": wl.d, "d_ff": wl.f, "E": wl.E,
@@ -582,15 +649,35 @@ def run_oracle_timings(args):
                           else "token-by-token definition path"}), flush=True)
 
 
+def _sweep_cells(spec: str):
+    """Cells of a paired sweep: "seq" (sequential mode) or "C[/mgb]" (overlapped mode,
+    C consumer SMs, 0 = the cost model; mgb row bands per consumer item)."""
+    cells = []
+    for tok in spec.split(","):
+        tok = tok.strip()
+        if tok == "seq":
+            cells.append(("seq", None, 0, 1))
+        else:
+            c, _, m = tok.partition("/")
+            cells.append((tok, "ovl", int(c), int(m) if m else 1))
+    return cells
+
+
 def run_sweep(args):
-    """Every sweep cell: the overlapped mode at a fixed consumer-SM count (2, 4, 8)
-    or the cost model's choice (0), against the sequential mode, timed as paired
-    alternating steps (medians)."""
+    """Paired sweep of layers x cells.  Per layer, every cell (the sequential mode,
+    the overlapped mode at the cost model's split, at fixed consumer-SM counts, or at
+    other segment sizes mgb) runs once per round, the order rotated from round to
+    round, each step timed with CUDA events on the stream; medians per cell.  So the
+    cells of a layer see the same clock and power history, and none always runs
+    first.  One JSON line per layer, with the clocks sampled during it."""
     from combine_overlap_b200 import moe
     torch.cuda.set_device(0)
     peaks, src = load_peaks()
-    peak_tf = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
-    names = [n for n in synth.WORKLOADS if n.startswith("sweep_")]
+    peak_tf = peaks["bf16_tflops"]
+    names = args.sweep_layers.split(",") if args.sweep_layers else \
+        [n for n in synth.WORKLOADS if n.startswith("sweep_")]
+    cells = _sweep_cells(args.sweep_cells)
+    clk = Clocks(0, not args.no_clocks)
     for name in names:
         wl = synth.WORKLOADS[name]
         x, logits, W1, W3, W2 = rank_inputs(wl, 0, "cuda")
@@ -599,36 +686,62 @@ def run_sweep(args):
         counts = moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, outputs=True)[1]["counts"].cpu().tolist()
         F, B = flops_and_bytes(wl, counts)
         t_roof = max(F / (peak_tf * 1e12), B / (peaks["hbm_gbs"] * 1e9)) * 1e3
-        for C in (2, 4, 8, 0):
-            def step(mode):
-                moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, mode, out=out, consumer_sms=C)
-            for _ in range(args.warmup):
-                step(moe.MODE_OVERLAPPED)
-                step(moe.MODE_SEQUENTIAL)
-            evs = {m: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                       for _ in range(args.steps)] for m in ("seq", "ovl")}
-            torch.cuda.synchronize()
-            for i in range(args.steps):
-                for m, mode in (("seq", moe.MODE_SEQUENTIAL), ("ovl", moe.MODE_OVERLAPPED)):
-                    evs[m][i][0].record()
-                    step(mode)
-                    evs[m][i][1].record()
-            torch.cuda.synchronize()
-            code, c_used, _ = moe.get_status(ws)
-            if code != moe.MOE_OK:
-                raise RuntimeError(f"{name} C={C}: {moe.status_string(code)}")
-            med = {m: statistics.median(a.elapsed_time(b) for a, b in evs[m]) for m in evs}
-            print(json.dumps({
-                "sweep": name, "T": wl.T, "router": wl.router,
-                "consumer_sms": "cost model" if C == 0 else C, "consumer_sms_used": c_used,
-                "ovl_ms": med["ovl"], "seq_ms": med["seq"], "speedup_vs_sequential": med["seq"] / med["ovl"],
-                "tokens_per_s": wl.T / (med["ovl"] * 1e-3), "tflops": F / (med["ovl"] * 1e-3) / 1e12,
-                "roofline_frac_layer": t_roof / med["ovl"],
-                "roofline_bound": "tensor" if F / (peak_tf * 1e12) >= B / (peaks["hbm_gbs"] * 1e9) else "hbm",
-                "mma_tile": moe.TILE_VARIANTS[moe.tile_variant(wl.T, wl.f, wl.E, wl.k)],
-            }), flush=True)
+
+        def step(cell):
+            _, mode, C, mgb = cell
+            m = moe.MODE_SEQUENTIAL if mode is None else moe.MODE_OVERLAPPED
+            moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, m, out=out, consumer_sms=C, mgb=mgb)
+
+        used = {}
+        for cell in cells:
+            for _ in range(max(1, args.warmup)):
+                step(cell)
+            if cell[1] is not None:
+                torch.cuda.synchronize()
+                code, c_used, _ = moe.get_status(ws)
+                if code != moe.MOE_OK:
+                    raise RuntimeError(f"{name} {cell[0]}: {moe.status_string(code)}")
+                used[cell[0]] = c_used
+        evs = {c[0]: [] for c in cells}
+        torch.cuda.synchronize()
+        h0 = time.monotonic()
+        n = len(cells)
+        for i in range(args.steps):
+            for j in range(n):
+                cell = cells[(i + j) % n]
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                step(cell)
+                e1.record()
+                evs[cell[0]].append((e0, e1))
+        torch.cuda.synchronize()
+        clk.mark(name, h0, time.monotonic())
+        code, _, _ = moe.get_status(ws)
+        if code != moe.MOE_OK:
+            raise RuntimeError(f"{name}: {moe.status_string(code)}")
+        ms = {c: sorted(a.elapsed_time(b) for a, b in v) for c, v in evs.items()}
+        med = {c: statistics.median(v) for c, v in ms.items()}
+        q = {c: (v[len(v) // 4], v[(3 * len(v)) // 4]) for c, v in ms.items()}
+        res = {"sweep": name, "T": wl.T, "router": wl.router, "steps": args.steps,
+               "mma_tile": moe.TILE_VARIANTS[moe.tile_variant(wl.T, wl.f, wl.E, wl.k)],
+               "roofline_ms": t_roof, "flops": F, "min_bytes": B,
+               "roofline_bound": "tensor" if F / (peak_tf * 1e12) >= B / (peaks["hbm_gbs"] * 1e9) else "hbm",
+               "peaks": f"{src}: bf16 burst {peak_tf} TFLOP/s, HBM {peaks['hbm_gbs']} GB/s",
+               "cells": {}}
+        for c in ms:
+            cell = {"ms": med[c], "q25_ms": q[c][0], "q75_ms": q[c][1],
+                    "tokens_per_s": wl.T / (med[c] * 1e-3), "tflops": F / (med[c] * 1e-3) / 1e12,
+                    "roofline_frac": t_roof / med[c]}
+            if c in used:
+                cell["consumer_sms_used"] = used[c]
+            if "seq" in med and c != "seq":
+                cell["speedup_vs_sequential"] = med["seq"] / med[c]
+            res["cells"][c] = cell
+        res["clocks"] = clk.summary(name)
+        print(json.dumps(res), flush=True)
         del x, logits, W1, W3, W2, ws, out
         torch.cuda.empty_cache()
+    clk.stop()
 
 
 def main():

@@ -334,7 +334,10 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   moe_status s = check_shape(A.T, A.d, A.f, A.E, A.k);
   if (s != MOE_OK) return s;
   if (mode != MOE_MODE_SEQUENTIAL && mode != MOE_MODE_OVERLAPPED) return MOE_ERR_INVALID;
-  if (!ok_ptr(A.x) || !ok_ptr(A.logits) || !ok_ptr(A.W1) || !ok_ptr(A.W3) || !ok_ptr(A.W2) ||
+  // identity experts read no weights: W1, W3, W2 may then be NULL
+  const bool identity = (A.flags & MOE_DBG_IDENTITY_EXPERTS) != 0;
+  auto ok_w = [&](const void* p) { return identity ? ok_opt(p) : ok_ptr(p); };
+  if (!ok_ptr(A.x) || !ok_ptr(A.logits) || !ok_w(A.W1) || !ok_w(A.W3) || !ok_w(A.W2) ||
       !ok_ptr(A.out) || !ok_opt(A.topk_idx) || !ok_opt(A.topk_gate) || !ok_opt(A.counts) ||
       !ok_opt(A.offsets) || !ok_opt(A.perm))
     return MOE_ERR_INVALID;
@@ -345,7 +348,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   // MOE_SCHED_GATHER_A: GEMM1 gathers its A rows from x with TMA gather4 instead
   // of reading x_perm (no x_perm pass, but 32 gather instructions per k-block);
   // 128-row gathers only, so not with V = 3
-  const int gather_a = (A.flags & MOE_SCHED_GATHER_A) ? 1 : 0;
+  const int gather_a = (A.flags & (MOE_SCHED_GATHER_A | MOE_DBG_IDENTITY_EXPERTS)) == MOE_SCHED_GATHER_A;
   int V = choose_variant(A.T, A.f, A.E, A.k, A.flags);
   if (gather_a && V == 3) {
     if (A.flags & MOE_SCHED_WIDE_CTA) return MOE_ERR_UNSUPPORTED;
@@ -373,6 +376,14 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   MOE_TRY(launch_scatter(w.topk_idx, T, E, k, w.blk_base, w.perm, w.row_of, gather_a ? &w : nullptr, st));
   if (!gather_a)
     MOE_TRY(launch_gather(static_cast<const __nv_bfloat16*>(A.x), w.row_of, T, d, k, w.x_perm, nsm, st));
+  if (identity) {
+    // identity experts: y = x_perm, so the combine reads the permuted rows directly
+    if (A.ev_ffn_begin) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_begin), st));
+    if (A.ev_ffn_end) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_end), st));
+    MOE_TRY(launch_combine(w.x_perm, w.row_of, w.topk_gate, T, d, k,
+                           static_cast<__nv_bfloat16*>(A.out), nsm, st));
+    return MOE_OK;
+  }
   FfnArgs a;
   memset(&a, 0, sizeof(a));
   a.w = w;
@@ -445,6 +456,7 @@ moe_status moe_get_status(void* ws, void* stream, int* consumer_sms, int* n_band
   if (consumer_sms) *consumer_sms = h.consumer_sms;
   if (n_bands) *n_bands = h.n_bands;
   if (h.code == ST_TIMEOUT) return MOE_ERR_TIMEOUT;
+  if (h.code == ST_INVALID) return MOE_ERR_INVALID;
   return h.code == ST_OK ? MOE_OK : MOE_ERR_CUDA;
 }
 

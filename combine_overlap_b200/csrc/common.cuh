@@ -34,7 +34,9 @@ constexpr uint32_t TOKEN_DONE = 0x80000000u;   // arrive[t] flag: a consumer com
 constexpr int MAX_K = 8;
 
 // ----------------------------------------------------------------- status ---
-enum : uint32_t { ST_OK = 0, ST_TIMEOUT = 4 };
+// ST_INVALID: a caller-supplied expert id outside [0, E) (moe_permute); ST_TIMEOUT: a
+// bounded device wait ran out.
+enum : uint32_t { ST_OK = 0, ST_INVALID = 1, ST_TIMEOUT = 4 };
 // where a wait ran out (Status::where)
 enum : uint32_t {
   W_NONE = 0, W_SCHED_EMPTY = 1, W_SCHED_FULL = 2, W_STAGE_EMPTY = 3, W_STAGE_FULL = 4,

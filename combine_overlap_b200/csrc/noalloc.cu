@@ -12,11 +12,15 @@
 // The scratch is one file-scope __device__ array of PERMUTE_NOALLOC_SCRATCH_BYTES
 // (a little over 4 MiB), present on every GPU that loads the library until the
 // process exits.  In host code the array's name is only a host-side stand-in,
-// never a device address, so its device address is looked up once per device
-// with cudaGetSymbolAddress (with that device current) and cached.
+// never a device address, so its device address is looked up with
+// cudaGetSymbolAddress (with that device current) and cached per device and per
+// CUDA context: after cudaDeviceReset the device gets a new primary context, in
+// which the library's module (and so the array) may sit at another address, and
+// the first call in the new context looks it up again.
 #include "kernels.h"
 #include "../../include/moe.h"
 
+#include <cuda.h>
 #include <mutex>
 #include <string.h>
 
@@ -39,23 +43,51 @@ static __device__ __align__(256) unsigned char g_permute_scratch[PERMUTE_NOALLOC
 constexpr int MAX_DEVICES = 64;
 std::mutex g_mutex;
 void* g_scratch_ptr[MAX_DEVICES] = {nullptr};
+CUcontext g_scratch_ctx[MAX_DEVICES] = {nullptr};   // the context g_scratch_ptr[dev] belongs to
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The calling thread's current driver context (null if the runtime has not made
+// one current yet).  The driver entry point is looked up once through the
+// runtime, so the library needs no link against libcuda.
+cudaError_t current_context(CUcontext* ctx) {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return cudaErrorNotSupported;
+    fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  return fn(ctx) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
 
 // Device address of g_permute_scratch on the current device (looked up on the
-// first call on that device, then cached).
+// first call on that device, and again whenever the device's context changed,
+// e.g. after cudaDeviceReset; cached otherwise).
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= MAX_DEVICES) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_permute_scratch);
-    if (e != cudaSuccess) return e;
-    if (!p) return cudaErrorInvalidSymbol;
-    g_scratch_ptr[dev] = p;
+  CUcontext ctx = nullptr;
+  // cudaGetSymbolAddress makes the device's primary context current if none is,
+  // so the context is read after it on a miss
+  if (current_context(&ctx) == cudaSuccess && ctx && g_scratch_ptr[dev] && ctx == g_scratch_ctx[dev]) {
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
   }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_permute_scratch);
+  if (e != cudaSuccess) return e;
+  if (!p) return cudaErrorInvalidSymbol;
+  e = current_context(&ctx);
+  if (e != cudaSuccess) return e;
+  g_scratch_ptr[dev] = p;
+  g_scratch_ctx[dev] = ctx;
+  *out = p;
   return cudaSuccess;
 }
 

@@ -138,7 +138,8 @@ cudaError_t launch_colsum(const int32_t* blk_hist, int nblk, int E, int32_t* cou
 }
 
 // Per-block expert histogram of given top-k ids (moe_permute's entry, where the
-// routing came from the caller rather than route_kernel).
+// routing came from the caller rather than route_kernel).  An id outside [0, E)
+// is not counted; the plan kernel sees the short total and records ST_INVALID.
 __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ topk_idx, int T,
                                                    int E, int k, int32_t* __restrict__ blk_hist) {
   pdl_trigger();
@@ -148,7 +149,10 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ t
   __syncthreads();
   const long p0 = (long)blockIdx.x * ROUTE_TOK * k;
   const long p1 = (long)min(T, (int)(blockIdx.x + 1) * ROUTE_TOK) * k;
-  for (long p = p0 + threadIdx.x; p < p1; p += blockDim.x) atomicAdd(&hist[topk_idx[p]], 1);
+  for (long p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+    const int e = topk_idx[p];
+    if ((unsigned)e < (unsigned)E) atomicAdd(&hist[e], 1);
+  }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) blk_hist[(size_t)blockIdx.x * E + e] = hist[e];
 }
@@ -231,7 +235,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
   __shared__ int t1start[MAX_E + 1];
   __shared__ int part[1024];        // [g][e]: rows' sums of chunk g, then its exclusive base
   __shared__ int totals[3];
+  __shared__ int bad_in;            // caller-supplied offsets were not a valid scan
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) bad_in = 0;
+  __syncthreads();
   // Counts and per-block scatter bases.  Thread (g, e) = (tid / E, tid % E) owns
   // expert e over the contiguous chunk g of route blocks, so a warp's loads and
   // stores cover consecutive experts of the same rows (coalesced).
@@ -265,7 +272,17 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
       cnt[e] = run;
     }
   } else {
-    for (int e = tid; e < E; e += blockDim.x) cnt[e] = offsets_in[e + 1] - offsets_in[e];
+    // caller-supplied offsets (moe_grouped_ffn): they must start at 0, never
+    // decrease and end at most at T*k, or no row is planned and ST_INVALID is
+    // recorded (no tile would stay inside the row buffers otherwise)
+    for (int e = tid; e < E; e += blockDim.x) {
+      cnt[e] = offsets_in[e + 1] - offsets_in[e];
+      if (cnt[e] < 0) bad_in = 1;
+    }
+    if (tid == 0 && (offsets_in[0] != 0 || offsets_in[E] > T * k)) bad_in = 1;
+    __syncthreads();
+    if (bad_in)
+      for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
   }
   __syncthreads();
   if (warp == 0) {
@@ -329,13 +346,14 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
   }
   if (tid == 0) {
     const long long R = offs[E];
-    // without producers joining, at least one CTA group must consume from the start
+    // ids from the caller (nblk > 0 and no route kernel before us) that fell outside
+    // [0, E) were not counted: the total comes up short of T*k
     const int cmin = join ? 0 : cg;
     int C = consumer_hint > 0 ? consumer_hint : choose_consumers(num_sms, cg, cmin, R, T, d, f, cm);
     C = cg * cdiv(C, cg);                       // consumers come in whole CTA groups
     C = max(cmin, min(C, num_sms - cg));        // and leave at least one producer group
     Status st;
-    st.code = ST_OK;
+    st.code = (bad_in || (nblk > 0 && R != (long long)T * k)) ? ST_INVALID : ST_OK;
     st.consumer_sms = C;
     st.n_bands = nb;
     st.n_tiles1 = nt1;
@@ -392,8 +410,8 @@ cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int 
 }
 
 // ---------------------------------------------------------------- scatter ---
-// Block b owns the slots of route block b (tokens [b*128, b*128+128)) and walks
-// them in ascending order, 256 at a time.  Within a warp, __match_any_sync gives
+// Block b owns the slots of route block b (tokens [b*ROUTE_TOK, (b+1)*ROUTE_TOK))
+// and walks them in ascending order, 256 at a time.  Within a warp, __match_any_sync gives
 // each slot's rank among earlier lanes with the same expert; per-warp counts in
 // shared memory give the rank among earlier warps; a running count per expert
 // carries across chunks.  row = (expert's offset + earlier blocks' count, from
@@ -420,8 +438,12 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
   const uint32_t lt = (1u << lane) - 1u;
   for (long c = p0; c < p1; c += 256) {
     const long p = c + threadIdx.x;
-    const bool valid = p < p1;
-    const int e = valid ? topk_idx[p] : -1;
+    const bool in_block = p < p1;
+    int e = in_block ? topk_idx[p] : -1;
+    // an id outside [0, E) (a caller's bad input) gets no row: row_of = -1
+    const bool valid = in_block && (unsigned)e < (unsigned)E;
+    if (!valid) e = -1;
+    if (in_block && !valid) row_of[p] = -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
     const int rank_w = __popc(peers & lt);
     if (valid && rank_w == 0) wcnt[warp][e] = __popc(peers);
@@ -457,7 +479,6 @@ cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const i
 }
 
 // ----------------------------------------------------------------- gather ---
-// x_perm[r] = x[perm[r] / k]: one warp per row, 16-byte vector loads and stores.
 // x_perm[row_of[t*k + j]] = x[t] for every slot: token-major, so each x row is
 // read from memory once and written to its k expert rows (a row-major walk of
 // x_perm would re-read x[t] k times, from DRAM once x outgrows L2).  One warp per
@@ -465,6 +486,7 @@ cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const i
 __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x,
                                                      const int32_t* __restrict__ row_of, int T,
                                                      int dv, int k, uint4* __restrict__ x_perm) {
+  const unsigned R = (unsigned)T * (unsigned)k;   // rows of x_perm; row_of = -1 marks none
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -485,7 +507,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ x
       }
 #pragma unroll
       for (int j = 0; j < MAX_K; ++j) {
-        if (j < k) {
+        if (j < k && (unsigned)rows[j] < R) {
           uint4* dst = x_perm + (size_t)rows[j] * dv;
 #pragma unroll
           for (int u = 0; u < U; ++u) {

@@ -34,6 +34,7 @@ SCHED_CTA_PAIR = 0x20
 SCHED_B_PER_ATOM = 0x40
 SCHED_FULL_TILES = 0x80
 SCHED_WIDE_CTA = 0x100
+DBG_IDENTITY_EXPERTS = 0x200
 
 
 class MoEError(RuntimeError):
@@ -265,11 +266,12 @@ def combine(y: torch.Tensor, row_of: torch.Tensor, topk_gate: torch.Tensor, out=
 
 def make_args(x, logits, W1, W3, W2, k, out, topk_idx=None, topk_gate=None, counts=None,
               offsets=None, perm=None, consumer_sms=0, mgb=1, flags=0, timeout_us=0,
-              ev_begin=None, ev_end=None) -> LayerArgs:
+              ev_begin=None, ev_end=None, d_ff=None) -> LayerArgs:
     T, d = x.shape
-    E, _, f = W1.shape
-    return LayerArgs(T, d, f, E, k, x.data_ptr(), logits.data_ptr(), W1.data_ptr(), W3.data_ptr(),
-                     W2.data_ptr(), out.data_ptr(),
+    E = logits.shape[1]
+    f = W1.shape[2] if W1 is not None else d_ff
+    wp = [0 if w is None else w.data_ptr() for w in (W1, W3, W2)]
+    return LayerArgs(T, d, f, E, k, x.data_ptr(), logits.data_ptr(), *wp, out.data_ptr(),
                      *(0 if t is None else t.data_ptr() for t in (topk_idx, topk_gate, counts, offsets, perm)),
                      consumer_sms, mgb, flags, timeout_us,
                      None if ev_begin is None else ev_begin.cuda_event,
@@ -278,13 +280,20 @@ def make_args(x, logits, W1, W3, W2, k, out, topk_idx=None, topk_gate=None, coun
 
 def layer_forward(x, logits, W1, W3, W2, k, ws, mode=MODE_OVERLAPPED, out=None, outputs=False,
                   consumer_sms=0, mgb=1, flags=0, timeout_us=0, stream=None, ev_begin=None,
-                  ev_end=None):
-    """One MoE layer.  Returns out, or (out, dict of routing outputs) if outputs."""
+                  ev_end=None, d_ff=None):
+    """One MoE layer.  Returns out, or (out, dict of routing outputs) if outputs.
+    With flags DBG_IDENTITY_EXPERTS the weights may be None (then d_ff gives the
+    FFN width the workspace was sized for)."""
     _need(x, torch.bfloat16, "x")
     _need(logits, torch.float32, "logits")
     T, d = x.shape
-    E, _, f = _weights(W1, W3, W2, d)
+    if W1 is None and W3 is None and W2 is None and (flags & DBG_IDENTITY_EXPERTS):
+        E, f = logits.shape[1], int(d_ff)
+    else:
+        E, _, f = _weights(W1, W3, W2, d)
     _shape(logits, (T, E), "logits")
+    if ws.numel() < workspace_size(T, d, f, E, k):
+        raise ValueError("workspace smaller than moe_workspace_size for this shape")
     dev = x.device
     if out is None:
         out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
@@ -305,7 +314,8 @@ def layer_forward(x, logits, W1, W3, W2, k, ws, mode=MODE_OVERLAPPED, out=None, 
         if ev is not None:
             ev.record(s)
     args = make_args(x, logits, W1, W3, W2, k, out, consumer_sms=consumer_sms, mgb=mgb,
-                     flags=flags, timeout_us=timeout_us, ev_begin=ev_begin, ev_end=ev_end, **extra)
+                     flags=flags, timeout_us=timeout_us, ev_begin=ev_begin, ev_end=ev_end,
+                     d_ff=f, **extra)
 
     _check(_lib.moe_layer_forward(ctypes.byref(args), int(mode), _ptr(ws), ws.numel(),
                                   _stream(stream)), "moe_layer_forward")

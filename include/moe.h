@@ -92,6 +92,11 @@ typedef enum {
 #define MOE_SCHED_FULL_TILES   0x80u /* CTA pairs run an expert's odd last row band as a
                                         full 256-row tile (half of it masked) instead of a
                                         128-row half tile (M=128 cta_group::2 MMA) */
+#define MOE_DBG_IDENTITY_EXPERTS 0x200u /* every expert is the identity map (y = x_perm):
+                                        the call runs route, permute and the combine only,
+                                        in either mode, so out[t] = bf16(sum_j g_j x[t])
+                                        checks those steps apart from the GEMMs; W1, W3
+                                        and W2 are not read and may be NULL */
 #define MOE_SCHED_WIDE_CTA     0x100u /* force 256-row MMA tiles on single CTAs: two
                                         128-row MMAs per K step share one B stage and
                                         fill the CTA's two accumulators (an expert's odd
@@ -148,7 +153,12 @@ moe_status moe_route(const float* logits, int T, int E, int k,
  * expert e are its slots p = t*k + j in ascending p.
  * perm [T*k]: row r -> slot p; row_of [T*k]: slot p -> row r;
  * x_perm [T*k][d] bf16: x_perm[r] = x[perm[r] / k].
- * counts [E] and offsets [E+1] are outputs (offsets required, counts optional). */
+ * counts [E] and offsets [E+1] are outputs (offsets required, counts optional).
+ * Every topk_idx value must lie in [0, E).  An id outside that range (e.g. -1
+ * for a dropped token) is skipped rather than indexed with: its slot gets
+ * row_of = -1 and no row, offsets[E] comes out below T*k (perm past offsets[E]
+ * is left unwritten), and the status block records MOE_ERR_INVALID, which
+ * moe_get_status(ws, ...) returns. */
 moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t* topk_idx,
                        int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* row_of,
                        void* x_perm, void* ws, size_t ws_bytes, void* stream);
@@ -159,7 +169,8 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
  *   h[r] = bf16(silu(x_perm[r] W1_e) * (x_perm[r] W3_e)),  y[r] = bf16(h[r] W2_e)
  * (fp32 accumulation).  x_perm [R][d], y [R][d] bf16, R = offsets[E] <= T*k;
  * h [R][f] bf16 is written to the caller's buffer if non-NULL, else kept in the
- * workspace.  flags: 0, or MOE_SCHED_ONE_CTA / MOE_SCHED_CTA_PAIR /
+ * workspace.  offsets must start at 0, never decrease and end at most at T*k;
+ * otherwise nothing is computed and moe_get_status returns MOE_ERR_INVALID.  flags: 0, or MOE_SCHED_ONE_CTA / MOE_SCHED_CTA_PAIR /
  * MOE_SCHED_B_PER_ATOM / MOE_SCHED_FULL_TILES (tile variant); any other bit is
  * MOE_ERR_INVALID. */
 moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, int d, int f,
@@ -169,7 +180,9 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
 
 /* Step (d) alone, the weighted reduction (paper Section 2.1, "Weighted reduction
  * (scale)"): out[t] = bf16( sum_{j<k} g[t][j] * y[row_of[t*k+j]] ), fp32 in slot
- * order.  y [T*k][d] bf16, row_of [T*k], topk_gate [T][k] -> out [T][d] bf16. */
+ * order.  y [T*k][d] bf16, row_of [T*k], topk_gate [T][k] -> out [T][d] bf16.
+ * Every row_of value must lie in [0, T*k) (as moe_permute writes it when all
+ * expert ids are in range); the kernel reads y[row_of[p]] without a check. */
 moe_status moe_combine(const void* y, const int32_t* row_of, const float* topk_gate,
                        int T, int d, int k, void* out, void* stream);
 
@@ -184,9 +197,13 @@ moe_status moe_combine(const void* y, const int32_t* row_of, const float* topk_g
  * nothing and calls no allocating routine.
  *  - Limits: T <= 65536 (MOE_ERR_UNSUPPORTED above that), E <= 256, k <= 8,
  *    d % 8 == 0; counts may be NULL.
- *  - The first call on a device looks up the array's device address (once per
- *    device, with that device current); make that first call before any stream
- *    capture.
+ *  - An expert id outside [0, E) is skipped as in moe_permute (row_of = -1, no
+ *    row); with no status block to record it in, the sign is offsets[E] < T*k.
+ *  - The first call on a device looks up the array's device address (with that
+ *    device current) and caches it for that device's CUDA context; make that
+ *    first call before any stream capture.  After cudaDeviceReset (a new
+ *    context) the next call looks the address up again, and so is again a
+ *    first call.
  *  - Every call on a device shares the one array and leaves its contents behind;
  *    nothing in it needs to start at zero.  Calls whose work overlaps on the GPU
  *    (e.g. on two streams at once) race on the array: order them on one stream. */

@@ -44,3 +44,40 @@ def assert_close(got_bits, ref_bits, tol=REL_TOL, what="output"):
 
 def assert_gates(gpu_gate: np.ndarray, ref_gate: np.ndarray):
     np.testing.assert_allclose(gpu_gate, ref_gate, rtol=1e-6, atol=1e-30)
+
+
+def assert_combine_close(got_bits, ref_bits, what="output"):
+    """Element-wise bound for a combine of the same bf16 rows with the same gates:
+    the two sides accumulate in fp32 in the same order but may round the products
+    differently (fused multiply-add against multiply then add), which can move the
+    final bf16 rounding by at most one bf16 ulp, i.e. |gpu - ref| <= 2^-7 |ref|."""
+    g, r = bf16_f64(got_bits), bf16_f64(ref_bits)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite values in the GPU output"
+    bad = np.abs(g - r) > np.abs(r) * 2.0 ** -7 + 1e-30
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond one bf16 ulp, e.g. " \
+        f"{g[bad][:3]} vs {r[bad][:3]}"
+
+
+def band_covering_tokens(offsets, perm, wl, n_random=48, band_rows=128, seed=None):
+    """Tokens to check through the oracle's definition path: for every 128-row band
+    of every expert (rows [offsets[e] + 128 i, ...)), the token of one seeded random
+    row of it; plus the first and last tokens and n_random seeded random tokens."""
+    rng = np.random.default_rng(wl.seed if seed is None else seed)
+    toks = [0, wl.T - 1]
+    for e in range(len(offsets) - 1):
+        for r0 in range(int(offsets[e]), int(offsets[e + 1]), band_rows):
+            r1 = min(r0 + band_rows, int(offsets[e + 1]))
+            toks.append(int(perm[rng.integers(r0, r1)]) // wl.k)
+    toks.extend(rng.choice(wl.T, size=min(n_random, wl.T), replace=False).tolist())
+    return np.unique(np.asarray(toks, np.int64)).astype(np.int32)
+
+
+def bands_covered(offsets, perm, wl, toks, band_rows=128) -> bool:
+    """Does every band hold a routed row of one of the tokens?"""
+    tset = set(int(t) for t in toks)
+    for e in range(len(offsets) - 1):
+        for r0 in range(int(offsets[e]), int(offsets[e + 1]), band_rows):
+            r1 = min(r0 + band_rows, int(offsets[e + 1]))
+            if not any(int(p) // wl.k in tset for p in perm[r0:r1]):
+                return False
+    return True

@@ -6,9 +6,17 @@
   variants; the overlapped mode bit-identical to the sequential mode
   for every consumer-SM count tried (cost model, 1, 2, 4, 8, 32), segment size
   mgb in {1, 2, 3} and with or without producers joining the combine.
-* Every benchmark workload at full size, in the configuration the benchmark
-  times: routing outputs in full, and a seeded sample of tokens through the
-  oracle's token-by-token definition path; overlapped == sequential in full."""
+* Every benchmark workload at full size (the Mixtral-shaped, fine-grained and
+  imbalanced layers and all twelve T x router layers of the d=4096/E=32 grid), in
+  the configuration the benchmark times: routing outputs in full; a sample of
+  tokens through the oracle's token-by-token definition path that holds at least
+  one routed row of every 128-row band (so every producer tile row group and
+  every consumer band is checked), plus the first and last tokens and a seeded
+  random set; overlapped == sequential in full.
+* The same layers with identity experts (MOE_DBG_IDENTITY_EXPERTS): route,
+  permute and combine, checked element by element over the whole output.
+* The oracle's fp32-intermediate variant (h kept in fp32): the GPU output is
+  within the same bound of it as of the bf16-h oracle."""
 import os
 
 import numpy as np
@@ -50,6 +58,18 @@ def test_layer_small(orc, wl):
     ref = orc.forward(gu.host(inp["x"]), gu.host(inp["logits"]), gu.host(inp["W1"]),
                       gu.host(inp["W3"]), gu.host(inp["W2"]), wl.k)
     pair = moe.SCHED_CTA_PAIR
+    if wl.name == "tiny":
+        # the fp32-intermediate reading of the oracle (h not rounded to bf16)
+        ref32 = orc.forward(gu.host(inp["x"]), gu.host(inp["logits"]), gu.host(inp["W1"]),
+                            gu.host(inp["W3"]), gu.host(inp["W2"]), wl.k, fp32_h=True)
+        dflt32, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED)
+        gu.assert_close(gu.host(dflt32), ref32["out"], what="tiny vs fp32-h oracle")
+        # identity experts: route, permute and combine alone, every element
+        refI = orc.forward(gu.host(inp["x"]), gu.host(inp["logits"]), None, None, None, wl.k,
+                           identity=True)
+        for mode in (moe.MODE_SEQUENTIAL, moe.MODE_OVERLAPPED):
+            outI, _, _ = _forward(inp, wl, ws, mode, flags=moe.DBG_IDENTITY_EXPERTS)
+            gu.assert_combine_close(gu.host(outI), refI["out"], what=f"tiny identity experts {mode}")
     seq, extra, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL, flags=pair)
     assert np.array_equal(gu.host(extra["topk_idx"]), ref["topk_idx"])
     gu.assert_gates(gu.host(extra["topk_gate"]), ref["topk_gate"])
@@ -106,8 +126,8 @@ def test_layer_repeat_bitwise():
         assert torch.equal(again, first)
 
 
-FULL = ["mixtral", "fine_grained", "imbalanced", "sweep_T512_hot", "sweep_T2048_uniform",
-        "sweep_T8192_zipf", "sweep_T32768_uniform"]
+FULL = ["mixtral", "fine_grained", "imbalanced"] + \
+    [f"sweep_T{T}_{r}" for T in (512, 2048, 8192, 32768) for r in ("uniform", "zipf", "hot")]
 # (workload, flags): every layer in its default variant (256-row single-CTA
 # tiles from 256 rows per expert up, 128-row tiles below), and the other variants
 # on a few
@@ -136,13 +156,35 @@ def test_layer_full_size_sampled(orc, name, flags):
     assert np.array_equal(gu.host(extra["counts"]), oc)
     assert np.array_equal(gu.host(extra["offsets"]), oo)
     assert np.array_equal(gu.host(extra["perm"]), op)
-    # sampled tokens through the definition path (always including the first and last)
-    n = 48 if wl.d * wl.f * wl.k > 4096 * 4096 * 4 else 96
-    rng = np.random.default_rng(wl.seed)
-    toks = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(wl.T, size=n, replace=False)])).astype(np.int32)
+    # sampled tokens through the definition path: one routed row of every band,
+    # the first and last tokens, and a seeded random set
+    toks = gu.band_covering_tokens(oo, op, wl, n_random=48 if wl.d * wl.f * wl.k > 4096 * 4096 * 4 else 96)
+    assert gu.bands_covered(oo, op, wl, toks)
     ref = orc.tokens(gu.host(inp["x"]), oidx, ogate, gu.host(inp["W1"]), gu.host(inp["W3"]),
                      gu.host(inp["W2"]), toks)
-    gu.assert_close(ovl_bits[toks], ref, what=f"{name} sampled tokens")
+    gu.assert_close(ovl_bits[toks], ref, what=f"{name} sampled tokens ({len(toks)})")
+    if name == "mixtral" and flags == 0:
+        # the fp32-intermediate reading of the oracle: within the same bound
+        ref32 = orc.tokens(gu.host(inp["x"]), oidx, ogate, gu.host(inp["W1"]), gu.host(inp["W3"]),
+                           gu.host(inp["W2"]), toks, fp32_h=True)
+        gu.assert_close(ovl_bits[toks], ref32, what=f"{name} sampled tokens vs fp32-h oracle")
+
+
+@pytest.mark.parametrize("name", ["fine_grained", "imbalanced", "sweep_T32768_zipf", "sweep_T512_hot"])
+def test_layer_full_size_identity_experts(orc, name):
+    """Identity experts: the whole output of route -> permute -> combine at full
+    size against the oracle's, element by element, in both modes."""
+    wl = synth.WORKLOADS[name]
+    orc.set_threads(os.cpu_count() or 1)
+    inp = gu.inputs(wl, weights=False)
+    ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
+    ref = orc.forward(gu.host(inp["x"]), gu.host(inp["logits"]), None, None, None, wl.k, identity=True)
+    for mode in (moe.MODE_SEQUENTIAL, moe.MODE_OVERLAPPED):
+        out, extra = moe.layer_forward(inp["x"], inp["logits"], None, None, None, wl.k, ws, mode,
+                                       outputs=True, flags=moe.DBG_IDENTITY_EXPERTS, d_ff=wl.f)
+        assert moe.get_status(ws)[0] == moe.MOE_OK
+        assert np.array_equal(gu.host(extra["perm"]), ref["perm"])
+        gu.assert_combine_close(gu.host(out), ref["out"], what=f"{name} identity experts, mode {mode}")
 
 
 def _check_variants(orc, wl, inp):
