@@ -87,6 +87,8 @@ def parse():
     ap.add_argument("--cta-pair", action="store_true", help="force 256-row tiles on CTA pairs")
     ap.add_argument("--wide-cta", action="store_true",
                     help="force 256-row tiles on single CTAs (two 128-row MMAs per K step)")
+    ap.add_argument("--flags", default="0",
+                    help="extra moe_layer_args.flags bits (e.g. 0x400 = MOE_SCHED_INTERLEAVE)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -257,7 +259,7 @@ def run_ours(args):
               flags=(moe.SCHED_NO_JOIN if args.no_join else 0) | (moe.SCHED_ONE_CTA if args.one_cta else 0)
               | (moe.SCHED_CTA_PAIR if args.cta_pair else 0)
               | (moe.SCHED_B_PER_ATOM if args.b_per_atom else 0)
-              | (moe.SCHED_WIDE_CTA if args.wide_cta else 0))
+              | (moe.SCHED_WIDE_CTA if args.wide_cta else 0) | int(args.flags, 0))
 
     def step(mode, evb=None, eve=None):
         moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, mode, out=out, ev_begin=evb, ev_end=eve, **kw)
@@ -650,16 +652,19 @@ def run_oracle_timings(args):
 
 
 def _sweep_cells(spec: str):
-    """Cells of a paired sweep: "seq" (sequential mode) or "C[/mgb]" (overlapped mode,
-    C consumer SMs, 0 = the cost model; mgb row bands per consumer item)."""
+    """Cells of a paired sweep: "seq[+flags]" (sequential mode) or "C[/mgb][+flags]"
+    (overlapped mode, C consumer SMs, 0 = the cost model; mgb row bands per consumer
+    item; flags = extra moe_layer_args.flags bits, e.g. +0x400)."""
     cells = []
     for tok in spec.split(","):
         tok = tok.strip()
-        if tok == "seq":
-            cells.append(("seq", None, 0, 1))
+        body, _, fl = tok.partition("+")
+        flags = int(fl, 0) if fl else 0
+        if body == "seq":
+            cells.append((tok, None, 0, 1, flags))
         else:
-            c, _, m = tok.partition("/")
-            cells.append((tok, "ovl", int(c), int(m) if m else 1))
+            c, _, m = body.partition("/")
+            cells.append((tok, "ovl", int(c), int(m) if m else 1, flags))
     return cells
 
 
@@ -688,9 +693,10 @@ def run_sweep(args):
         t_roof = max(F / (peak_tf * 1e12), B / (peaks["hbm_gbs"] * 1e9)) * 1e3
 
         def step(cell):
-            _, mode, C, mgb = cell
+            _, mode, C, mgb, fl = cell
             m = moe.MODE_SEQUENTIAL if mode is None else moe.MODE_OVERLAPPED
-            moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, m, out=out, consumer_sms=C, mgb=mgb)
+            moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, m, out=out, consumer_sms=C, mgb=mgb,
+                              flags=fl)
 
         used = {}
         for cell in cells:
@@ -736,6 +742,9 @@ def run_sweep(args):
                 cell["consumer_sms_used"] = used[c]
             if "seq" in med and c != "seq":
                 cell["speedup_vs_sequential"] = med["seq"] / med[c]
+            base = cells[0][0]
+            if c != base:
+                cell[f"ratio_vs_{base}"] = med[base] / med[c]
             res["cells"][c] = cell
         res["clocks"] = clk.summary(name)
         print(json.dumps(res), flush=True)

@@ -31,7 +31,7 @@ struct Layout {
   size_t status, sync, stamps, blk_hist, blk_base, counts, offsets, topk_idx, topk_gate, perm, row_of, arrive, ready_q;
   size_t routing_end;
   size_t sorted_e, band_start, tile_start1, bands, band_done1, band_done2, groups, group_start,
-      tok_band, expert_rank;
+      tok_band, expert_rank, band_dest;
   size_t plan_end;
   size_t x_perm, h, y;
   size_t total;
@@ -67,6 +67,7 @@ Layout layout(int T, int d, int f, int E, int k) {
   L.group_start = o; o = up(o + (size_t)(E + 1) * 4);
   L.tok_band = o; o = up(o + mb * BM * 4);
   L.expert_rank = o; o = up(o + (size_t)E * 4);
+  L.band_dest = o; o = up(o + mb * sizeof(int2));
   L.plan_end = o;
   L.x_perm = o; o = up(o + R * d * 2);
   L.h = o; o = up(o + R * f * 2);
@@ -74,6 +75,9 @@ Layout layout(int T, int d, int f, int E, int k) {
   L.total = o;
   return L;
 }
+
+// Band-table capacity of a layout (the band_dest region holds one int2 per band).
+int max_bands_of(const Layout& L) { return (int)((L.plan_end - L.band_dest) / sizeof(int2)); }
 
 template <class T>
 T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
@@ -105,6 +109,7 @@ Work work_from(void* ws, const Layout& L, bool plan, bool acts) {
     w.group_start = at<int32_t>(ws, L.group_start);
     w.tok_band = at<int32_t>(ws, L.tok_band);
     w.expert_rank = at<int32_t>(ws, L.expert_rank);
+    // the combine plan exists only for an expert-parallel owner (set by its entry)
   }
   if (acts) {
     w.x_perm = at<__nv_bfloat16>(ws, L.x_perm);
@@ -285,7 +290,8 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
       !ok_ptr(y) || !ok_opt(h))
     return MOE_ERR_INVALID;
   constexpr unsigned tile_flags = MOE_SCHED_ONE_CTA | MOE_SCHED_CTA_PAIR | MOE_SCHED_WIDE_CTA |
-                                  MOE_SCHED_B_PER_ATOM | MOE_SCHED_FULL_TILES;
+                                  MOE_SCHED_B_PER_ATOM | MOE_SCHED_FULL_TILES |
+                                  MOE_SCHED_INTERLEAVE | MOE_SCHED_EVICT_FIRST;
   if (flags & ~tile_flags) return MOE_ERR_INVALID;
   const Layout L = layout(T, d, f, E, k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
@@ -305,6 +311,7 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
   a.y = static_cast<__nv_bfloat16*>(y);
   a.W1 = W1; a.W3 = W3; a.W2 = W2;
   a.R = T * k; a.T = T; a.d = d; a.f = f; a.E = E; a.k = k;
+  a.n_units = E;
   a.V = V;
   a.phase = PH_G1 | PH_G2;
   a.join = 0;
@@ -397,6 +404,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   a.gate = w.topk_gate;
   a.out = static_cast<__nv_bfloat16*>(A.out);
   a.R = R; a.T = T; a.d = d; a.f = f; a.E = E; a.k = k;
+  a.n_units = E;
   a.V = V;
   a.mgb = mgb;
   a.flags = A.flags;
@@ -418,6 +426,120 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
     if (A.ev_ffn_end) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_end), st));
     MOE_TRY(launch_combine(w.y, w.row_of, w.topk_gate, T, d, k, a.out, nsm, st));
   }
+  return MOE_OK;
+}
+
+size_t moe_ep_owner_workspace_size(int N, int d, int f, int El, int W) {
+  if (N < 0 || d < 1 || f < 1 || El < 1 || W < 1 || W > MAX_W || (long long)El * W > MAX_E) return 0;
+  if (d % BN2 != 0 || f % BN1 != 0) return 0;
+  if ((long long)N * (d > f ? d : f) >= (1LL << 40)) return 0;
+  // rows N (k = 1), planning units W * El
+  return layout(N > 0 ? N : 1, d, f, El * W, 1).total;
+}
+
+moe_status moe_ep_owner_forward(const moe_ep_owner_args* args, moe_mode mode, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (!args) return MOE_ERR_INVALID;
+  const moe_ep_owner_args& A = *args;
+  if (A.W < 1 || A.rank < 0 || A.rank >= A.W || A.El < 1 || A.N < 0 || A.d < 1 || A.f < 1 ||
+      A.k < 1)
+    return MOE_ERR_INVALID;
+  if (A.W > MAX_W || (long long)A.El * A.W > MAX_E || A.k > MAX_K) return MOE_ERR_UNSUPPORTED;
+  if (A.d % BN2 != 0 || A.f % BN1 != 0) return MOE_ERR_UNSUPPORTED;
+  if ((long long)A.N * (A.d > A.f ? A.d : A.f) >= (1LL << 40)) return MOE_ERR_UNSUPPORTED;
+  if (mode != MOE_MODE_SEQUENTIAL && mode != MOE_MODE_OVERLAPPED) return MOE_ERR_INVALID;
+  if (A.consumer_sms < 0 || A.mgb < 0 || A.timeout_us < 0) return MOE_ERR_INVALID;
+  if (!ok_ptr(A.x_recv) || !ok_ptr(A.slot_recv) || !ok_ptr(A.recv_counts) || !ok_ptr(A.W1) ||
+      !ok_ptr(A.W3) || !ok_ptr(A.W2))
+    return MOE_ERR_INVALID;
+  for (int r = 0; r < A.W; ++r) {
+    if (!ok_ptr(A.home_y[r]) || !A.home_arrive[r] || (reinterpret_cast<uintptr_t>(A.home_arrive[r]) & 3u))
+      return MOE_ERR_INVALID;
+    if (A.recv_base[r] < 0) return MOE_ERR_INVALID;
+  }
+  const int U = A.El * A.W;
+  const Layout L = layout(A.N > 0 ? A.N : 1, A.d, A.f, U, 1);
+  if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const int nsm = device_sms();
+  int V = choose_variant(A.N > 0 ? A.N : 1, A.f, U, 1, A.flags);
+  int grid = 0;
+  MOE_TRY(ffn_grid(V, &grid));
+  if (nsm <= 1 || grid <= ctas_per_tile(V)) return cuda_fail(cudaErrorInvalidConfiguration);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Work w = work_from(ws, L, true, true);
+  w.band_dest = at<int2>(ws, L.band_dest);
+  w.tok_band = nullptr;
+  w.expert_rank = nullptr;
+  const int mgb = A.mgb > 0 ? A.mgb : 1;
+  const int join = (A.flags & MOE_SCHED_NO_JOIN) ? 0 : 1;
+  EpPlanIn in;
+  memset(&in, 0, sizeof(in));
+  in.W = A.W; in.rank = A.rank; in.El = A.El; in.N = A.N;
+  for (int r = 0; r < A.W; ++r) in.recv_base[r] = A.recv_base[r];
+  MOE_TRY(launch_plan_ep(w, A.recv_counts, in, A.d, A.f, grid, A.consumer_sms, mgb, bands_per_tile(V),
+                         ctas_per_tile(V), join, default_cost_model(), st));
+  if (A.N == 0) return MOE_OK;   // nothing received: no tile, no row to return
+  FfnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.w = w;
+  a.x_perm = static_cast<const __nv_bfloat16*>(A.x_recv);
+  a.h = w.h;
+  a.y = w.y;
+  a.W1 = A.W1; a.W3 = A.W3; a.W2 = A.W2;
+  a.R = A.N; a.T = A.N; a.d = A.d; a.f = A.f; a.E = A.El; a.k = A.k;
+  a.n_units = U;
+  a.V = V;
+  a.mgb = mgb;
+  a.flags = A.flags & ~(MOE_SCHED_GATHER_A | MOE_DBG_IDENTITY_EXPERTS);
+  a.timeout_ns = (A.timeout_us > 0 ? (uint64_t)A.timeout_us : 2000000ull) * 1000ull;
+  a.ep = 1;
+  a.ep_slot = A.slot_recv;
+  for (int r = 0; r < A.W; ++r) {
+    a.ep_home_y[r] = A.home_y[r];
+    a.ep_home_arrive[r] = A.home_arrive[r];
+  }
+  if (mode == MOE_MODE_OVERLAPPED) {
+    a.phase = PH_G1 | PH_G2 | PH_CONS;
+    a.join = join;
+    MOE_TRY(launch_ffn(a, grid, st));
+  } else {
+    // the baseline: expert compute, then the whole return as a separate pass
+    a.phase = PH_G1;
+    MOE_TRY(launch_ffn(a, grid, st));
+    a.phase = PH_G2;
+    MOE_TRY(launch_ffn(a, grid, st));
+    a.phase = PH_CONS;
+    a.join = 1;
+    MOE_TRY(launch_ffn(a, grid, st));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_ep_home_combine(const void* home_y, uint32_t* arrive, const int32_t* row_of,
+                               const float* topk_gate, int T, int d, int k, void* out,
+                               uint32_t* status, int timeout_us, void* stream) {
+  if (T < 1 || d < 1 || k < 1 || timeout_us < 0) return MOE_ERR_INVALID;
+  if (k > MAX_K || d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!ok_ptr(home_y) || !ok_ptr(arrive) || !ok_ptr(row_of) || !ok_ptr(topk_gate) || !ok_ptr(out) ||
+      !status || (reinterpret_cast<uintptr_t>(status) & 3u))
+    return MOE_ERR_INVALID;
+  const int nsm = device_sms();
+  if (nsm <= 0) return cuda_fail(cudaErrorInvalidDevice);
+  const uint64_t tmo = (timeout_us > 0 ? (uint64_t)timeout_us : 2000000ull) * 1000ull;
+  return cuda_status(launch_home_combine(static_cast<const __nv_bfloat16*>(home_y), arrive, row_of,
+                                         topk_gate, T, d, k, static_cast<__nv_bfloat16*>(out), status,
+                                         tmo, nsm, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_ep_debug_plan(void* ws, int N, int d, int f, int El, int W, void* stream,
+                             int32_t* host_out, int max_bands) {
+  if (!ws || !aligned16(ws) || !host_out || max_bands < 1) return MOE_ERR_INVALID;
+  if (moe_ep_owner_workspace_size(N, d, f, El, W) == 0) return MOE_ERR_INVALID;
+  MOE_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  const Layout L = layout(N > 0 ? N : 1, d, f, El * W, 1);
+  const int mb = max_bands < max_bands_of(L) ? max_bands : max_bands_of(L);
+  MOE_TRY(cudaMemcpy(host_out, static_cast<char*>(ws) + L.band_dest, (size_t)mb * sizeof(int2),
+                     cudaMemcpyDeviceToHost));
   return MOE_OK;
 }
 

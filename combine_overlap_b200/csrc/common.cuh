@@ -32,6 +32,7 @@ constexpr int STAMP_BANDS = 2048;  // debug per-band stamps: at most this many b
 constexpr int MAX_E = 256;
 constexpr uint32_t TOKEN_DONE = 0x80000000u;   // arrive[t] flag: a consumer combined token t
 constexpr int MAX_K = 8;
+constexpr int MAX_W = 8;        // ranks of an expert-parallel group
 
 // ----------------------------------------------------------------- status ---
 // ST_INVALID: a caller-supplied expert id outside [0, E) (moe_permute); ST_TIMEOUT: a
@@ -108,6 +109,8 @@ struct Work {
   uint32_t* arrive;     // [T] rows of token t that have arrived; TOKEN_DONE set once out[t]
                         // is written by a consumer
   uint32_t* ready_q;    // [T] tokens whose k rows all arrived (t + 1; 0 = entry not yet written)
+  int2* band_dest;      // [max_bands] expert-parallel owner: (home rank, home row of the band's
+                        // first row) -- the combine plan; null on one GPU
   Sync* sync;
   Status* status;
   unsigned long long* stamps;  // [STAMP_CTAS][NSTAMP] debug timestamps (MOE_DBG_TIMESTAMPS),
@@ -161,6 +164,31 @@ __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
   uint32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
+}
+
+// An L2 cache policy that marks the lines a store writes as first to evict.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 16-byte global store with an L2 cache policy.
+__device__ __forceinline__ void st_global_v4_policy(void* ptr, uint4 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;"
+               :: "l"(ptr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy) : "memory");
+}
+
+// System-scope release add and acquire load: arrival words that another GPU's
+// kernel (or, on one GPU, another rank's kernel) writes or reads over NVLink.
+__device__ __forceinline__ void red_release_sys_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.sys.global.add.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -287,14 +287,34 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
   unsigned long long* my_stamps = w.stamps + (size_t)blockIdx.x * NSTAMP;
   unsigned long long n_g1 = 0, n_g2 = 0;
 
+  // With MOE_SCHED_INTERLEAVE, GEMM2 tiles interleave with GEMM1 tiles: while
+  // GEMM1 tiles remain, the scheduler takes the head GEMM2 tile if every GEMM1
+  // tile of its row group is already stored (a peek, then a compare-and-swap on
+  // the queue head), else the next GEMM1 tile.  A GEMM2 tile taken this way never
+  // waits; once the GEMM1 queue is empty, GEMM2 tiles are taken unconditionally,
+  // and each of them waits only on GEMM1 tiles that resident CTAs have dequeued.
+  const bool interleave = (a.flags & MOE_SCHED_INTERLEAVE) != 0;
+  auto group_stored = [&](int group) {
+    const Group gr = w.groups[group];
+    if (ld_acquire(&w.band_done1[gr.band0]) < BAND_UNIT * (uint32_t)NT1) return false;
+    return gr.rows <= BM || ld_acquire(&w.band_done1[gr.band0 + 1]) >= BAND_UNIT * (uint32_t)NT1;
+  };
   // Next work item: dequeued and published by a leader, read by a peer.
   auto next_item = [&](Item& it) -> bool {
     if (leader) {
       it.kind = K_END;
       if (*abort) g1 = g2 = false;
-      if (g1) {
+      if (g1 && g2 && interleave) {
+        uint32_t t2 = *reinterpret_cast<volatile uint32_t*>(&w.sync->q2);
+        while (t2 < (uint32_t)n2 && group_stored((int)t2 / NT2)) {
+          const uint32_t seen = atomicCAS(&w.sync->q2, t2, t2 + 1u);
+          if (seen == t2) { it = decode_g2(w, (int)t2, NT2); break; }
+          t2 = seen;   // another CTA took it: look at the new head
+        }
+      }
+      if (it.kind == K_END && g1) {
         const int t = (int)atomicAdd(&w.sync->q1, 1u);
-        if (t < n1) it = decode_g1(w, t, a.E);
+        if (t < n1) it = decode_g1(w, t, a.n_units);
         else {
           g1 = false;
           if (stamp) my_stamps[1] = globaltimer();
@@ -563,7 +583,7 @@ static_assert(EPI_WARPS == 8, "the epilogue splits each accumulator's columns be
 // the tile is published.
 __device__ __forceinline__ void store_chunk(uint8_t* ost, const uint32_t (&pk)[16], int lane,
                                             unsigned vmask, __nv_bfloat16* base_row0,
-                                            size_t ld, int col) {
+                                            size_t ld, int col, bool evict_first, uint64_t pol) {
 #pragma unroll
   for (int v = 0; v < 4; ++v)
     *reinterpret_cast<uint4*>(ost + lane * OSTAGE_ROW + v * 16) =
@@ -573,8 +593,11 @@ __device__ __forceinline__ void store_chunk(uint8_t* ost, const uint32_t (&pk)[1
   for (int v = 0; v < 4; ++v) {
     const int r = (lane >> 2) + 8 * v;            // row of the warp this lane writes
     const uint4 val = *reinterpret_cast<const uint4*>(ost + r * OSTAGE_ROW + (lane & 3) * 16);
-    if ((vmask >> r) & 1u)
-      *reinterpret_cast<uint4*>(base_row0 + (size_t)r * ld + col + (lane & 3) * 8) = val;
+    if ((vmask >> r) & 1u) {
+      uint4* dst = reinterpret_cast<uint4*>(base_row0 + (size_t)r * ld + col + (lane & 3) * 8);
+      if (evict_first) st_global_v4_policy(dst, val, pol);
+      else *dst = val;
+    }
   }
   __syncwarp();
 }
@@ -585,6 +608,8 @@ __device__ __forceinline__ void drain_acc(const FfnArgs& a, int kind, uint32_t t
   const int lane = threadIdx.x & 31;
   const unsigned vmask = __ballot_sync(0xffffffffu, valid);
   const size_t row0 = row - (size_t)lane;         // the warp's first row
+  const bool ef = (a.flags & MOE_SCHED_EVICT_FIRST) != 0;
+  const uint64_t pol = ef ? l2_policy_evict_first() : 0ull;
   if (kind == K_G1) {
     __nv_bfloat16* base = a.h + row0 * a.f + col0;
 #pragma unroll 1
@@ -598,7 +623,7 @@ __device__ __forceinline__ void drain_acc(const FfnArgs& a, int kind, uint32_t t
       for (int i = 0; i < 16; ++i)
         pk[i] = pack_bf16x2(silu_mul(__uint_as_float(ra[2 * i]), __uint_as_float(rb[2 * i])),
                             silu_mul(__uint_as_float(ra[2 * i + 1]), __uint_as_float(rb[2 * i + 1])));
-      store_chunk(ost, pk, lane, vmask, base, (size_t)a.f, c * 32);
+      store_chunk(ost, pk, lane, vmask, base, (size_t)a.f, c * 32, ef, pol);
     }
   } else {
     __nv_bfloat16* base = a.y + row0 * a.d + col0;
@@ -610,7 +635,7 @@ __device__ __forceinline__ void drain_acc(const FfnArgs& a, int kind, uint32_t t
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
-      store_chunk(ost, pk, lane, vmask, base, (size_t)a.d, c * 32);
+      store_chunk(ost, pk, lane, vmask, base, (size_t)a.d, c * 32, ef, pol);
     }
   }
 }
@@ -948,6 +973,83 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
     w.stamps[(size_t)blockIdx.x * NSTAMP + 6] = n_bands_done;
 }
 
+// ------------------------------------------------------------- EP return ---
+// The consumer role of an expert-parallel owner: the return all-to-all of "Fine-
+// grained Computation-Communication Overlap via Tile-level Signaling and
+// Scheduling for Mixture-of-Experts", fused into the persistent kernel
+// (Sections 3.3.2-3.3.3).  A consuming CTA takes the next segment item (mgb row
+// bands; the first and last items one band each) by ticket, waits (bounded) until
+// every band of it is flagged, and moves each band -- its rows are contiguous on
+// both sides -- into its home rank's return buffer at the combine plan's row,
+// with 16-byte loads and stores (no TMA, no loads from the home's memory).  It
+// then fences at system scope and adds 1 to the home's arrival word of each row's
+// token with a system-scope release, so the home can combine a token as soon as
+// its k rows have landed.  Unlike the one-GPU combine, consumers keep going until
+// every item is returned: nothing is left for a later pass.
+__device__ void role_return(const FfnArgs& a, SmemCtl* ctl, int nb, int n_items,
+                            const volatile uint32_t* abort) {
+  const Work& w = a.w;
+  const uint32_t NT2 = (uint32_t)(a.d / BN2);
+  const int dv = a.d >> 3;
+  const int k = a.k;
+  constexpr int U = 4;   // 16-byte vectors in flight per thread
+  while (true) {
+    if (threadIdx.x == 0) {
+      int act = C_DONE, b0 = 0, b1 = 0;
+      if (*abort) act = C_ERROR;
+      else {
+        const int t = (int)atomicAdd(&w.sync->qc, 1u);
+        if (t < n_items) {
+          item_range(t, nb, a.mgb, b0, b1);
+          bool ok = true;
+          for (int b = b0; b < b1 && ok; ++b)
+            ok = wait_count(&w.band_done2[b], BAND_UNIT * NT2, a.timeout_ns, abort);
+          if (ok) act = C_BAND;
+          else { set_error(w.status, W_CONS_QUEUE); act = C_ERROR; }
+        }
+      }
+      ctl->item = act;
+      ctl->ok = b0;
+      ctl->cn = b1;
+    }
+    __syncthreads();
+    const int act = ctl->item, b0 = ctl->ok, b1 = ctl->cn;
+    __syncthreads();
+    if (act != C_BAND) break;
+    for (int b = b0; b < b1; ++b) {
+      const Band bd = w.bands[b];
+      const int2 dst = w.band_dest[b];
+      const uint4* src = reinterpret_cast<const uint4*>(a.y) + (size_t)bd.row0 * dv;
+      uint4* home = reinterpret_cast<uint4*>(a.ep_home_y[dst.x]) + (size_t)dst.y * dv;
+      const size_t n = (size_t)bd.rows * dv;
+      for (size_t i0 = threadIdx.x; i0 < n; i0 += (size_t)FFN_THREADS * U) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const size_t i = i0 + (size_t)u * FFN_THREADS;
+          if (i < n) v[u] = __ldcg(src + i);   // y rows were stored by other SMs: read through L2
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const size_t i = i0 + (size_t)u * FFN_THREADS;
+          if (i < n) home[i] = v[u];
+        }
+      }
+    }
+    __threadfence_system();   // the rows reach the home before any arrival below
+    __syncthreads();
+    for (int b = b0; b < b1; ++b) {
+      const Band bd = w.bands[b];
+      uint32_t* arrive = a.ep_home_arrive[w.band_dest[b].x];
+      for (int r = threadIdx.x; r < bd.rows; r += FFN_THREADS)
+        red_release_sys_add(&arrive[a.ep_slot[bd.row0 + r] / k], 1u);
+    }
+    if (threadIdx.x == 0 && (a.flags & MOE_DBG_TIMESTAMPS) && blockIdx.x < STAMP_CTAS)
+      w.stamps[(size_t)blockIdx.x * NSTAMP + 6] += (unsigned long long)(b1 - b0);
+    __syncthreads();
+  }
+}
+
 // ------------------------------------------------------------------- kernel ---
 template <int V>
 __global__ void __launch_bounds__(FFN_THREADS, 1)
@@ -997,9 +1099,14 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   Status* st = a.w.status;
   const volatile uint32_t* abort = &st->code;
   const int n1 = st->n_tiles1, n2 = st->n_tiles2, nb = st->n_bands, n_items = st->n_items;
-  // consumer CTAs come in whole tiles' CTAs (the plan rounds C to a multiple of cg)
+  // consumer CTAs come in whole tiles' CTAs (the plan rounds C to a multiple of cg).
+  // With GEMM2 tiles interleaved (MOE_SCHED_INTERLEAVE), bands complete from early
+  // on, so the consumers are a partition of their own from the start (the paper's
+  // disjoint SM subsets); otherwise no band completes before the GEMM1 queue
+  // drains, and the consumers help with GEMM1 until then.
   const bool consumer_cta = (a.phase & PH_CONS) && (int)blockIdx.x < st->consumer_sms;
-  const bool run_g1 = (a.phase & PH_G1) != 0;
+  const bool interleaved = (a.phase & PH_G1) && (a.phase & PH_G2) && (a.flags & MOE_SCHED_INTERLEAVE);
+  const bool run_g1 = (a.phase & PH_G1) && !(consumer_cta && interleaved);
   const bool run_g2 = (a.phase & PH_G2) && !consumer_cta;
   const bool do_consume = (a.phase & PH_CONS) && (consumer_cta || a.join);
   const bool stamp = (a.flags & MOE_DBG_TIMESTAMPS) && blockIdx.x < STAMP_CTAS;
@@ -1028,7 +1135,10 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
   // A pair's peer may still be read by the leader's MMAs until the leader is
   // done; nobody reuses the operand ring before both CTAs finished producing.
   if (V == 2) cluster_sync();
-  if (do_consume) role_consumer(a, ctl, smem, nb, n_items, abort);
+  if (do_consume) {
+    if (a.ep) role_return(a, ctl, nb, n_items, abort);
+    else role_consumer(a, ctl, smem, nb, n_items, abort);
+  }
   __syncthreads();
   if (stamp && threadIdx.x == 0) my_stamps[3] = globaltimer();
   if (V == 2) cluster_sync();

@@ -47,6 +47,24 @@ cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int 
 // With a plan (w.bands etc. set), also fills w.tok_band, GEMM1's gather indices.
 cudaError_t launch_scatter(const int32_t* topk_idx, int T, int E, int k, const int32_t* blk_base,
                            int32_t* perm, int32_t* row_of, const Work* plan, cudaStream_t s);
+// Expert-parallel owner plan: the owner's received rows (source rank major, then
+// local expert) are planned as W*El segments (local expert e, source s), each a
+// contiguous run of rows with one destination; bands and tiles follow the
+// remote-first order.  recv_base[s]: home row of the first row source s sent.
+struct EpPlanIn {
+  int W, rank, El, N;
+  int recv_base[MAX_W];
+};
+cudaError_t launch_plan_ep(const Work& w, const int32_t* recv_counts, const EpPlanIn& in, int d,
+                           int f, int num_sms, int consumer_hint, int mgb, int G, int cg, int join,
+                           const CostModel& cm, cudaStream_t s);
+// Home side of the expert-parallel return: waits (bounded) for each token's k rows
+// to arrive, combines them exactly as launch_combine does, and zeroes its arrival
+// word; a wait that runs out sets *status to MOE_ERR_TIMEOUT (if it was 0).
+cudaError_t launch_home_combine(const __nv_bfloat16* y, uint32_t* arrive, const int32_t* row_of,
+                                const float* gate, int T, int d, int k, __nv_bfloat16* out,
+                                uint32_t* status, uint64_t timeout_ns, int num_sms, cudaStream_t s);
+
 // x_perm[row_of[p]] = x[p / k] for every slot p < T*k (token-major copy).
 cudaError_t launch_gather(const __nv_bfloat16* x, const int32_t* row_of, int T, int d, int k,
                           __nv_bfloat16* x_perm, int num_sms, cudaStream_t s);
@@ -80,6 +98,16 @@ struct FfnArgs {
   int b_atoms;                   // single CTA: weight maps are 4-D, one box carries all 64-column atoms
   uint32_t flags;
   uint64_t timeout_ns;
+  int n_units;                   // planning units in w.tile_start1 / w.group_start: E on one
+                                 // GPU, (local expert, source rank) segments for an EP owner
+  // Expert-parallel owner (ep != 0): the consumer role returns each finished band to
+  // its home rank instead of combining: the band's rows are copied to
+  // ep_home_y[rank] at the combine plan's row (w.band_dest), then the arrival word
+  // of each row's token (ep_slot[row] / k) is bumped in ep_home_arrive[rank].
+  int ep;
+  const int32_t* ep_slot;        // [rows] home slot p = t*k + j of each owner row
+  void* ep_home_y[MAX_W];        // [R_home][d] bf16 return buffer of each home rank
+  uint32_t* ep_home_arrive[MAX_W];  // [T_home] arrival words of each home rank
 };
 
 size_t ffn_smem_bytes();

@@ -221,6 +221,104 @@ __device__ int warp_scan_smem(int* a, int n, int lane) {
   return __shfl_sync(0xffffffffu, inc, 31);
 }
 
+// The tile plan shared by the one-GPU plan and the expert-parallel owner plan.
+// U planning units (experts; or an owner's (local expert, source rank) segments)
+// in priority order sorted[0..U); unit u has cnt[u] rows from row row0[u],
+// computes with expert unit_e[u] (null: u itself) and, for an owner, returns to
+// rank dest[u] at home row home0[u] (null on one GPU).  Writes the per-unit
+// band/group/GEMM1-tile starts, the status block (`code`, the consumer split, the
+// counts) and a zeroed sync block; with w.bands set also the band and group
+// tables, the combine plan (w.band_dest) and zeroed band counters.
+__device__ void plan_tables(const Work& w, int U, const int* cnt, const int* row0,
+                            const int* unit_e, const int* dest, const int* home0,
+                            const int* sorted, uint32_t code, long long R, int T, int d, int f,
+                            int num_sms, int consumer_hint, int mgb, int G, int cg, int join,
+                            const CostModel& cm) {
+  __shared__ int bstart[MAX_E + 1];
+  __shared__ int gstart[MAX_E + 1];
+  __shared__ int t1start[MAX_E + 1];
+  __shared__ int totals[3];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NT1 = f / BN1, NT2 = d / BN2;
+  // bands, groups and GEMM1 tiles of the units in priority order, prefix-summed
+  for (int s2 = tid; s2 < U; s2 += blockDim.x) {
+    const int bands = cdiv(cnt[sorted[s2]], BM);
+    const int groups = cdiv(bands, G);
+    bstart[s2] = bands;
+    gstart[s2] = groups;
+    t1start[s2] = groups * NT1;
+  }
+  __syncthreads();
+  if (warp < 3) {
+    int* arr = warp == 0 ? bstart : (warp == 1 ? gstart : t1start);
+    const int total = warp_scan_smem(arr, U, lane);
+    if (lane == 0) { arr[U] = total; totals[warp] = total; }
+  }
+  __syncthreads();
+  const int nb = totals[0], ng = totals[1], nt1 = totals[2];
+  if (w.bands) {
+    for (int s2 = tid; s2 <= U; s2 += blockDim.x) {
+      w.band_start[s2] = bstart[s2];
+      w.group_start[s2] = gstart[s2];
+      w.tile_start1[s2] = t1start[s2];
+    }
+  }
+  if (tid == 0) {
+    const int cmin = join ? 0 : cg;
+    int C = consumer_hint > 0 ? consumer_hint : choose_consumers(num_sms, cg, cmin, R, T, d, f, cm);
+    C = cg * cdiv(C, cg);                       // consumers come in whole CTA groups
+    C = max(cmin, min(C, num_sms - cg));        // and leave at least one producer group
+    Status st;
+    st.code = code;
+    st.consumer_sms = C;
+    st.n_bands = nb;
+    st.n_tiles1 = nt1;
+    st.n_tiles2 = ng * NT2;
+    st.where = W_NONE;
+    st.n_items = n_items_for(nb, mgb);
+    st.n_groups = ng;
+    *w.status = st;
+    Sync z;
+    z.q1 = z.q2 = z.qc = z.rq_alloc = z.rq_head = z.prod_done = 0;
+    z.pad[0] = z.pad[1] = 0;
+    *w.sync = z;
+  }
+  if (w.bands == nullptr) return;   // permutation only: no tile plan wanted
+  for (int s = tid; s < U; s += blockDim.x) {
+    w.sorted_e[s] = sorted[s];
+    if (w.expert_rank) w.expert_rank[sorted[s]] = s;
+  }
+  __syncthreads();
+  for (int s = tid; s < U; s += blockDim.x) {
+    const int u = sorted[s];
+    const int e = unit_e ? unit_e[u] : u;
+    const int b0 = bstart[s], nbe = bstart[s + 1] - b0;
+    for (int i = 0; i < nbe; ++i) {
+      Band bd;
+      bd.expert = e;
+      bd.row0 = row0[u] + i * BM;
+      bd.rows = min(BM, cnt[u] - i * BM);
+      bd.pad = 0;
+      w.bands[b0 + i] = bd;
+      if (w.band_dest && dest) w.band_dest[b0 + i] = make_int2(dest[u], home0[u] + i * BM);
+    }
+    const int g0 = gstart[s], nge = gstart[s + 1] - g0;
+    for (int i = 0; i < nge; ++i) {
+      Group gr;
+      gr.expert = e;
+      gr.band0 = b0 + i * G;
+      gr.row0 = row0[u] + i * G * BM;
+      gr.rows = min(G * BM, cnt[u] - i * G * BM);
+      w.groups[g0 + i] = gr;
+    }
+  }
+  for (int i = tid; i < nb; i += blockDim.x) { w.band_done1[i] = 0u; w.band_done2[i] = 0u; }
+  if (w.tok_band) {
+    int4* tb = reinterpret_cast<int4*>(w.tok_band);
+    for (int i = tid; i < nb * (BM / 4); i += blockDim.x) tb[i] = make_int4(0, 0, 0, 0);
+  }
+}
+
 __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int32_t* offsets_in,
                                                     int T, int d, int f, int E, int k, int num_sms,
                                                     int consumer_hint, int mgb, int G, int cg,
@@ -230,11 +328,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
   __shared__ int cnt[MAX_E];
   __shared__ int offs[MAX_E + 1];
   __shared__ int sorted[MAX_E];
-  __shared__ int bstart[MAX_E + 1];
-  __shared__ int gstart[MAX_E + 1];
-  __shared__ int t1start[MAX_E + 1];
   __shared__ int part[1024];        // [g][e]: rows' sums of chunk g, then its exclusive base
-  __shared__ int totals[3];
   __shared__ int bad_in;            // caller-supplied offsets were not a valid scan
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) bad_in = 0;
@@ -320,92 +414,117 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
     sorted[r] = e;
   }
   __syncthreads();
-  const int NT1 = f / BN1, NT2 = d / BN2;
-  // bands, groups and GEMM1 tiles of the experts in priority order, prefix-summed
-  for (int s2 = tid; s2 < E; s2 += blockDim.x) {
-    const int bands = cdiv(cnt[sorted[s2]], BM);
-    const int groups = cdiv(bands, G);
-    bstart[s2] = bands;
-    gstart[s2] = groups;
-    t1start[s2] = groups * NT1;
-  }
-  __syncthreads();
-  if (warp < 3) {
-    int* arr = warp == 0 ? bstart : (warp == 1 ? gstart : t1start);
-    const int total = warp_scan_smem(arr, E, lane);
-    if (lane == 0) { arr[E] = total; totals[warp] = total; }
-  }
-  __syncthreads();
-  const int nb = totals[0], ng = totals[1], nt1 = totals[2];
-  if (w.bands) {
-    for (int s2 = tid; s2 <= E; s2 += blockDim.x) {
-      w.band_start[s2] = bstart[s2];
-      w.group_start[s2] = gstart[s2];
-      w.tile_start1[s2] = t1start[s2];
-    }
-  }
-  if (tid == 0) {
-    const long long R = offs[E];
-    // ids from the caller (nblk > 0 and no route kernel before us) that fell outside
-    // [0, E) were not counted: the total comes up short of T*k
-    const int cmin = join ? 0 : cg;
-    int C = consumer_hint > 0 ? consumer_hint : choose_consumers(num_sms, cg, cmin, R, T, d, f, cm);
-    C = cg * cdiv(C, cg);                       // consumers come in whole CTA groups
-    C = max(cmin, min(C, num_sms - cg));        // and leave at least one producer group
-    Status st;
-    st.code = (bad_in || (nblk > 0 && R != (long long)T * k)) ? ST_INVALID : ST_OK;
-    st.consumer_sms = C;
-    st.n_bands = nb;
-    st.n_tiles1 = nt1;
-    st.n_tiles2 = ng * NT2;
-    st.where = W_NONE;
-    st.n_items = n_items_for(nb, mgb);
-    st.n_groups = ng;
-    *w.status = st;
-    Sync z;
-    z.q1 = z.q2 = z.qc = z.rq_alloc = z.rq_head = z.prod_done = 0;
-    z.pad[0] = z.pad[1] = 0;
-    *w.sync = z;
-  }
-  const int nbands_s = nb;
-  if (w.bands == nullptr) return;   // permutation only: no tile plan wanted
-  for (int s = tid; s < E; s += blockDim.x) {
-    w.sorted_e[s] = sorted[s];
-    if (w.expert_rank) w.expert_rank[sorted[s]] = s;
-  }
-  __syncthreads();
-  for (int s = tid; s < E; s += blockDim.x) {
-    const int e = sorted[s];
-    const int b0 = bstart[s], nbe = bstart[s + 1] - b0;
-    for (int i = 0; i < nbe; ++i) {
-      Band bd;
-      bd.expert = e;
-      bd.row0 = offs[e] + i * BM;
-      bd.rows = min(BM, cnt[e] - i * BM);
-      bd.pad = 0;
-      w.bands[b0 + i] = bd;
-    }
-    const int g0 = gstart[s], nge = gstart[s + 1] - g0;
-    for (int i = 0; i < nge; ++i) {
-      Group gr;
-      gr.expert = e;
-      gr.band0 = b0 + i * G;
-      gr.row0 = offs[e] + i * G * BM;
-      gr.rows = min(G * BM, cnt[e] - i * G * BM);
-      w.groups[g0 + i] = gr;
-    }
-  }
-  for (int i = tid; i < nbands_s; i += blockDim.x) { w.band_done1[i] = 0u; w.band_done2[i] = 0u; }
-  if (w.tok_band) {
-    int4* tb = reinterpret_cast<int4*>(w.tok_band);
-    for (int i = tid; i < nbands_s * (BM / 4); i += blockDim.x) tb[i] = make_int4(0, 0, 0, 0);
-  }
+  // ids from the caller (nblk > 0 and no route kernel before us) that fell outside
+  // [0, E) were not counted: the total comes up short of T*k
+  const long long R = offs[E];
+  const uint32_t code = (bad_in || (nblk > 0 && R != (long long)T * k)) ? ST_INVALID : ST_OK;
+  plan_tables(w, E, cnt, offs, nullptr, nullptr, nullptr, sorted, code, R, T, d, f, num_sms,
+              consumer_hint, mgb, G, cg, join, cm);
 }
 
 cudaError_t launch_plan(const Work& w, int nblk, const int32_t* offsets_in, int T, int d, int f,
                         int E, int k, int num_sms, int consumer_hint, int mgb, int G, int cg,
                         int join, const CostModel& cm, cudaStream_t s) {
   return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, w, nblk, offsets_in, T, d, f, E, k, num_sms,
+                    consumer_hint, mgb, G, cg, join, cm);
+}
+
+// ------------------------------------------------------------ owner plan ---
+// The expert-parallel owner's plan ("Fine-grained Computation-Communication
+// Overlap via Tile-level Signaling and Scheduling for Mixture-of-Experts",
+// Section 3.2): the rows it received arrive source rank major, then local expert
+// ascending, each source's rows in its own (slot) order, so the rows of local
+// expert e from source s are one contiguous run -- a segment.  Planning units are
+// the W*El segments:
+//  * remote-owner-aligned layout (Section 3.2.1): a segment's rows all return to
+//    one rank, and bands never straddle two segments, so every band has a single
+//    destination (the paper pads each run to a band boundary with zero rows; here
+//    the last band of a run is masked instead, as every expert's last band is);
+//  * remote-first schedule (Section 3.2.2): every remote segment before any local
+//    one; remote segments by their expert's remote band count, descending (ties:
+//    lower expert), an expert's segments together in source order; then the local
+//    segments by expert;
+//  * combine plan (Section 3.2.3): per band, the home rank and the row in the
+//    home's return buffer (its dispatch order) where the band's first row goes.
+__global__ void __launch_bounds__(1024) plan_ep_kernel(Work w, const int32_t* __restrict__ recv_counts,
+                                                       EpPlanIn in, int d, int f, int num_sms,
+                                                       int consumer_hint, int mgb, int G, int cg,
+                                                       int join, CostModel cm) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int cnt[MAX_E];        // per segment u = e * W + s
+  __shared__ int row0[MAX_E];
+  __shared__ int unit_e[MAX_E];
+  __shared__ int dest[MAX_E];
+  __shared__ int home0[MAX_E];
+  __shared__ int sorted[MAX_E];
+  __shared__ int rbands[MAX_E];     // remote bands per local expert
+  __shared__ int bad;
+  const int tid = threadIdx.x;
+  const int W = in.W, El = in.El, U = W * El;
+  if (tid == 0) bad = 0;
+  __syncthreads();
+  for (int u = tid; u < U; u += blockDim.x) {
+    const int e = u / W, src = u - e * W;
+    const int c = recv_counts[src * El + e];
+    if (c < 0) bad = 1;
+    cnt[u] = c;
+    unit_e[u] = e;
+    dest[u] = src;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // segment starts in the received rows (source major, expert ascending) and in
+    // the home's return buffer (recv_base[s] + the source's rows of earlier experts)
+    long long run = 0;
+    for (int src = 0; src < W; ++src) {
+      int within = 0;
+      for (int e = 0; e < El; ++e) {
+        const int u = e * W + src;
+        row0[u] = (int)run + within;
+        home0[u] = in.recv_base[src] + within;
+        within += cnt[u];
+      }
+      run += within;
+    }
+    if (run != (long long)in.N) bad = 1;
+  }
+  __syncthreads();
+  if (bad)
+    for (int u = tid; u < U; u += blockDim.x) cnt[u] = 0;
+  for (int e = tid; e < El; e += blockDim.x) {
+    int rb = 0;
+    for (int src = 0; src < W; ++src)
+      if (src != in.rank) rb += cdiv(cnt[e * W + src], BM);
+    rbands[e] = rb;
+  }
+  __syncthreads();
+  // rank of each segment under (local?, remote bands desc, expert asc, source asc)
+  for (int u = tid; u < U; u += blockDim.x) {
+    const int e = u / W, src = u - e * W;
+    const bool loc = src == in.rank;
+    int r = 0;
+    for (int v = 0; v < U; ++v) {
+      const int e2 = v / W, s2 = v - e2 * W;
+      const bool loc2 = s2 == in.rank;
+      bool before;
+      if (loc2 != loc) before = !loc2;                          // remote segments first
+      else if (!loc && rbands[e2] != rbands[e]) before = rbands[e2] > rbands[e];
+      else if (e2 != e) before = e2 < e;
+      else before = s2 < src;
+      r += before;
+    }
+    sorted[r] = u;
+  }
+  __syncthreads();
+  plan_tables(w, U, cnt, row0, unit_e, dest, home0, sorted, bad ? ST_INVALID : ST_OK,
+              bad ? 0 : in.N, bad ? 1 : in.N, d, f, num_sms, consumer_hint, mgb, G, cg, join, cm);
+}
+
+cudaError_t launch_plan_ep(const Work& w, const int32_t* recv_counts, const EpPlanIn& in, int d,
+                           int f, int num_sms, int consumer_hint, int mgb, int G, int cg, int join,
+                           const CostModel& cm, cudaStream_t s) {
+  return launch_pdl(plan_ep_kernel, dim3(1), dim3(1024), 0, s, w, recv_counts, in, d, f, num_sms,
                     consumer_hint, mgb, G, cg, join, cm);
 }
 

@@ -114,3 +114,54 @@ def return_rows(rows_owner_order: torch.Tensor, order: torch.Tensor, ex: Exchang
     received = torch.empty_like(rows_owner_order)
     received[order.to(rows_owner_order.device)] = rows_owner_order   # back to received order
     return _exchange(received, sum(ex.send_rows), ex.send_rows, ex.recv_rows, group)
+
+
+def virtual_ranks_forward(xs, logits, W1, W3, W2, k: int, mode: int = 1, consumer_sms: int = 0,
+                          mgb: int = 1, flags: int = 0, timeout_us: int = 0):
+    """One expert-parallel MoE layer over W virtual ranks on the current GPU, with
+    the fused return (Sections 3.2-3.3 of the paper).  xs[r], logits[r]: rank r's
+    tokens and gate logits; W1, W3, W2: all E experts (rank o owns
+    [o*E/W, (o+1)*E/W)).  Per rank: route and permute (the library); the dispatch
+    all-to-all -- on several GPUs dispatch() above, over NCCL -- is stood in for by
+    device copies of each home's row runs (with their home slots) into each
+    owner's receive buffer; each owner runs moe_ep_owner_forward, whose consumer
+    CTAs store every finished band into its home's return buffer and bump the
+    home's arrival words; each home runs moe_ep_home_combine.  Returns (outs,
+    state) with outs[r] rank r's layer output.  Owners run one after another, so
+    no kernel here waits on a kernel that has not already finished."""
+    from . import moe
+    Wn = len(xs)
+    E, d, f = W1.shape
+    El = local_experts(E, Wn)
+    dev = xs[0].device
+    homes = []
+    for r in range(Wn):
+        T = xs[r].shape[0]
+        ws = moe.alloc_workspace(T, d, f, E, k, dev)
+        idx, gate = moe.route(logits[r], k, ws)
+        counts, offsets, perm, row_of, x_perm = moe.permute(xs[r], idx, E, ws)
+        homes.append(dict(T=T, ws=ws, idx=idx, gate=gate, counts=counts, offsets=offsets, perm=perm,
+                          row_of=row_of, x_perm=x_perm,
+                          y=torch.empty((T * k, d), dtype=torch.bfloat16, device=dev),
+                          arrive=torch.zeros(T, dtype=torch.int32, device=dev)))
+    offs = [h["offsets"].cpu() for h in homes]     # the exchange sizes, on the host
+    owners = []
+    for o in range(Wn):
+        lo, hi = o * El, (o + 1) * El
+        runs = [(int(offs[s][lo]), int(offs[s][hi])) for s in range(Wn)]
+        x_recv = torch.cat([homes[s]["x_perm"][a:b] for s, (a, b) in enumerate(runs)])
+        slot_recv = torch.cat([homes[s]["perm"][a:b] for s, (a, b) in enumerate(runs)])
+        recv_counts = torch.stack([homes[s]["counts"][lo:hi] for s in range(Wn)]).contiguous()
+        N = x_recv.shape[0]
+        ws_o = torch.empty(moe.ep_owner_workspace_size(N, d, f, El, Wn), dtype=torch.uint8, device=dev)
+        moe.ep_owner_forward(x_recv, slot_recv, recv_counts, W1[lo:hi], W3[lo:hi], W2[lo:hi], k, o,
+                             [a for a, _ in runs], [h["y"] for h in homes], [h["arrive"] for h in homes],
+                             ws_o, mode, consumer_sms=consumer_sms, mgb=mgb, flags=flags,
+                             timeout_us=timeout_us)
+        owners.append(dict(ws=ws_o, N=N, x_recv=x_recv, slot_recv=slot_recv, recv_counts=recv_counts))
+    outs, statuses = [], []
+    for h in homes:
+        out, st = moe.ep_home_combine(h["y"], h["arrive"], h["row_of"], h["gate"], timeout_us=timeout_us)
+        outs.append(out)
+        statuses.append(st)
+    return outs, dict(homes=homes, owners=owners, status=statuses)

@@ -35,6 +35,8 @@ SCHED_B_PER_ATOM = 0x40
 SCHED_FULL_TILES = 0x80
 SCHED_WIDE_CTA = 0x100
 DBG_IDENTITY_EXPERTS = 0x200
+SCHED_INTERLEAVE = 0x400
+SCHED_EVICT_FIRST = 0x800
 
 
 class MoEError(RuntimeError):
@@ -58,6 +60,23 @@ class LayerArgs(ctypes.Structure):
         ("consumer_sms", ctypes.c_int), ("mgb", ctypes.c_int), ("flags", ctypes.c_uint),
         ("timeout_us", ctypes.c_int),
         ("ev_ffn_begin", ctypes.c_void_p), ("ev_ffn_end", ctypes.c_void_p),
+    ]
+
+
+MAX_EP_RANKS = 8
+
+
+class EpOwnerArgs(ctypes.Structure):
+    _fields_ = [
+        ("W", ctypes.c_int), ("rank", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int),
+        ("f", ctypes.c_int), ("El", ctypes.c_int), ("k", ctypes.c_int),
+        ("x_recv", ctypes.c_void_p), ("slot_recv", ctypes.c_void_p), ("recv_counts", ctypes.c_void_p),
+        ("W1", ctypes.c_void_p), ("W3", ctypes.c_void_p), ("W2", ctypes.c_void_p),
+        ("recv_base", ctypes.c_int * MAX_EP_RANKS),
+        ("home_y", ctypes.c_void_p * MAX_EP_RANKS),
+        ("home_arrive", ctypes.c_void_p * MAX_EP_RANKS),
+        ("consumer_sms", ctypes.c_int), ("mgb", ctypes.c_int), ("flags", ctypes.c_uint),
+        ("timeout_us", ctypes.c_int),
     ]
 
 
@@ -86,8 +105,14 @@ _lib.moe_debug_band_stamps.restype = _I
 _lib.moe_permute_noalloc.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
 _lib.moe_permute_noalloc.restype = _I
 _lib.moe_permute_noalloc_scratch_bytes.restype = _S
+_lib.moe_ep_owner_workspace_size.argtypes = [_I, _I, _I, _I, _I]
+_lib.moe_ep_owner_workspace_size.restype = _S
+_lib.moe_ep_owner_forward.argtypes = [ctypes.POINTER(EpOwnerArgs), _I, _P, _S, _P]
+_lib.moe_ep_home_combine.argtypes = [_P, _P, _P, _P, _I, _I, _I, _P, _P, _I, _P]
+_lib.moe_ep_debug_plan.argtypes = [_P, _I, _I, _I, _I, _I, _P, _P, _I]
+_lib.moe_ep_debug_plan.restype = _I
 for _fn in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_combine", "moe_layer_forward",
-            "moe_get_status"):
+            "moe_get_status", "moe_ep_owner_forward", "moe_ep_home_combine"):
     getattr(_lib, _fn).restype = _I
 
 
@@ -367,3 +392,82 @@ class MoELayer:
         if x.shape[0] > self.max_tokens:
             raise ValueError("more tokens than the workspace was sized for")
         return layer_forward(x, logits, self.W1, self.W3, self.W2, self.k, self.ws, mode, **kw)
+
+
+# ---- expert parallelism: the fused return -----------------------------------
+def ep_owner_workspace_size(N: int, d: int, f: int, El: int, W: int) -> int:
+    return int(_lib.moe_ep_owner_workspace_size(N, d, f, El, W))
+
+
+def ep_owner_forward(x_recv, slot_recv, recv_counts, W1, W3, W2, k: int, rank: int, recv_base,
+                     home_y, home_arrive, ws, mode=MODE_OVERLAPPED, consumer_sms=0, mgb=1,
+                     flags=0, timeout_us=0, stream=None):
+    """The owner side of an expert-parallel layer (moe_ep_owner_forward): runs
+    this rank's experts on the rows it received and returns every finished row
+    band into its home rank's buffer (home_y[s], home_arrive[s], one per rank)."""
+    _need(x_recv, torch.bfloat16, "x_recv")
+    _need(slot_recv, torch.int32, "slot_recv")
+    _need(recv_counts, torch.int32, "recv_counts")
+    N, d = x_recv.shape
+    El, _, f = _weights(W1, W3, W2, d)
+    W = recv_counts.shape[0]
+    _shape(recv_counts, (W, El), "recv_counts")
+    _shape(slot_recv, (N,), "slot_recv")
+    if not (1 <= W <= MAX_EP_RANKS) or len(home_y) != W or len(home_arrive) != W or len(recv_base) != W:
+        raise ValueError("one home buffer, arrival array and receive base per rank")
+    for s_, (y, a) in enumerate(zip(home_y, home_arrive)):
+        _need(y, torch.bfloat16, f"home_y[{s_}]")
+        _need(a, torch.int32, f"home_arrive[{s_}]")
+        if y.shape[1] != d:
+            raise ValueError(f"home_y[{s_}] rows must have d = {d}")
+    if ws.numel() < ep_owner_workspace_size(N, d, f, El, W):
+        raise ValueError("workspace smaller than moe_ep_owner_workspace_size")
+    if N == 0:
+        return   # nothing received: no band to compute or return
+    a = EpOwnerArgs()
+    a.W, a.rank, a.N, a.d, a.f, a.El, a.k = W, rank, N, d, f, El, k
+    a.x_recv, a.slot_recv, a.recv_counts = x_recv.data_ptr(), slot_recv.data_ptr(), recv_counts.data_ptr()
+    a.W1, a.W3, a.W2 = W1.data_ptr(), W3.data_ptr(), W2.data_ptr()
+    for s_ in range(W):
+        a.recv_base[s_] = int(recv_base[s_])
+        a.home_y[s_] = home_y[s_].data_ptr()
+        a.home_arrive[s_] = home_arrive[s_].data_ptr()
+    a.consumer_sms, a.mgb, a.flags, a.timeout_us = consumer_sms, mgb, flags, timeout_us
+    _check(_lib.moe_ep_owner_forward(ctypes.byref(a), int(mode), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_ep_owner_forward")
+
+
+def ep_home_combine(home_y, arrive, row_of, topk_gate, out=None, status=None, timeout_us=0,
+                    stream=None):
+    """The home side (moe_ep_home_combine): waits for each token's k returned
+    rows, combines them and zeroes the arrival words.  Returns (out, status) with
+    status a one-element int32 device tensor (0, or MOE_ERR_TIMEOUT)."""
+    _need(home_y, torch.bfloat16, "home_y")
+    _need(arrive, torch.int32, "arrive")
+    _need(row_of, torch.int32, "row_of")
+    _need(topk_gate, torch.float32, "topk_gate")
+    T, k = topk_gate.shape
+    d = home_y.shape[1]
+    _shape(home_y, (T * k, d), "home_y")
+    _shape(arrive, (T,), "arrive")
+    _shape(row_of, (T * k,), "row_of")
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=home_y.device)
+    _shape(out, (T, d), "out")
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=home_y.device)
+    _check(_lib.moe_ep_home_combine(_ptr(home_y), _ptr(arrive), _ptr(row_of), _ptr(topk_gate), T, d, k,
+                                    _ptr(out), _ptr(status), int(timeout_us), _stream(stream)),
+           "moe_ep_home_combine")
+    return out, status
+
+
+def ep_band_dest(ws, N: int, d: int, f: int, El: int, W: int, n_bands: int, stream=None):
+    """The combine plan of the last owner call on ws: [n_bands][2] int32 (home
+    rank, home row of the band's first row), bands in schedule order."""
+    import numpy as np
+    out = np.zeros((max(1, n_bands), 2), dtype=np.int32)
+    _check(_lib.moe_ep_debug_plan(_ptr(ws), N, d, f, El, W, _stream(stream),
+                                  out.ctypes.data_as(ctypes.c_void_p), max(1, n_bands)),
+           "moe_ep_debug_plan")
+    return out[:n_bands]

@@ -97,6 +97,17 @@ typedef enum {
                                         in either mode, so out[t] = bf16(sum_j g_j x[t])
                                         checks those steps apart from the GEMMs; W1, W3
                                         and W2 are not read and may be NULL */
+#define MOE_SCHED_INTERLEAVE   0x400u /* GEMM2 tiles interleave with GEMM1 tiles: a
+                                        scheduler takes the next GEMM2 tile (in priority
+                                        order) as soon as every GEMM1 tile of its row group
+                                        is stored, and GEMM1 tiles otherwise, so row bands
+                                        complete throughout the launch; dedicated consumer
+                                        CTAs then skip GEMM1.  Default: every CTA takes
+                                        GEMM1 tiles until that queue is empty before any
+                                        GEMM2 tile.  Same bits */
+#define MOE_SCHED_EVICT_FIRST  0x800u /* the epilogue stores h and y with an L2
+                                        evict-first policy (they compete with the weights
+                                        for L2).  Same bits */
 #define MOE_SCHED_WIDE_CTA     0x100u /* force 256-row MMA tiles on single CTAs: two
                                         128-row MMAs per K step share one B stage and
                                         fill the CTA's two accumulators (an expert's odd
@@ -170,9 +181,10 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
  * (fp32 accumulation).  x_perm [R][d], y [R][d] bf16, R = offsets[E] <= T*k;
  * h [R][f] bf16 is written to the caller's buffer if non-NULL, else kept in the
  * workspace.  offsets must start at 0, never decrease and end at most at T*k;
- * otherwise nothing is computed and moe_get_status returns MOE_ERR_INVALID.  flags: 0, or MOE_SCHED_ONE_CTA / MOE_SCHED_CTA_PAIR /
- * MOE_SCHED_B_PER_ATOM / MOE_SCHED_FULL_TILES (tile variant); any other bit is
- * MOE_ERR_INVALID. */
+ * otherwise nothing is computed and moe_get_status returns MOE_ERR_INVALID.
+ * flags: 0, or MOE_SCHED_ONE_CTA / MOE_SCHED_CTA_PAIR / MOE_SCHED_WIDE_CTA /
+ * MOE_SCHED_B_PER_ATOM / MOE_SCHED_FULL_TILES (tile variant), MOE_SCHED_INTERLEAVE,
+ * MOE_SCHED_EVICT_FIRST; any other bit is MOE_ERR_INVALID. */
 moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, int d, int f,
                            int E, int k, const void* W1, const void* W3, const void* W2,
                            void* h, void* y, unsigned flags, void* ws, size_t ws_bytes,
@@ -217,6 +229,85 @@ size_t moe_permute_noalloc_scratch_bytes(void);
 /* The whole layer, steps (a)-(e).  Both modes give bit-identical outputs. */
 moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode,
                              void* ws, size_t ws_bytes, void* stream);
+
+/* ---- Expert parallelism: the fused return ---------------------------------
+ * W ranks; rank o owns the local experts [o*El, (o+1)*El) of E = W*El.  Each
+ * home rank routes and permutes its own tokens (moe_route, moe_permute); its
+ * routed rows, grouped by expert and so by owner, are dispatched to the owners
+ * (an all-to-all outside this library, e.g. NCCL) together with each row's home
+ * slot p = t*k + j.  The owner runs moe_ep_owner_forward: the paper's rank-wide
+ * persistent expert GEMM (Section 3.3.1) whose consumer partition returns every
+ * finished row band straight into its home rank's return buffer (the return
+ * all-to-all, fused: Sections 3.2.1-3.2.3 and 3.3.2-3.3.3).  Each home then runs
+ * moe_ep_home_combine.  The result is bit-identical to moe_layer_forward on the
+ * home's tokens with every expert local.
+ *
+ * The owner only STORES into home buffers (16-byte stores and system-scope
+ * release adds; no loads from them, no TMA), so home_y / home_arrive may be
+ * another GPU's memory mapped into this one (CUDA IPC, symmetric memory); on one
+ * GPU they are plain device pointers of W virtual ranks. */
+#define MOE_MAX_EP_RANKS 8
+
+typedef struct {
+  int W;                     /* ranks, 1..MOE_MAX_EP_RANKS                           */
+  int rank;                  /* this owner's rank o                                  */
+  int N;                     /* rows received                                        */
+  int d, f, El, k;           /* d_model, d_ff, local experts (W*El <= 256), top-k    */
+  const void* x_recv;        /* [N][d] bf16: source rank major, then local expert
+                                ascending, each source's rows in its own order       */
+  const int32_t* slot_recv;  /* [N] home slot p = t*k + j of each received row       */
+  const int32_t* recv_counts;/* [W][El] device: rows from source s for local expert e */
+  const void* W1;            /* [El][d][f] bf16, this owner's experts                */
+  const void* W3;            /* [El][d][f] bf16                                      */
+  const void* W2;            /* [El][f][d] bf16                                      */
+  int recv_base[MOE_MAX_EP_RANKS];  /* per source s: row, in s's return buffer (its
+                                       dispatch order), of the first row s sent here */
+  void* home_y[MOE_MAX_EP_RANKS];   /* per rank: return buffer [T_s*k][d] bf16, in the
+                                       home's permutation order (rows of x_perm)     */
+  uint32_t* home_arrive[MOE_MAX_EP_RANKS]; /* per rank: arrival words [T_s], zero
+                                       before the first call                         */
+  int consumer_sms;          /* 0 = cost model; > 0 = this many return CTAs          */
+  int mgb;                   /* row bands per middle return segment (paper's x); 0 = 1 */
+  unsigned flags;            /* MOE_SCHED_* bits (tile variant, NO_JOIN, INTERLEAVE,
+                                EVICT_FIRST); MOE_DBG_TIMESTAMPS                      */
+  int timeout_us;            /* bound on each device wait; 0 = 2 s                   */
+} moe_ep_owner_args;
+
+/* Workspace bytes moe_ep_owner_forward needs (0 on an invalid shape). */
+size_t moe_ep_owner_workspace_size(int N, int d, int f, int El, int W);
+
+/* The owner side of one expert-parallel MoE layer.  Plan (on the device, from
+ * recv_counts): the (local expert, source) segments of the received rows are the
+ * planning units -- every row band has one destination; remote segments are
+ * scheduled first, experts with more remote bands first (Section 3.2.2); the
+ * combine plan gives each band its home rank and home row (Section 3.2.3).
+ * OVERLAPPED: one persistent launch; consumer CTAs (consumer_sms, or the cost
+ * model; producers join once the tile queue drains) wait for each segment's
+ * bands, copy them into home_y[s] at the planned row and add 1 per row to
+ * home_arrive[s][p / k].  SEQUENTIAL: GEMM1, GEMM2, then the whole return as a
+ * separate pass (the baseline).  Both modes store the same bytes.
+ * Errors: argument errors at once; a device wait that runs out is reported by
+ * moe_get_status(ws, ...); recv_counts that do not sum to N give MOE_ERR_INVALID
+ * there (nothing is computed). */
+moe_status moe_ep_owner_forward(const moe_ep_owner_args* args, moe_mode mode, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/* The home side: for every token t, waits (bounded by timeout_us; 0 = 2 s) until
+ * arrive[t] == k, then out[t] = bf16( sum_j g[t][j] * home_y[row_of[t*k+j]] ) in
+ * fp32, slot order (moe_combine's arithmetic), and zeroes arrive[t] for the next
+ * call.  status: a device word, 0 on entry; a wait that runs out sets it to
+ * MOE_ERR_TIMEOUT and ends the other waits (that token's out row is not
+ * written).  home_y [T*k][d] bf16, arrive [T], row_of [T*k], topk_gate [T][k]. */
+moe_status moe_ep_home_combine(const void* home_y, uint32_t* arrive, const int32_t* row_of,
+                               const float* topk_gate, int T, int d, int k, void* out,
+                               uint32_t* status, int timeout_us, void* stream);
+
+/* Debug aid: synchronises `stream` and copies the combine plan of the last
+ * moe_ep_owner_forward on `ws` (same N, d, f, El, W) into host_out: per row band
+ * in schedule order, (home rank, home row of the band's first row) -- 2 int32
+ * each; host_out holds max_bands pairs. */
+moe_status moe_ep_debug_plan(void* ws, int N, int d, int f, int El, int W, void* stream,
+                             int32_t* host_out, int max_bands);
 
 /* Synchronises `stream`, then reads the status block the last call left in `ws`.
  * Returns MOE_OK or the device-side error (MOE_ERR_TIMEOUT).  Host outputs may be

@@ -101,3 +101,51 @@ def test_tile_variant_rule():
     assert tv(4096, 14336, 8, 2, moe.SCHED_NO_JOIN | moe.SCHED_B_PER_ATOM) == 3
     assert tv(0, 14336, 8, 2) == 0
     assert set(moe.TILE_VARIANTS) == {1, 2, 3}
+
+
+def test_ep_owner_host_side_argument_errors():
+    # moe_ep_owner_forward refuses bad shapes and pointers before any CUDA call
+    ws = moe.ep_owner_workspace_size
+    assert ws(1000, 512, 256, 4, 2) > 0
+    assert ws(0, 512, 256, 4, 2) > 0            # an owner may receive nothing
+    assert ws(1000, 500, 256, 4, 2) == 0        # d not a multiple of 256
+    assert ws(1000, 512, 256, 4, 9) == 0        # more ranks than MOE_MAX_EP_RANKS
+    assert ws(1000, 512, 256, 64, 8) == 0       # W * El > 256 planning units
+    assert ws(-1, 512, 256, 4, 2) == 0
+
+    def args(**kw):
+        a = moe.EpOwnerArgs()
+        a.W, a.rank, a.N, a.d, a.f, a.El, a.k = 2, 0, 100, 512, 256, 4, 2
+        a.x_recv, a.slot_recv, a.recv_counts = 0x1000, 0x2000, 0x3000
+        a.W1, a.W3, a.W2 = 0x4000, 0x5000, 0x6000
+        for r in range(2):
+            a.home_y[r] = 0x10000 * (r + 1)
+            a.home_arrive[r] = 0x20000 * (r + 1)
+        for k_, v in kw.items():
+            setattr(a, k_, v)
+        return a
+
+    def call(a, mode=1, wsb=1 << 40):
+        return moe._lib.moe_ep_owner_forward(ctypes.byref(a), mode, ctypes.c_void_p(0x100000), wsb, None)
+
+    assert call(args(W=0)) == moe.MOE_ERR_INVALID
+    assert call(args(rank=2)) == moe.MOE_ERR_INVALID
+    assert call(args(W=9)) == moe.MOE_ERR_UNSUPPORTED
+    assert call(args(El=200)) == moe.MOE_ERR_UNSUPPORTED      # 400 planning units
+    assert call(args(d=320)) == moe.MOE_ERR_UNSUPPORTED
+    assert call(args(x_recv=0)) == moe.MOE_ERR_INVALID
+    assert call(args(x_recv=0x1008)) == moe.MOE_ERR_INVALID   # misaligned
+    assert call(args(), mode=5) == moe.MOE_ERR_INVALID
+    a = args()
+    a.home_y[1] = 0
+    assert call(a) == moe.MOE_ERR_INVALID
+    assert call(args(), wsb=1024) == moe.MOE_ERR_WORKSPACE
+    assert moe._lib.moe_ep_owner_forward(None, 1, None, 0, None) == moe.MOE_ERR_INVALID
+    P = ctypes.c_void_p
+    hc = moe._lib.moe_ep_home_combine
+    assert hc(P(0x1000), P(0x2000), P(0x3000), P(0x4000), 0, 512, 2, P(0x5000), P(0x6000), 0,
+              None) == moe.MOE_ERR_INVALID
+    assert hc(P(0x1000), P(0x2000), P(0x3000), P(0x4000), 16, 512, 9, P(0x5000), P(0x6000), 0,
+              None) == moe.MOE_ERR_UNSUPPORTED
+    assert hc(P(0x1000), P(0x2000), P(0x3000), P(0x4000), 16, 512, 2, P(0x5000), None, 0,
+              None) == moe.MOE_ERR_INVALID

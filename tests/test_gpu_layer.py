@@ -108,8 +108,12 @@ def test_layer_small(orc, wl):
     # and single CTAs loading the weight tiles one 64-column atom per copy (3-D
     # maps) instead of one 4-D copy per operand: the same bytes in the same places
     # and CTA pairs running an expert's odd last band as a full 256-row tile
+    # and the schedule and store-policy variants: GEMM2 tiles interleaved with
+    # GEMM1 tiles (instead of all GEMM1 tiles first), evict-first h/y stores
     for fl in (moe.SCHED_GATHER_A | pair, moe.SCHED_GATHER_A | one, moe.SCHED_B_PER_ATOM | one,
-               moe.SCHED_FULL_TILES | pair):
+               moe.SCHED_FULL_TILES | pair, moe.SCHED_INTERLEAVE | one, moe.SCHED_INTERLEAVE | pair,
+               moe.SCHED_INTERLEAVE | wide, moe.SCHED_EVICT_FIRST | wide,
+               moe.SCHED_EVICT_FIRST | moe.SCHED_INTERLEAVE | one):
         gat, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=fl)
         base = seq_bits if fl & pair else gu.host(seq1)
         assert np.array_equal(gu.host(gat), base), f"flags {fl:#x} differ"

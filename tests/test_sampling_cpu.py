@@ -48,3 +48,12 @@ def test_combine_bound_is_one_bf16_ulp():
         pass
     else:
         raise AssertionError("two ulps accepted")
+
+
+def test_sweep_cell_spec():
+    import sys
+    sys.argv = ["bench.py"]
+    import bench
+    cells = bench._sweep_cells("seq,0,2/2,0+0x400,seq+0x800")
+    assert cells == [("seq", None, 0, 1, 0), ("0", "ovl", 0, 1, 0), ("2/2", "ovl", 2, 2, 0),
+                     ("0+0x400", "ovl", 0, 1, 0x400), ("seq+0x800", None, 0, 1, 0x800)]
