@@ -31,7 +31,7 @@ struct Layout {
   size_t status, sync, stamps, blk_hist, blk_base, counts, offsets, topk_idx, topk_gate, perm, row_of, arrive, ready_q;
   size_t routing_end;
   size_t sorted_e, band_start, tile_start1, bands, band_done1, band_done2, groups, group_start,
-      tok_band, expert_rank, band_dest;
+      tok_band, expert_rank, band_dest, g2_start;
   size_t plan_end;
   size_t x_perm, h, y;
   size_t total;
@@ -67,6 +67,7 @@ Layout layout(int T, int d, int f, int E, int k) {
   L.group_start = o; o = up(o + (size_t)(E + 1) * 4);
   L.tok_band = o; o = up(o + mb * BM * 4);
   L.expert_rank = o; o = up(o + (size_t)E * 4);
+  L.g2_start = o; o = up(o + (size_t)(E + 1) * 4);
   L.band_dest = o; o = up(o + mb * sizeof(int2));
   L.plan_end = o;
   L.x_perm = o; o = up(o + R * d * 2);
@@ -109,6 +110,7 @@ Work work_from(void* ws, const Layout& L, bool plan, bool acts) {
     w.group_start = at<int32_t>(ws, L.group_start);
     w.tok_band = at<int32_t>(ws, L.tok_band);
     w.expert_rank = at<int32_t>(ws, L.expert_rank);
+    w.g2_start = at<int32_t>(ws, L.g2_start);
     // the combine plan exists only for an expert-parallel owner (set by its entry)
   }
   if (acts) {

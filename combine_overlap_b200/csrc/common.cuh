@@ -57,12 +57,17 @@ struct Status {
 };
 
 struct Sync {          // zeroed by the plan kernel on every call
-  uint32_t q1, q2, qc;  // GEMM1 tiles, GEMM2 tiles, consumer band items taken
+  uint32_t q1, q2;      // GEMM1 tiles, GEMM2 tiles taken (MOE_SCHED_INTERLEAVE: q1 counts
+                        // the one interleaved queue)
+  uint32_t pad0[30];    // the producer queues get a 128-byte line of their own, apart from
+                        // the consumers' counters
+  uint32_t qc;          // consumer band items taken
   uint32_t rq_alloc;    // ready-token queue: entries allocated
   uint32_t rq_head;     // ready-token queue: entries claimed for combining
   uint32_t prod_done;   // CTAs that have left the producer role
-  uint32_t pad[2];
+  uint32_t pad1[28];
 };
+static_assert(sizeof(Sync) == 256, "two 128-byte lines");
 
 struct Band {          // one row band: up to BM rows of one expert
   int32_t expert, row0, rows, pad;
@@ -104,6 +109,8 @@ struct Work {
   int32_t* tile_start1; // [E+1] first GEMM1 tile of the s-th sorted expert
   Group* groups;        // [max_bands] producer row groups in priority order
   int32_t* group_start; // [E+1] first group of the s-th sorted expert
+  int32_t* g2_start;    // [E+1] MOE_SCHED_INTERLEAVE: position in the interleaved queue of
+                        // the s-th unit's first GEMM2 tile ([E]: the queue's length)
   uint32_t* band_done1; // [max_bands] GEMM1 tiles finished per band
   uint32_t* band_done2; // [max_bands] GEMM2 tiles finished per band
   uint32_t* arrive;     // [T] rows of token t that have arrived; TOKEN_DONE set once out[t]

@@ -195,6 +195,25 @@ __device__ Item decode_g2(const Work& w, int t, int NT2) {
   return make_item(K_G2, group, t % NT2, w.groups[group]);
 }
 
+// Position t of the interleaved queue (MOE_SCHED_INTERLEAVE): unit s's GEMM2 block
+// occupies [g2_start[s], g2_start[s] + its GEMM2 tiles); every other position is
+// the next GEMM1 tile.  Blocks do not overlap and their starts never decrease.
+__device__ Item decode_mixed(const Work& w, int t, int U, int NT2) {
+  int lo = -1, hi = U;   // the last block with g2_start <= t is lo (-1: none)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (w.g2_start[mid] <= t) lo = mid; else hi = mid;
+  }
+  int g2_before = 0;     // GEMM2 tiles at positions before t
+  if (lo >= 0) {
+    const int n2b = (w.group_start[lo + 1] - w.group_start[lo]) * NT2;
+    const int off = t - w.g2_start[lo];
+    if (off < n2b) return decode_g2(w, w.group_start[lo] * NT2 + off, NT2);
+    g2_before = w.group_start[lo + 1] * NT2;
+  }
+  return decode_g1(w, t - g2_before, U);
+}
+
 __device__ __forceinline__ void item_range(int item, int nb, int mgb, int& b0, int& b1) {
   if (mgb <= 1 || nb <= 2) { b0 = item; b1 = item + 1; return; }
   const int nmid = cdiv(nb - 2, mgb);
@@ -287,32 +306,26 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
   unsigned long long* my_stamps = w.stamps + (size_t)blockIdx.x * NSTAMP;
   unsigned long long n_g1 = 0, n_g2 = 0;
 
-  // With MOE_SCHED_INTERLEAVE, GEMM2 tiles interleave with GEMM1 tiles: while
-  // GEMM1 tiles remain, the scheduler takes the head GEMM2 tile if every GEMM1
-  // tile of its row group is already stored (a peek, then a compare-and-swap on
-  // the queue head), else the next GEMM1 tile.  A GEMM2 tile taken this way never
-  // waits; once the GEMM1 queue is empty, GEMM2 tiles are taken unconditionally,
-  // and each of them waits only on GEMM1 tiles that resident CTAs have dequeued.
-  const bool interleave = (a.flags & MOE_SCHED_INTERLEAVE) != 0;
-  auto group_stored = [&](int group) {
-    const Group gr = w.groups[group];
-    if (ld_acquire(&w.band_done1[gr.band0]) < BAND_UNIT * (uint32_t)NT1) return false;
-    return gr.rows <= BM || ld_acquire(&w.band_done1[gr.band0 + 1]) >= BAND_UNIT * (uint32_t)NT1;
-  };
+  // With MOE_SCHED_INTERLEAVE (and both GEMMs in this launch) one queue hands out
+  // GEMM1 and GEMM2 tiles interleaved, in the order the plan fixed (decode_mixed):
+  // a GEMM2 tile comes a grid's worth of GEMM1 tiles after the last GEMM1 tile of
+  // its unit, so every GEMM1 tile it waits on sits earlier in the queue and was
+  // taken by a resident CTA (no deadlock), and is most likely stored already.
+  const bool interleave = (a.flags & MOE_SCHED_INTERLEAVE) && g1 && g2;
   // Next work item: dequeued and published by a leader, read by a peer.
   auto next_item = [&](Item& it) -> bool {
     if (leader) {
       it.kind = K_END;
       if (*abort) g1 = g2 = false;
-      if (g1 && g2 && interleave) {
-        uint32_t t2 = *reinterpret_cast<volatile uint32_t*>(&w.sync->q2);
-        while (t2 < (uint32_t)n2 && group_stored((int)t2 / NT2)) {
-          const uint32_t seen = atomicCAS(&w.sync->q2, t2, t2 + 1u);
-          if (seen == t2) { it = decode_g2(w, (int)t2, NT2); break; }
-          t2 = seen;   // another CTA took it: look at the new head
+      if (interleave && g1) {
+        const int t = (int)atomicAdd(&w.sync->q1, 1u);
+        if (t < n1 + n2) it = decode_mixed(w, t, a.n_units, NT2);
+        else {
+          g1 = g2 = false;
+          if (stamp) my_stamps[1] = globaltimer();
         }
       }
-      if (it.kind == K_END && g1) {
+      if (!interleave && it.kind == K_END && g1) {
         const int t = (int)atomicAdd(&w.sync->q1, 1u);
         if (t < n1) it = decode_g1(w, t, a.n_units);
         else {
@@ -320,7 +333,7 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
           if (stamp) my_stamps[1] = globaltimer();
         }
       }
-      if (it.kind == K_END && g2) {
+      if (!interleave && it.kind == K_END && g2) {
         const int t = (int)atomicAdd(&w.sync->q2, 1u);
         if (t < n2) it = decode_g2(w, t, NT2); else g2 = false;
       }

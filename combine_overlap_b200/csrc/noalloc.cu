@@ -30,7 +30,7 @@ using namespace moe;
 
 constexpr int NOALLOC_MAX_T = 65536;
 constexpr int NOALLOC_MAX_BLK = (NOALLOC_MAX_T + ROUTE_TOK - 1) / ROUTE_TOK;   // 2048
-constexpr size_t HDR_BYTES = 256;   // Status + Sync, padded to 256 bytes
+constexpr size_t HDR_BYTES = 512;   // Status + Sync, padded to 512 bytes
 constexpr size_t CNT_BYTES = (size_t)MAX_E * sizeof(int32_t);   // counts when the caller passes none
 constexpr size_t HIST_BYTES = (size_t)NOALLOC_MAX_BLK * MAX_E * sizeof(int32_t);
 constexpr size_t PERMUTE_NOALLOC_SCRATCH_BYTES = HDR_BYTES + CNT_BYTES + 2 * HIST_BYTES;

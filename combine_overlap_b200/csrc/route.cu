@@ -234,6 +234,7 @@ __device__ void plan_tables(const Work& w, int U, const int* cnt, const int* row
                             const int* sorted, uint32_t code, long long R, int T, int d, int f,
                             int num_sms, int consumer_hint, int mgb, int G, int cg, int join,
                             const CostModel& cm) {
+  const int lag = num_sms;   // GEMM1 tiles between a unit's last one and its GEMM2 block
   __shared__ int bstart[MAX_E + 1];
   __shared__ int gstart[MAX_E + 1];
   __shared__ int t1start[MAX_E + 1];
@@ -262,6 +263,16 @@ __device__ void plan_tables(const Work& w, int U, const int* cnt, const int* row
       w.group_start[s2] = gstart[s2];
       w.tile_start1[s2] = t1start[s2];
     }
+    // The interleaved queue (MOE_SCHED_INTERLEAVE): GEMM1 tiles in their order, with
+    // unit s's block of GEMM2 tiles inserted once `lag` more GEMM1 tiles have been
+    // handed out after unit s's last one (so its GEMM1 tiles are likely stored by
+    // the time its GEMM2 tiles are taken).  Insertion points never decrease, so the
+    // blocks keep the priority order; g2_start[s] is block s's queue position.
+    if (w.g2_start) {
+      for (int s2 = tid; s2 < U; s2 += blockDim.x)
+        w.g2_start[s2] = min(t1start[s2 + 1] + lag, nt1) + gstart[s2] * NT2;
+      if (tid == 0) w.g2_start[U] = nt1 + ng * NT2;
+    }
   }
   if (tid == 0) {
     const int cmin = join ? 0 : cg;
@@ -278,10 +289,8 @@ __device__ void plan_tables(const Work& w, int U, const int* cnt, const int* row
     st.n_items = n_items_for(nb, mgb);
     st.n_groups = ng;
     *w.status = st;
-    Sync z;
-    z.q1 = z.q2 = z.qc = z.rq_alloc = z.rq_head = z.prod_done = 0;
-    z.pad[0] = z.pad[1] = 0;
-    *w.sync = z;
+    uint32_t* z = reinterpret_cast<uint32_t*>(w.sync);
+    for (int i = 0; i < (int)(sizeof(Sync) / 4); ++i) z[i] = 0u;
   }
   if (w.bands == nullptr) return;   // permutation only: no tile plan wanted
   for (int s = tid; s < U; s += blockDim.x) {
