@@ -160,7 +160,8 @@ int device_sms() {
   return n;
 }
 
-// Per-SM throughputs for the split cost model, from B200 measurements: a
+// Per-SM throughputs for the split cost model (the search starts at one dedicated
+// consumer CTA group; see choose_consumers), from B200 measurements: a
 // producer SM sustains about 1/148 of ~1.2 PFLOP/s of bf16 MMA inside this kernel
 // (power-capped), one consumer SM moves about 30 GB/s of combine traffic (bulk
 // reads of expert rows plus output stores), HBM ~6.5 TB/s.
@@ -293,7 +294,7 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
     return MOE_ERR_INVALID;
   constexpr unsigned tile_flags = MOE_SCHED_ONE_CTA | MOE_SCHED_CTA_PAIR | MOE_SCHED_WIDE_CTA |
                                   MOE_SCHED_B_PER_ATOM | MOE_SCHED_FULL_TILES |
-                                  MOE_SCHED_INTERLEAVE | MOE_SCHED_EVICT_FIRST;
+                                  MOE_SCHED_INTERLEAVE | MOE_SCHED_EVICT_FIRST | MOE_SCHED_PREFETCH;
   if (flags & ~tile_flags) return MOE_ERR_INVALID;
   const Layout L = layout(T, d, f, E, k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;

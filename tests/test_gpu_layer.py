@@ -82,7 +82,7 @@ def test_layer_small(orc, wl):
                dict(consumer_sms=8), dict(consumer_sms=32), dict(mgb=2), dict(mgb=3, consumer_sms=3),
                dict(flags=moe.SCHED_NO_JOIN, consumer_sms=2)):
         ovl, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=pair | kw.pop("flags", 0), **kw)
-        assert c >= 0 and c % 2 == 0      # whole CTA pairs (0: producers join at the end)
+        assert c >= 2 and c % 2 == 0      # whole CTA pairs, at least one
         assert np.array_equal(gu.host(ovl), seq_bits), f"overlapped {kw} differs from sequential"
     # the single-CTA (128-row tile) variant: same checks
     one = moe.SCHED_ONE_CTA
@@ -108,12 +108,14 @@ def test_layer_small(orc, wl):
     # and single CTAs loading the weight tiles one 64-column atom per copy (3-D
     # maps) instead of one 4-D copy per operand: the same bytes in the same places
     # and CTA pairs running an expert's odd last band as a full 256-row tile
-    # and the schedule and store-policy variants: GEMM2 tiles interleaved with
-    # GEMM1 tiles (instead of all GEMM1 tiles first), evict-first h/y stores
+    # and the schedule and memory-policy variants: GEMM2 tiles interleaved with
+    # GEMM1 tiles (instead of all GEMM1 tiles first), evict-first h/y stores, L2
+    # prefetch of the weight tiles
     for fl in (moe.SCHED_GATHER_A | pair, moe.SCHED_GATHER_A | one, moe.SCHED_B_PER_ATOM | one,
                moe.SCHED_FULL_TILES | pair, moe.SCHED_INTERLEAVE | one, moe.SCHED_INTERLEAVE | pair,
                moe.SCHED_INTERLEAVE | wide, moe.SCHED_EVICT_FIRST | wide,
-               moe.SCHED_EVICT_FIRST | moe.SCHED_INTERLEAVE | one):
+               moe.SCHED_EVICT_FIRST | moe.SCHED_INTERLEAVE | one, moe.SCHED_PREFETCH | wide,
+               moe.SCHED_PREFETCH | one, moe.SCHED_PREFETCH | moe.SCHED_INTERLEAVE | wide):
         gat, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=fl)
         base = seq_bits if fl & pair else gu.host(seq1)
         assert np.array_equal(gu.host(gat), base), f"flags {fl:#x} differ"
