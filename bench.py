@@ -21,6 +21,7 @@ the CPU oracle on each configuration; each prints one JSON line per case.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -92,6 +93,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cool-down", type=float, default=0.5,
+                    help="seconds the GPU idles before each timed region (same starting power state)")
     ap.add_argument("--sweep", action="store_true",
                     help="d=4096/E=32/top-4 sweep: T x router x consumer SMs, overlapped vs "
                          "sequential; one JSON line per cell (not the benchmark line)")
@@ -108,10 +111,11 @@ def parse():
 # ----------------------------------------------------------------- clocks ---
 class Clocks:
     """nvidia-smi samples of the SM clock, power and throttle reasons, every 50 ms,
-    from before the warm-up to the end of the GPU work; each sample is stamped with
-    the host's monotonic clock so that a timed region can take the samples that fall
-    inside it."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    from before the warm-up to the end of the GPU work.  Each sample carries
+    nvidia-smi's own wall-clock timestamp (its output reaches this process in
+    bursts, so the time of arrival is not the time of the sample), and a timed
+    region takes the samples whose timestamps fall inside its wall-clock window."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
@@ -119,7 +123,7 @@ class Clocks:
     def __init__(self, device: int, enabled: bool = True, period_ms: int = 50):
         import threading
         self.proc = None
-        self.samples = []          # (t_monotonic, sm_mhz, max_mhz, power_w, reasons)
+        self.samples = []          # (t_wall, sm_mhz, max_mhz, power_w, reasons)
         self.windows = {}
         if not enabled:
             return
@@ -145,6 +149,7 @@ class Clocks:
                 continue
             try:
                 sm, smax = float(parts[1]), float(parts[2])
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
             except ValueError:
                 continue
             try:
@@ -152,10 +157,10 @@ class Clocks:
             except ValueError:
                 pw = None
             reasons = {n for n, v in zip(self.REASONS, parts[5:9]) if v.lower().startswith("active")}
-            self.samples.append((time.monotonic(), sm, smax, pw, reasons))
+            self.samples.append((ts, sm, smax, pw, reasons))
 
     def mark(self, name: str, t0: float, t1: float):
-        """Record the host-clock window [t0, t1] of a timed region."""
+        """Record the wall-clock window [t0, t1] (time.time()) of a timed region."""
         self.windows[name] = (t0, t1)
 
     def stop(self):
@@ -282,24 +287,32 @@ def run_ours(args):
     counts = moe.layer_forward(x, logits, W1, W3, W2, wl.k, ws, moe.MODE_OVERLAPPED, outputs=True,
                                **kw)[1]["counts"].cpu().tolist()
 
+    def cool_down():
+        # every timed region starts from the same power state: the part is capped at
+        # 1 kW and lowers its clock after ~0.1 s of dense MMA work, so without a pause
+        # a region would inherit the clock the previous regions left
+        torch.cuda.synchronize()
+        time.sleep(args.cool_down)
+
     def timed(mode, name, hooks=False):
         K = args.steps
         evb = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if hooks else [None] * K
         eve = [torch.cuda.Event(enable_timing=True) for _ in range(K)] if hooks else [None] * K
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cool_down()
         # a few untimed steps right before the region, so it starts in the steady
         # state rather than after the host-side pause above
         for _ in range(3):
             step(mode)
         barrier()
         torch.cuda.synchronize()
-        h0 = time.monotonic()
+        h0 = time.time()
         e0.record(stream)
         for i in range(K):
             step(mode, evb[i], eve[i])
         e1.record(stream)
         torch.cuda.synchronize()
-        clk.mark(name, h0, time.monotonic())
+        clk.mark(name, h0, time.time())
         barrier()
         total = e0.elapsed_time(e1) / K
         ffn = sum(b.elapsed_time(e) for b, e in zip(evb, eve)) / K if hooks else None
@@ -319,9 +332,10 @@ def run_ours(args):
     ev = {m: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
                torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)] for m in ("seq", "ovl")}
+    cool_down()
     barrier()
     torch.cuda.synchronize()
-    h0 = time.monotonic()
+    h0 = time.time()
     for i in range(K):
         # alternate which mode goes first, so neither always follows the other
         order = (("seq", moe.MODE_SEQUENTIAL), ("ovl", moe.MODE_OVERLAPPED))
@@ -331,7 +345,7 @@ def run_ours(args):
             step(mode, fb, fe)
             e1.record(stream)
     torch.cuda.synchronize()
-    clk.mark("paired", h0, time.monotonic())
+    clk.mark("paired", h0, time.time())
     barrier()
     step_ms = {m: [e0.elapsed_time(e1) for e0, e1, _, _ in ev[m]] for m in ev}
     ffn_ms = {m: [fb.elapsed_time(fe) for _, _, fb, fe in ev[m]] for m in ev}
@@ -349,18 +363,19 @@ def run_ours(args):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         step(moe.MODE_OVERLAPPED)
+    cool_down()
     for _ in range(max(3, args.warmup)):
         g.replay()
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h0 = time.monotonic()
+    h0 = time.time()
     e0.record(stream)
     for _ in range(args.steps):
         g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
-    clk.mark("graph", h0, time.monotonic())
+    clk.mark("graph", h0, time.time())
     barrier()
     t_graph = e0.elapsed_time(e1) / args.steps
     del g
@@ -403,17 +418,18 @@ def run_ours(args):
                 ev_d2h[b].record(d2h)
         stream.wait_stream(d2h)
 
+    cool_down()
     e2e_steps(max(2, args.warmup))
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h0 = time.monotonic()
+    h0 = time.time()
     e0.record(stream)
     h2d.wait_event(e0)
     e2e_steps(args.steps)
     e1.record(stream)
     torch.cuda.synchronize()
-    clk.mark("e2e", h0, time.monotonic())
+    clk.mark("e2e", h0, time.time())
     barrier()
     t_e2e = e0.elapsed_time(e1) / args.steps
     clk.stop()
@@ -710,7 +726,7 @@ def run_sweep(args):
                 used[cell[0]] = c_used
         evs = {c[0]: [] for c in cells}
         torch.cuda.synchronize()
-        h0 = time.monotonic()
+        h0 = time.time()
         n = len(cells)
         for i in range(args.steps):
             for j in range(n):
@@ -721,7 +737,7 @@ def run_sweep(args):
                 e1.record()
                 evs[cell[0]].append((e0, e1))
         torch.cuda.synchronize()
-        clk.mark(name, h0, time.monotonic())
+        clk.mark(name, h0, time.time())
         code, _, _ = moe.get_status(ws)
         if code != moe.MOE_OK:
             raise RuntimeError(f"{name}: {moe.status_string(code)}")

@@ -294,7 +294,7 @@ moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, in
     return MOE_ERR_INVALID;
   constexpr unsigned tile_flags = MOE_SCHED_ONE_CTA | MOE_SCHED_CTA_PAIR | MOE_SCHED_WIDE_CTA |
                                   MOE_SCHED_B_PER_ATOM | MOE_SCHED_FULL_TILES |
-                                  MOE_SCHED_INTERLEAVE | MOE_SCHED_EVICT_FIRST | MOE_SCHED_PREFETCH;
+                                  MOE_SCHED_INTERLEAVE | MOE_SCHED_EVICT_FIRST | MOE_SCHED_EXP_SILU;
   if (flags & ~tile_flags) return MOE_ERR_INVALID;
   const Layout L = layout(T, d, f, E, k);
   if (!ws || !aligned16(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
@@ -369,6 +369,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   if (nsm <= 1 || grid <= ctas_per_tile(V)) return cuda_fail(cudaErrorInvalidConfiguration);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Work w = work_from(ws, L, true, true);
+  if (!gather_a) w.tok_band = nullptr;   // GEMM1's gather indices exist only on that path
   if (A.topk_idx) w.topk_idx = A.topk_idx;
   if (A.topk_gate) w.topk_gate = A.topk_gate;
   if (A.counts) w.counts = A.counts;

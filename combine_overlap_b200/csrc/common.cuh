@@ -291,12 +291,6 @@ __device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, uint64_
       : "memory");
 }
 
-// L2 prefetch of one box of a 4-D tensor (no shared-memory destination).
-__device__ __forceinline__ void tma_prefetch_l2_4d(const void* tmap, int c0, int c1, int c2, int c3) {
-  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
-               :: "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
-}
-
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(tmap) : "memory");
 }

@@ -37,7 +37,7 @@ SCHED_WIDE_CTA = 0x100
 DBG_IDENTITY_EXPERTS = 0x200
 SCHED_INTERLEAVE = 0x400
 SCHED_EVICT_FIRST = 0x800
-SCHED_PREFETCH = 0x1000
+SCHED_EXP_SILU = 0x4000
 
 
 class MoEError(RuntimeError):

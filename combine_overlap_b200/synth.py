@@ -132,6 +132,9 @@ WORKLOADS: dict[str, Workload] = {
     "mixtral": Workload("mixtral", 4096, 4096, 14336, 8, 2, "uniform", 0x5EED0000 + 1),
     "fine_grained": Workload("fine_grained", 8192, 2048, 1408, 64, 6, "zipf", 0x5EED0000 + 2),
     "imbalanced": Workload("imbalanced", 16384, 4096, 1536, 128, 8, "normal2", 0x5EED0000 + 3),
+    # a profiling case of the Mixtral-shaped layer: the same expert shape and rows per
+    # expert (1024) with 2 experts instead of 8, about a quarter of the device memory
+    "mixtral_e2": Workload("mixtral_e2", 1024, 4096, 14336, 2, 2, "uniform", 0x5EED0000 + 5),
     **_sweep(),
 }
 

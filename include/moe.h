@@ -105,11 +105,11 @@ typedef enum {
                                         CTAs then skip GEMM1.  Default: every CTA takes
                                         GEMM1 tiles until that queue is empty before any
                                         GEMM2 tile.  Same bits */
-#define MOE_SCHED_PREFETCH     0x1000u /* single-CTA tiles prefetch their weight tiles
-                                        into L2 8 k-blocks ahead of the TMA loads, 256 K
-                                        rows per prefetch, running on into the next work
-                                        item: more weight bytes in flight per SM where the
-                                        weights stream from DRAM.  Same bits */
+#define MOE_SCHED_EXP_SILU     0x4000u /* GEMM1's epilogue computes silu(a) = a / (1 +
+                                        exp(-a)) (two special-function ops per element)
+                                        instead of the default a/2 (1 + tanh(a/2)) with the
+                                        hardware tanh approximation (one op; other bits in
+                                        h, within the same bound of the oracle) */
 #define MOE_SCHED_EVICT_FIRST  0x800u /* the epilogue stores h and y with an L2
                                         evict-first policy (they compete with the weights
                                         for L2).  Same bits */
@@ -189,7 +189,7 @@ moe_status moe_permute(const void* x, int T, int d, int E, int k, const int32_t*
  * otherwise nothing is computed and moe_get_status returns MOE_ERR_INVALID.
  * flags: 0, or MOE_SCHED_ONE_CTA / MOE_SCHED_CTA_PAIR / MOE_SCHED_WIDE_CTA /
  * MOE_SCHED_B_PER_ATOM / MOE_SCHED_FULL_TILES (tile variant), MOE_SCHED_INTERLEAVE,
- * MOE_SCHED_EVICT_FIRST, MOE_SCHED_PREFETCH; any other bit is MOE_ERR_INVALID. */
+ * MOE_SCHED_EVICT_FIRST, MOE_SCHED_EXP_SILU; any other bit is MOE_ERR_INVALID. */
 moe_status moe_grouped_ffn(const void* x_perm, const int32_t* offsets, int T, int d, int f,
                            int E, int k, const void* W1, const void* W3, const void* W2,
                            void* h, void* y, unsigned flags, void* ws, size_t ws_bytes,
