@@ -359,11 +359,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   // of reading x_perm (no x_perm pass, but 32 gather instructions per k-block);
   // 128-row gathers only, so not with V = 3
   const int gather_a = (A.flags & (MOE_SCHED_GATHER_A | MOE_DBG_IDENTITY_EXPERTS)) == MOE_SCHED_GATHER_A;
-  int V = choose_variant(A.T, A.f, A.E, A.k, A.flags);
-  if (gather_a && V == 3) {
-    if (A.flags & MOE_SCHED_WIDE_CTA) return MOE_ERR_UNSUPPORTED;
-    V = 1;
-  }
+  const int V = choose_variant(A.T, A.f, A.E, A.k, A.flags);
   int grid = 0;
   MOE_TRY(ffn_grid(V, &grid));
   if (nsm <= 1 || grid <= ctas_per_tile(V)) return cuda_fail(cudaErrorInvalidConfiguration);

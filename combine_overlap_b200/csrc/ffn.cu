@@ -102,7 +102,7 @@ struct SmemCtl {
   uint64_t cempty[CONS_SLOTS];   // consumer ring: the slot's token is reduced and stored
   uint64_t gbar[2];              // a GEMM1 tile's gather indices landed (two items in flight)
   Item ring[SCHED_DEPTH];
-  int4 gidx[2][BM / 4];          // token of each of this CTA's 128 rows of a GEMM1 tile
+  int4 gidx[2][2 * BM / 4];      // token of each row of a GEMM1 tile (up to 256 rows)
   uint32_t tmem_base;
   int item;
   int ok;
@@ -290,6 +290,68 @@ __device__ __forceinline__ void arrive_leader(uint64_t* bar, uint32_t rank) {
   else mbar_arrive_remote(mapa_shared(smem_u32(bar), 0));
 }
 
+// ---------------------------------------------------------------- scheduler ---
+// The work-item scheduler of a CTA (a single CTA, or a pair's leader): takes the
+// next item from the atomic queues and publishes it in the item ring (the leader
+// also writes it into its peer's ring over distributed shared memory); a pair's
+// peer reads it from its own ring.  One thread runs it.
+struct Sched {
+  int slot;
+  uint32_t sph;
+  bool g1, g2;
+  bool interleave;
+  unsigned long long* stamp;   // per-CTA debug stamps, or null
+};
+
+template <int V>
+__device__ bool sched_next(Sched& sc, Item& it, const FfnArgs& a, SmemCtl* ctl, uint32_t rank,
+                           int n1, int n2, const volatile uint32_t* abort) {
+  const Work& w = a.w;
+  const int NT2 = a.d / BN2;
+  const uint64_t tmo = a.timeout_ns;
+  const bool leader = V != 2 || rank == 0;
+  if (leader) {
+    it.kind = K_END;
+    if (*abort) sc.g1 = sc.g2 = false;
+    if (sc.interleave && sc.g1) {
+      const int t = (int)atomicAdd(&w.sync->q1, 1u);
+      if (t < n1 + n2) it = decode_mixed(w, t, a.n_units, NT2);
+      else {
+        sc.g1 = sc.g2 = false;
+        if (sc.stamp) sc.stamp[1] = globaltimer();
+      }
+    }
+    if (!sc.interleave && it.kind == K_END && sc.g1) {
+      const int t = (int)atomicAdd(&w.sync->q1, 1u);
+      if (t < n1) it = decode_g1(w, t, a.n_units);
+      else {
+        sc.g1 = false;
+        if (sc.stamp) sc.stamp[1] = globaltimer();
+      }
+    }
+    if (!sc.interleave && it.kind == K_END && sc.g2) {
+      const int t = (int)atomicAdd(&w.sync->q2, 1u);
+      if (t < n2) it = decode_g2(w, t, NT2); else sc.g2 = false;
+    }
+    if (!wait_bar<V == 2>(&ctl->sempty[sc.slot], sc.sph ^ 1u, tmo, abort)) { set_error(w.status, W_SCHED_EMPTY); return false; }
+    ctl->ring[sc.slot] = it;
+    if (V == 2) {
+      const uint4* src = reinterpret_cast<const uint4*>(&it);
+      const uint32_t dst = mapa_shared(smem_u32(&ctl->ring[sc.slot]), 1);
+      st_cluster_v4(dst, src[0]);
+      st_cluster_v4(dst + 16, src[1]);
+      mbar_arrive_remote(mapa_shared(smem_u32(&ctl->sfull[sc.slot]), 1));
+    }
+    mbar_arrive(&ctl->sfull[sc.slot]);
+  } else {
+    if (!wait_bar<true>(&ctl->sfull[sc.slot], sc.sph, tmo, abort)) { set_error(w.status, W_SCHED_FULL); return false; }
+    it = ctl->ring[sc.slot];
+    arrive_leader<V>(&ctl->sempty[sc.slot], rank);
+  }
+  if (++sc.slot == SCHED_DEPTH) { sc.slot = 0; sc.sph ^= 1u; }
+  return true;
+}
+
 // ------------------------------------------------------------ TMA producer ---
 // A single CTA, or the pair leader: takes work items from the atomic queues and puts
 // them in the ring (the leader also writes them into its peer's ring over
@@ -310,11 +372,11 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
                          const volatile uint32_t* abort) {
   using C = Cfg<V>;
   const Work& w = a.w;
-  const int NT1 = a.f / BN1, NT2 = a.d / BN2;
+  const int NT1 = a.f / BN1;
   const uint64_t tmo = a.timeout_ns;
   const bool leader = V != 2 || rank == 0;
-  int stage = 0, slot = 0;
-  uint32_t ph = 0, sph = 0;
+  int stage = 0;
+  uint32_t ph = 0;
   uint32_t pending = 0, pend_par = 0;   // stages with an issued fill, and its parity
   uint32_t gph = 0;                     // parity of the next wait on gbar[0], gbar[1]
   uint32_t gpend = 0;                   // index copies issued and not yet waited, per buffer
@@ -329,50 +391,8 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
   // a GEMM2 tile comes a grid's worth of GEMM1 tiles after the last GEMM1 tile of
   // its unit, so every GEMM1 tile it waits on sits earlier in the queue and was
   // taken by a resident CTA (no deadlock), and is most likely stored already.
-  const bool interleave = (a.flags & MOE_SCHED_INTERLEAVE) && g1 && g2;
-  // Next work item: dequeued and published by a leader, read by a peer.
-  auto next_item = [&](Item& it) -> bool {
-    if (leader) {
-      it.kind = K_END;
-      if (*abort) g1 = g2 = false;
-      if (interleave && g1) {
-        const int t = (int)atomicAdd(&w.sync->q1, 1u);
-        if (t < n1 + n2) it = decode_mixed(w, t, a.n_units, NT2);
-        else {
-          g1 = g2 = false;
-          if (stamp) my_stamps[1] = globaltimer();
-        }
-      }
-      if (!interleave && it.kind == K_END && g1) {
-        const int t = (int)atomicAdd(&w.sync->q1, 1u);
-        if (t < n1) it = decode_g1(w, t, a.n_units);
-        else {
-          g1 = false;
-          if (stamp) my_stamps[1] = globaltimer();
-        }
-      }
-      if (!interleave && it.kind == K_END && g2) {
-        const int t = (int)atomicAdd(&w.sync->q2, 1u);
-        if (t < n2) it = decode_g2(w, t, NT2); else g2 = false;
-      }
-      if (!wait_bar<V == 2>(&ctl->sempty[slot], sph ^ 1u, tmo, abort)) { set_error(w.status, W_SCHED_EMPTY); return false; }
-      ctl->ring[slot] = it;
-      if (V == 2) {
-        const uint4* src = reinterpret_cast<const uint4*>(&it);
-        const uint32_t dst = mapa_shared(smem_u32(&ctl->ring[slot]), 1);
-        st_cluster_v4(dst, src[0]);
-        st_cluster_v4(dst + 16, src[1]);
-        mbar_arrive_remote(mapa_shared(smem_u32(&ctl->sfull[slot]), 1));
-      }
-      mbar_arrive(&ctl->sfull[slot]);
-    } else {
-      if (!wait_bar<true>(&ctl->sfull[slot], sph, tmo, abort)) { set_error(w.status, W_SCHED_FULL); return false; }
-      it = ctl->ring[slot];
-      arrive_leader<V>(&ctl->sempty[slot], rank);
-    }
-    if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
-    return true;
-  };
+  Sched sc{0, 0u, g1, g2, (a.flags & MOE_SCHED_INTERLEAVE) && g1 && g2, stamp ? my_stamps : nullptr};
+  auto next_item = [&](Item& it) -> bool { return sched_next<V>(sc, it, a, ctl, rank, n1, n2, abort); };
   // Does this CTA gather indices for the item?  (GEMM1, gathered path, own rows)
   auto gathers = [&](const Item& it) {
     return a.gather && it.kind == K_G1 && my_rows<V>(it, rank, false).rows > 0;
@@ -506,6 +526,157 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
     while (globaltimer() < until) __nanosleep(1000);
   }
   if (stamp) { my_stamps[4] = n_g1; my_stamps[5] = n_g2; }
+}
+
+// ---------------------------------------------------- TMA producer, gathered ---
+// The producer of single-CTA tiles (V = 1, 3) whose GEMM1 A rows are gathered
+// straight from x (MOE_SCHED_GATHER_A), run by the whole of warp 0: lane 0
+// schedules items, waits on the ring and loads the weight tiles (and GEMM2's h
+// rows) exactly as role_tma does, and all 32 lanes issue the GEMM1 A gathers --
+// lane l the TMA tile::gather4 of rows 4l..4l+3 of each 128-row band of the tile
+// (one instruction per lane per band and k-block, instead of 32 or 64 from one
+// thread).  The tile's token indices (1 or 2 aligned 512-byte rows of tok_band)
+// are bulk-copied into shared memory one work item ahead.
+template <int V>
+__device__ void role_tma_gathered(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
+                                  const CUtensorMap* tm_w3, const CUtensorMap* tm_a2,
+                                  const CUtensorMap* tm_w2, const FfnArgs& a, SmemCtl* ctl,
+                                  uint8_t* smem, bool run_g1, bool run_g2, int n1, int n2,
+                                  const volatile uint32_t* abort) {
+  static_assert(V != 2, "CTA pairs gather from one thread (role_tma)");
+  using C = Cfg<V>;
+  const Work& w = a.w;
+  const int lane = threadIdx.x & 31;
+  const int NT1 = a.f / BN1;
+  const uint64_t tmo = a.timeout_ns;
+  const bool stamp = (a.flags & MOE_DBG_TIMESTAMPS) && blockIdx.x < STAMP_CTAS;
+  unsigned long long* my_stamps = w.stamps + (size_t)blockIdx.x * NSTAMP;
+  Sched sc{0, 0u, run_g1, run_g2, (a.flags & MOE_SCHED_INTERLEAVE) && run_g1 && run_g2,
+           stamp ? my_stamps : nullptr};
+  int stage = 0;
+  uint32_t ph = 0;
+  uint32_t pending = 0, pend_par = 0;   // (lane 0) stages with an issued fill, and its parity
+  uint32_t gph = 0;                     // parity of the next wait on gbar[0], gbar[1]
+  uint32_t gpend = 0;                   // (lane 0) index copies issued and not yet waited
+  unsigned long long n_g1 = 0, n_g2 = 0;
+  // lane 0 takes the next item; every lane gets it
+  auto next_item = [&](Item& it) -> bool {
+    int okf = 1;
+    if (lane == 0) okf = sched_next<V>(sc, it, a, ctl, 0u, n1, n2, abort) ? 1 : 0;
+    okf = __shfl_sync(0xffffffffu, okf, 0);
+    int* p = reinterpret_cast<int*>(&it);
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(Item) / 4); ++i) p[i] = __shfl_sync(0xffffffffu, p[i], 0);
+    return okf != 0;
+  };
+  // bands of the item this CTA computes (V = 3: 1 or 2)
+  auto n_bands = [&](const Item& it) { return (V == 3 && it.rows > BM) ? 2 : 1; };
+  auto fetch_indices = [&](const Item& it, int buf) {
+    if (lane != 0 || it.kind != K_G1 || it.rows <= 0) return;
+    const uint32_t bytes = (uint32_t)(n_bands(it) * BM * 4);   // consecutive bands: one copy
+    fence_proxy_async_shared();   // earlier generic reads of this buffer come first
+    gpend |= 1u << buf;
+    mbar_arrive_expect_tx(&ctl->gbar[buf], bytes);
+    bulk_load(&ctl->gidx[buf][0], a.tok_band + (size_t)it.band0 * BM, bytes, &ctl->gbar[buf]);
+  };
+
+  bool ok = true;
+  Item cur;
+  int buf = 0;
+  if (!next_item(cur)) ok = false;
+  else fetch_indices(cur, buf);
+  while (ok && cur.kind != K_END) {
+    Item nxt;
+    if (!next_item(nxt)) break;
+    fetch_indices(nxt, buf ^ 1);
+    const bool is1 = cur.kind == K_G1;
+    if (is1) ++n_g1; else ++n_g2;
+    const int nb = n_bands(cur);
+    int okw = 1;
+    if (is1 && cur.rows > 0) {
+      // every lane reads the indices: every lane waits for them
+      okw = wait_bar(&ctl->gbar[buf], (gph >> buf) & 1u, tmo, abort) ? 1 : 0;
+      okw = __all_sync(0xffffffffu, okw);
+      gph ^= 1u << buf;
+      if (lane == 0) gpend &= ~(1u << buf);
+    } else if (!is1 && lane == 0) {
+      // GEMM2 reads the group's h rows: every GEMM1 column block of its bands stored
+      okw = (wait_count(&w.band_done1[cur.band0], BAND_UNIT * (uint32_t)NT1, tmo, abort) &&
+             (nb < 2 || wait_count(&w.band_done1[cur.band0 + 1], BAND_UNIT * (uint32_t)NT1, tmo, abort)))
+                ? 1 : 0;
+      if (okw) fence_proxy_async_global();   // generic-proxy stores -> async-proxy (TMA) loads
+    }
+    okw = __shfl_sync(0xffffffffu, okw, 0);
+    if (!okw) { if (lane == 0) set_error(w.status, is1 ? W_STAGE_FULL : W_BAND1); break; }
+    // this lane's token rows of each band (4 per band)
+    int4 tk[2] = {make_int4(0, 0, 0, 0), make_int4(0, 0, 0, 0)};
+    if (is1)
+      for (int b = 0; b < nb; ++b) tk[b] = ctl->gidx[buf][b * (BM / 4) + lane];
+    const int nk = (is1 ? a.d : a.f) / BK;
+    for (int kb = 0; kb < nk; ++kb) {
+      int oks = 1;
+      if (lane == 0) {
+        oks = wait_bar(&ctl->empty[stage], ph ^ 1u, tmo, abort) ? 1 : 0;
+        if (oks) mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE - (nb < 2 ? (C::ABOX - 1) * A_STAGE_BYTES : 0));
+        else set_error(w.status, W_STAGE_EMPTY);
+      }
+      oks = __shfl_sync(0xffffffffu, oks, 0);   // (a warp shuffle orders lane 0's expect first)
+      if (!oks) { ok = false; break; }
+      uint8_t* sa = smem + (size_t)stage * C::STAGE;
+      uint8_t* sb = sa + C::ABOX * A_STAGE_BYTES;
+      uint64_t* fb = &ctl->full[stage];
+      if (is1) {
+        for (int b = 0; b < nb; ++b)
+          tma_gather4(sa + b * A_STAGE_BYTES + lane * 512, tm_a1, fb, kb * BK, tk[b].x, tk[b].y,
+                      tk[b].z, tk[b].w);
+      }
+      if (lane == 0) {
+        if (!is1) {
+          tma_load_2d(sa, tm_a2, fb, kb * BK, cur.row0);
+          if (nb == 2) tma_load_2d(sa + A_STAGE_BYTES, tm_a2, fb, kb * BK, cur.row0 + BM);
+        }
+        const int k0 = kb * BK;
+        if (a.b_atoms) {
+          if (is1) {
+            tma_load_4d(sb, tm_w1, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
+            tma_load_4d(sb + 2 * B_BOX_BYTES, tm_w3, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
+          } else {
+            tma_load_4d(sb, tm_w2, fb, 0, k0, cur.nt * (BN2 / 64), cur.expert);
+          }
+        } else if (is1) {
+          tma_load_3d(sb, tm_w1, fb, cur.nt * BN1, k0, cur.expert);
+          tma_load_3d(sb + B_BOX_BYTES, tm_w1, fb, cur.nt * BN1 + 64, k0, cur.expert);
+          tma_load_3d(sb + 2 * B_BOX_BYTES, tm_w3, fb, cur.nt * BN1, k0, cur.expert);
+          tma_load_3d(sb + 3 * B_BOX_BYTES, tm_w3, fb, cur.nt * BN1 + 64, k0, cur.expert);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            tma_load_3d(sb + q * B_BOX_BYTES, tm_w2, fb, cur.nt * BN2 + q * 64, k0, cur.expert);
+        }
+        pending |= 1u << stage;
+        pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
+      }
+      if (++stage == C::NST) { stage = 0; ph ^= 1u; }
+    }
+    __syncwarp();
+    cur = nxt;
+    buf ^= 1;
+  }
+  if (lane == 0) {
+    // index copies issued for items that were not processed must land too, and
+    // no copy may still be landing in shared memory when the CTA leaves
+    for (int b = 0; b < 2; ++b)
+      if (gpend & (1u << b)) wait_bar(&ctl->gbar[b], (gph >> b) & 1u, tmo, nullptr);
+    bool drained = true;
+    for (int s2 = 0; s2 < C::NST; ++s2)
+      if (pending & (1u << s2)) drained &= wait_bar(&ctl->full[s2], (pend_par >> s2) & 1u, tmo, nullptr);
+    if (!drained) {
+      const uint64_t until = globaltimer() + 100000ull;
+      while (globaltimer() < until) __nanosleep(1000);
+    }
+    if (stamp) { my_stamps[4] = n_g1; my_stamps[5] = n_g2; }
+  }
+  __syncwarp();
 }
 
 // --------------------------------------------------------------- MMA issuer ---
@@ -1164,7 +1335,15 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
 
   if (run_g1 || run_g2) {
     if (warp == 0) {
-      if (lane == 0)
+      bool warp_wide = false;
+      if constexpr (V != 2) {
+        if (a.gather) {
+          role_tma_gathered<V>(&tm_a1, &tm_w1, &tm_w3, &tm_a2, &tm_w2, a, ctl, smem, run_g1, run_g2, n1,
+                               n2, abort);
+          warp_wide = true;
+        }
+      }
+      if (!warp_wide && lane == 0)
         role_tma<V>(&tm_a1, &tm_w1, &tm_w3, &tm_a2, &tm_w2, a, ctl, smem, rank, run_g1, run_g2, n1, n2,
                     abort);
     } else if (warp == 1) {
@@ -1301,7 +1480,6 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (a.V == 3 && a.gather) return cudaErrorInvalidValue;   // gathered A rows: 128-row tiles only
   e = configure_variant(a.V, dev);
   if (e != cudaSuccess) return e;
   CUtensorMap tm_a1, tm_w1, tm_w3, tm_a2, tm_w2;

@@ -75,8 +75,10 @@ typedef enum {
 #define MOE_DBG_TIMESTAMPS     0x8u  /* the persistent kernel records per-CTA globaltimer
                                         stamps, read back with moe_debug_stamps */
 #define MOE_SCHED_GATHER_A     0x10u /* GEMM1 gathers its A rows from x with TMA gather4
-                                        instead of reading a permuted copy (measured slower
-                                        on B200: 32 gather instructions per k-block) */
+                                        (4 rows per instruction) instead of reading the
+                                        permuted copy x_perm, which is then not written:
+                                        single CTAs issue the gathers from all 32 lanes of
+                                        the producer warp, CTA pairs from one thread */
 #define MOE_SCHED_ONE_CTA      0x4u  /* force 128-row MMA tiles on single CTAs          */
 #define MOE_SCHED_CTA_PAIR     0x20u /* force 256-row MMA tiles on CTA pairs (tcgen05
                                         cta_group::2); an expert's odd last row band runs
@@ -116,8 +118,7 @@ typedef enum {
 #define MOE_SCHED_WIDE_CTA     0x100u /* force 256-row MMA tiles on single CTAs: two
                                         128-row MMAs per K step share one B stage and
                                         fill the CTA's two accumulators (an expert's odd
-                                        last band uses the first only).  Not with
-                                        MOE_SCHED_GATHER_A (MOE_ERR_UNSUPPORTED) */
+                                        last band uses the first only) */
 
 typedef struct {
   int T, d, f, E, k;        /* tokens, d_model, d_ff, experts, top-k                */
