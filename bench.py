@@ -43,7 +43,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the persistent FFN kernel, keyed by workload, valid only for the kernel sources
 # whose hash is recorded with it (see profiles/).
-TRAFFIC = {"mixtral": {"bytes": 4156785000 + 314484480, "kernel_hash": "bdecdd82a1a6"}}
+TRAFFIC = {"mixtral": {"bytes": 4165375000 + 311689728, "kernel_hash": "550528ecfe84"}}
 
 
 def kernel_source_hash() -> str:
@@ -102,6 +102,9 @@ def parse():
                     help="comma-separated workloads for --sweep (default: the d=4096/E=32 grid)")
     ap.add_argument("--sweep-cells", default="seq,0,2,4,8,16",
                     help="--sweep cells: 'seq' or 'C[/mgb]' (overlapped, C consumer SMs, 0 = cost model)")
+    ap.add_argument("--ep-sweep", action="store_true",
+                    help="fused expert-parallel return on 2 and 4 virtual ranks: owners' step "
+                         "overlapped vs sequential, and the homes' combine; one JSON line each")
     ap.add_argument("--oracle-timings", action="store_true",
                     help="time the CPU oracle on each benchmark configuration; one JSON line "
                          "per configuration (not the benchmark line)")
@@ -769,10 +772,93 @@ def run_sweep(args):
     clk.stop()
 
 
+def run_ep_sweep(args):
+    """The fused expert-parallel return on W virtual ranks of one GPU: per layer and
+    W, the owners' step (moe_ep_owner_forward: expert GEMMs plus the return of every
+    row band into its home rank's buffer) in the overlapped mode (consumer CTAs
+    return bands while the GEMM runs) against the sequential mode (GEMMs, then the
+    return as its own pass), and the homes' combine.  Each owner's two modes run as
+    paired steps, the order alternating, each timed with CUDA events; medians,
+    summed over the owners.  One JSON line per (layer, W)."""
+    from combine_overlap_b200 import ep, moe
+    torch.cuda.set_device(0)
+    names = args.sweep_layers.split(",") if args.sweep_layers else ["sweep_T8192_uniform", "mixtral"]
+    for name in names:
+        wl = synth.WORKLOADS[name]
+        for W in (2, 4):
+            if wl.E % W:
+                continue
+            T_r = wl.T // W
+            shards = [synth.Workload(f"{name}_r{r}", T_r, wl.d, wl.f, wl.E, wl.k, wl.router,
+                                     wl.seed + 1000 * r) for r in range(W)]
+            xs = [synth.make_x(sw, "cuda") for sw in shards]
+            ls = [synth.make_logits(sw, "cuda") for sw in shards]
+            W1, W3, W2 = synth.make_weights(wl, "cuda")
+            outs, st = ep.virtual_ranks_forward(xs, ls, W1, W3, W2, wl.k)
+            torch.cuda.synchronize()
+            El = wl.E // W
+            homes = st["homes"]
+            t_ovl, t_seq, t_home = 0.0, 0.0, 0.0
+            for o, own in enumerate(st["owners"]):
+                if own["N"] == 0:
+                    continue
+                lo, hi = o * El, (o + 1) * El
+                base = [int(h["offsets"][lo].item()) for h in homes]
+
+                def owner(mode):
+                    moe.ep_owner_forward(own["x_recv"], own["slot_recv"], own["recv_counts"], W1[lo:hi],
+                                         W3[lo:hi], W2[lo:hi], wl.k, o, base, [h["y"] for h in homes],
+                                         [h["arrive"] for h in homes], own["ws"], mode)
+                ev = {m: [] for m in ("ovl", "seq")}
+                for _ in range(max(1, args.warmup)):
+                    owner(moe.MODE_OVERLAPPED)
+                    owner(moe.MODE_SEQUENTIAL)
+                torch.cuda.synchronize()
+                for i in range(args.steps):
+                    order = (("ovl", moe.MODE_OVERLAPPED), ("seq", moe.MODE_SEQUENTIAL))
+                    for m, mode in (order if i % 2 == 0 else order[::-1]):
+                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        e0.record()
+                        owner(mode)
+                        e1.record()
+                        ev[m].append((e0, e1))
+                torch.cuda.synchronize()
+                code, c_used, nb = moe.get_status(own["ws"])
+                if code != moe.MOE_OK:
+                    raise RuntimeError(f"owner {o}: {moe.status_string(code)}")
+                t_ovl += statistics.median(a.elapsed_time(b) for a, b in ev["ovl"])
+                t_seq += statistics.median(a.elapsed_time(b) for a, b in ev["seq"])
+            # every owner ran its steps: each token's arrival word is now a multiple
+            # of k; one home combine per rank consumes the last round of rows
+            for h in homes:
+                h["arrive"].fill_(wl.k)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for h in homes:
+                moe.ep_home_combine(h["y"], h["arrive"], h["row_of"], h["gate"])
+            e1.record()
+            torch.cuda.synchronize()
+            t_home = e0.elapsed_time(e1)
+            ret_bytes = 2 * wl.T * wl.k * wl.d * 2
+            print(json.dumps({"ep_sweep": name, "W": W, "tokens_per_rank": T_r, "steps": args.steps,
+                              "owners_overlapped_ms": t_ovl, "owners_sequential_ms": t_seq,
+                              "speedup_vs_sequential": t_seq / t_ovl, "homes_combine_ms": t_home,
+                              "return_bytes": ret_bytes,
+                              "method": "per owner: overlapped and sequential steps alternating, "
+                                        "CUDA events, medians; summed over owners (run one after "
+                                        "another on one GPU)"}), flush=True)
+            del xs, ls, W1, W3, W2, outs, st
+            torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.ep_sweep:
+        run_ep_sweep(args)
         return
     if args.oracle_timings:
         run_oracle_timings(args)

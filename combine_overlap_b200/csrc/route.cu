@@ -176,21 +176,32 @@ cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int32_t* b
 // B200 of every benchmark layer put C = 0 behind C = 1 on all of them (by 0-5 %),
 // and C = 1 within noise of the best fixed C; the model's trade-off then decides
 // whether more consumers pay.
+// Run by one warp: lane l evaluates candidates C = cmin + (l + 32 i) cg; the pick is
+// the smallest C whose modelled time is within a relative 1e-9 of the minimum.
 __device__ int choose_consumers(int S, int cg, int cmin, long long R, int T, int d, int f,
-                                const CostModel& cm) {
+                                const CostModel& cm, int lane) {
   const double F2 = 2.0 * (double)R * f * d;
   const double Bc = 2.0 * (double)R * d + 2.0 * (double)T * d;
   const double drain = fmin((double)S * cm.copy_bytes_per_sm, (double)cm.hbm_bytes);
-  int best = cmin;
-  double best_t = 1e300;
   const int cmax = min(cm.max_consumers, S - cg);
-  for (int C = cmin; C <= cmax; C += cg) {
+  auto model = [&](int C) {
     const double t2 = F2 / ((double)(S - C) * cm.mma_flops_per_sm);
     const double left = fmax(0.0, Bc - (double)C * cm.copy_bytes_per_sm * t2);
-    const double t = t2 + left / drain;
-    if (t < best_t * (1.0 - 1e-9)) { best_t = t; best = C; }
+    return t2 + left / drain;
+  };
+  double my_t = 1e300;
+  int my_c = 0x7fffffff;
+  for (int C = cmin + lane * cg; C <= cmax; C += 32 * cg) {
+    const double t = model(C);
+    if (t < my_t) { my_t = t; my_c = C; }
   }
-  return best;
+  double tmin = my_t;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) tmin = fmin(tmin, __shfl_xor_sync(0xffffffffu, tmin, off));
+  int pick = my_t <= tmin * (1.0 + 1e-9) ? my_c : 0x7fffffff;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) pick = min(pick, __shfl_xor_sync(0xffffffffu, pick, off));
+  return pick == 0x7fffffff ? cmin : pick;
 }
 
 __host__ __device__ inline int n_items_for(int nb, int mgb) {
@@ -280,9 +291,18 @@ __device__ void plan_tables(const Work& w, int U, const int* cnt, const int* row
       if (tid == 0) w.g2_start[U] = nt1 + ng * NT2;
     }
   }
-  if (tid == 0) {
+  // the split: warp 0 evaluates the model for one candidate C per lane
+  __shared__ int c_pick;
+  if (warp == 0) {
     const int cmin = cg;   // at least one dedicated consumer group (measured: see choose_consumers)
-    int C = consumer_hint > 0 ? consumer_hint : choose_consumers(num_sms, cg, cmin, R, T, d, f, cm);
+    const int C = consumer_hint > 0 ? consumer_hint : choose_consumers(num_sms, cg, cmin, R, T, d, f, cm, lane);
+    if (lane == 0) c_pick = C;
+  }
+  for (int i = tid; i < (int)(sizeof(Sync) / 4); i += blockDim.x) reinterpret_cast<uint32_t*>(w.sync)[i] = 0u;
+  __syncthreads();
+  if (tid == 0) {
+    const int cmin = cg;
+    int C = c_pick;
     C = cg * cdiv(C, cg);                       // consumers come in whole CTA groups
     C = max(cmin, min(C, num_sms - cg));        // and leave at least one producer group
     Status st;
@@ -295,8 +315,6 @@ __device__ void plan_tables(const Work& w, int U, const int* cnt, const int* row
     st.n_items = n_items_for(nb, mgb);
     st.n_groups = ng;
     *w.status = st;
-    uint32_t* z = reinterpret_cast<uint32_t*>(w.sync);
-    for (int i = 0; i < (int)(sizeof(Sync) / 4); ++i) z[i] = 0u;
   }
   if (w.bands == nullptr) return;   // permutation only: no tile plan wanted
   for (int s = tid; s < U; s += blockDim.x) {
@@ -370,15 +388,27 @@ __global__ void __launch_bounds__(1024) plan_kernel(Work w, int nblk, const int3
     for (; b < cb1; ++b) sum += bh[(size_t)b * E + ge];
     if (owner) part[tid] = sum;
     __syncthreads();
-    // per expert, an exclusive scan over the NG chunks (NG <= 128 sequential steps)
-    for (int e = tid; e < E; e += blockDim.x) {
-      int run = 0;
-      for (int c = 0; c < NG; ++c) {
+    // per expert, an exclusive scan over the NG chunks: a warp per expert, each
+    // lane a run of cpl chunks (a sum, a shuffle scan of the sums, the prefixes)
+    const int nwarps = (int)(blockDim.x >> 5);
+    const int cpl = cdiv(NG, 32);
+    for (int e = warp; e < E; e += nwarps) {
+      const int c0 = lane * cpl, c1 = min(NG, c0 + cpl);
+      int sum = 0;
+      for (int c = c0; c < c1; ++c) sum += part[c * E + e];
+      int inc = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += t;
+      }
+      int run = inc - sum;
+      for (int c = c0; c < c1; ++c) {
         const int v = part[c * E + e];
         part[c * E + e] = run;
         run += v;
       }
-      cnt[e] = run;
+      if (lane == 31) cnt[e] = inc;
     }
   } else {
     // caller-supplied offsets (moe_grouped_ffn): they must start at 0, never
