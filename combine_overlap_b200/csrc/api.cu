@@ -358,8 +358,12 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   // MOE_SCHED_GATHER_A: GEMM1 gathers its A rows from x with TMA gather4 instead
   // of reading x_perm (no x_perm pass, but 32 gather instructions per k-block);
   // 128-row gathers only, so not with V = 3
-  const int gather_a = (A.flags & (MOE_SCHED_GATHER_A | MOE_DBG_IDENTITY_EXPERTS)) == MOE_SCHED_GATHER_A;
+  // MOE_SCHED_GATHER_LSU: the same, by extra warps with cp.async (single CTAs only)
+  const int gather_a = (A.flags & MOE_DBG_IDENTITY_EXPERTS) ? 0
+                       : (A.flags & MOE_SCHED_GATHER_LSU) ? 2
+                       : (A.flags & MOE_SCHED_GATHER_A) ? 1 : 0;
   const int V = choose_variant(A.T, A.f, A.E, A.k, A.flags);
+  if (gather_a == 2 && V == 2) return MOE_ERR_UNSUPPORTED;
   int grid = 0;
   MOE_TRY(ffn_grid(V, &grid));
   if (nsm <= 1 || grid <= ctas_per_tile(V)) return cuda_fail(cudaErrorInvalidConfiguration);

@@ -120,6 +120,10 @@ static_assert(sizeof(Item) == 32, "an item is two 16-byte stores");
 size_t ffn_smem_bytes() { return 1024 + (size_t)STAGE_AREA + sizeof(SmemCtl); }
 static_assert(1024 + STAGE_AREA + sizeof(SmemCtl) <= 227 * 1024, "over the 227 KB per-CTA limit");
 
+// Weight-tile bytes of one stage of variant V (the whole B share of a CTA).
+template <int V>
+__device__ __forceinline__ constexpr int NBOX_BYTES() { return Cfg<V>::NBOX * B_BOX_BYTES; }
+
 __device__ __forceinline__ void set_error(Status* st, uint32_t where) {
   if (atomicCAS(&st->code, (uint32_t)ST_OK, (uint32_t)ST_TIMEOUT) == (uint32_t)ST_OK) {
     st->where = where;
@@ -395,7 +399,7 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
   auto next_item = [&](Item& it) -> bool { return sched_next<V>(sc, it, a, ctl, rank, n1, n2, abort); };
   // Does this CTA gather indices for the item?  (GEMM1, gathered path, own rows)
   auto gathers = [&](const Item& it) {
-    return a.gather && it.kind == K_G1 && my_rows<V>(it, rank, false).rows > 0;
+    return a.gather == 1 && it.kind == K_G1 && my_rows<V>(it, rank, false).rows > 0;
   };
   auto fetch_indices = [&](const Item& it, int buf) {
     if (!gathers(it)) return;
@@ -419,7 +423,7 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
     const bool half = half_tile<V>(cur, a);
     const MyRows m = my_rows<V>(cur, rank, half);
     const bool two = V == 3 && m.rows > BM;   // V = 3: the group's second band is present
-    const bool gat = a.gather && is1;
+    const bool gat = a.gather == 1 && is1;
     if (gat && m.rows > 0) {
       if (!wait_bar(&ctl->gbar[buf], (gph >> buf) & 1u, tmo, abort)) { set_error(w.status, W_STAGE_FULL); break; }
       gph ^= 1u << buf;
@@ -442,11 +446,15 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
       uint64_t* fb = &ctl->full[stage];
       const uint32_t fbl = V == 2 ? mapa_shared(smem_u32(fb), 0) : 0u;
       // a pair's leader expects both CTAs' bytes; V = 3 without a second band
-      // loads one A box
+      // loads one A box; GEMM1 A rows copied by the gather warps are not TMA bytes
+      const bool lsu = is1 && a.gather == 2;
       if (leader)
-        mbar_arrive_expect_tx(fb, C::CTAS * C::STAGE - (V == 3 && !two ? A_STAGE_BYTES : 0));
+        mbar_arrive_expect_tx(fb, lsu ? NBOX_BYTES<V>() :
+                                  C::CTAS * C::STAGE - (V == 3 && !two ? A_STAGE_BYTES : 0));
       // A: 128 rows x 64 columns of x_perm (tiled) or of x (gathered); h for GEMM2
-      if (gat) {
+      if (lsu) {
+        // (the gather warps copy these A rows)
+      } else if (gat) {
 #pragma unroll 8
         for (int q = 0; q < BM / 4; ++q) {
           const int4 tk = m.rows > 0 ? ctl->gidx[buf][q] : make_int4(0, 0, 0, 0);
@@ -679,6 +687,79 @@ __device__ void role_tma_gathered(const CUtensorMap* tm_a1, const CUtensorMap* t
   __syncwarp();
 }
 
+// ------------------------------------------- GEMM1 A rows, load/store path ---
+// MOE_SCHED_GATHER_LSU (single CTAs): GW extra warps copy every GEMM1 k-block's
+// A rows straight from x into the stage with 16-byte cp.async, in the 128-byte-
+// swizzled layout a tiled TMA load gives -- chunk c of row r at r*128 +
+// ((c ^ (r & 7)) << 4) -- so x_perm is never written and the TMA thread loads the
+// weights only.  Thread t copies chunk t % 8 of rows t / 8, t / 8 + NT / 8, ...
+// (each warp instruction: 4 rows of 128 contiguous bytes on both sides).  The
+// warps walk the item ring like the MMA and epilogue warps; for every k-block of
+// every item each thread waits (through lane 0) for the stage to be free, issues
+// its copies (GEMM1 only: GEMM2's A rows come by TMA) and arrives on the stage's
+// full barrier with cp.async.mbarrier.arrive.noinc -- the arrival happens when its
+// copies have landed, so the warps never block on them.  The MMA thread, after it
+// waits on the full barrier, fences the generic proxy (these writes) against the
+// async proxy (its operand reads).
+template <int V, int GW>
+__device__ void role_gather_lsu(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int gw, int lane,
+                                const volatile uint32_t* abort) {
+  using C = Cfg<V>;
+  const Work& w = a.w;
+  const uint64_t tmo = a.timeout_ns;
+  constexpr int NT = GW * 32;                  // copying threads
+  constexpr int RSTEP = NT / 8;                // rows per pass of all threads
+  constexpr int ROWS = C::ABOX * BM;           // A rows of a k-block
+  const int gt = gw * 32 + lane;
+  const int c = gt & 7;
+  const size_t row_bytes = (size_t)a.d * 2;
+  const char* x = reinterpret_cast<const char*>(a.x);
+  int slot = 0, stage = 0;
+  uint32_t sph = 0, ph = 0;
+  bool ok = true;
+  while (ok) {
+    if (!__all_sync(0xffffffffu, wait_bar(&ctl->sfull[slot], sph, tmo, abort))) {
+      if (lane == 0 && gw == 0) set_error(w.status, W_SCHED_FULL);
+      break;
+    }
+    const Item it = ctl->ring[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->sempty[slot]);
+    if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
+    if (it.kind == K_END) break;
+    const bool is1 = it.kind == K_G1;
+    const int nk = (is1 ? a.d : a.f) / BK;
+    // rows to copy: the group's bands (V = 3 without a second band: the first 128)
+    const int nrows = (V == 3 && it.rows > BM) ? 2 * BM : BM;
+    const int32_t* tok = a.tok_band + (size_t)it.band0 * BM;   // 0 past the bands' rows
+    for (int kb = 0; kb < nk; ++kb) {
+      int okw = 1;
+      if (lane == 0) okw = wait_bar(&ctl->empty[stage], ph ^ 1u, tmo, abort) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) {
+        if (lane == 0 && gw == 0) set_error(w.status, W_STAGE_EMPTY);
+        ok = false;
+        break;
+      }
+      if (is1) {
+        uint8_t* sa = smem + (size_t)stage * C::STAGE;
+        const size_t col = (size_t)kb * BK * 2 + (size_t)c * 16;
+#pragma unroll 4
+        for (int r = gt >> 3; r < ROWS; r += RSTEP) {
+          if (r >= nrows) break;
+          const int t = __ldg(tok + r);
+          cp_async16(sa + r * 128 + ((c ^ (r & 7)) << 4), x + (size_t)t * row_bytes + col);
+        }
+        cp_async_arrive_noinc(&ctl->full[stage]);   // arrives when these copies landed
+      } else {
+        mbar_arrive(&ctl->full[stage]);
+      }
+      if (++stage == C::NST) { stage = 0; ph ^= 1u; }
+    }
+  }
+  cp_async_wait<0>();   // never leave with copies landing in shared memory
+}
+
 // --------------------------------------------------------------- MMA issuer ---
 // One thread (a single CTA's, or the pair leader's) issues every MMA.
 // V = 1, 2: one accumulator per tile, alternating, so the epilogue of tile i
@@ -694,6 +775,7 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
   constexpr uint32_t idesc_half = idesc_bf16_f32(BM, 256, true);   // V == 2 only
   int stage = 0, slot = 0, acc = 0;
   uint32_t ph = 0, sph = 0, aph = 0;
+  const bool lsu = a.gather == 2;
   while (true) {
     if (!wait_bar(&ctl->sfull[slot], sph, tmo, abort)) { set_error(a.w.status, W_SCHED_FULL); break; }
     const Item it = ctl->ring[slot];
@@ -724,6 +806,7 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
       };
       for (int kb = 0; kb < nk && ok; ++kb) {
         if (!wait_bar(&ctl->full[stage], ph, tmo, abort)) { set_error(a.w.status, W_STAGE_FULL); ok = false; break; }
+        if (lsu) fence_proxy_async_shared();   // the gather warps' generic-proxy writes
         tc_fence_after();
         for (int b = 0; b < 2; ++b) {
           if (kb == 0 && !acc_free(b)) { ok = false; break; }
@@ -746,6 +829,7 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
     const uint32_t idesc = half_tile<V>(it, a) ? idesc_half : idesc_full;
     for (int kb = 0; kb < nk; ++kb) {
       if (!wait_bar<V == 2>(&ctl->full[stage], ph, tmo, abort)) { set_error(a.w.status, W_STAGE_FULL); ok = false; break; }
+      if (lsu) fence_proxy_async_shared();   // the gather warps' generic-proxy writes
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + (size_t)stage * C::STAGE);
       const uint32_t sb = sa + A_STAGE_BYTES;
@@ -991,8 +1075,9 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
   const int k = a.k, d = a.d, dv = d >> 3;
   const uint32_t T = (uint32_t)a.T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NWARPS = FFN_THREADS / 32;
-  constexpr int NCW = NWARPS - 1;                         // reducing warps
+  const int NTHREADS = (int)blockDim.x;
+  const int NWARPS = NTHREADS / 32;
+  const int NCW = NWARPS - 1;                             // reducing warps
   const uint32_t row_bytes = (uint32_t)d * 2u;
   const uint32_t tok_bytes = row_bytes * (uint32_t)k;
   int S = (int)((size_t)STAGE_AREA / tok_bytes);
@@ -1071,7 +1156,7 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
         if (bstamp) { bs[0] = globaltimer(); bs[3] = blockIdx.x; }
         const Band bd = w.bands[b];
         unsigned long long completed = 0;
-        for (int r = threadIdx.x; r < bd.rows; r += FFN_THREADS) {
+        for (int r = threadIdx.x; r < bd.rows; r += NTHREADS) {
           const int t = w.perm[bd.row0 + r] / k;
           if (atom_acq_rel_add(&w.arrive[t], 1u) == (uint32_t)(k - 1)) {
             const uint32_t e = atomicAdd(&w.sync->rq_alloc, 1u);
@@ -1237,16 +1322,16 @@ __device__ void role_return(const FfnArgs& a, SmemCtl* ctl, int nb, int n_items,
       const uint4* src = reinterpret_cast<const uint4*>(a.y) + (size_t)bd.row0 * dv;
       uint4* home = reinterpret_cast<uint4*>(a.ep_home_y[dst.x]) + (size_t)dst.y * dv;
       const size_t n = (size_t)bd.rows * dv;
-      for (size_t i0 = threadIdx.x; i0 < n; i0 += (size_t)FFN_THREADS * U) {
+      for (size_t i0 = threadIdx.x; i0 < n; i0 += (size_t)blockDim.x * U) {
         uint4 v[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-          const size_t i = i0 + (size_t)u * FFN_THREADS;
+          const size_t i = i0 + (size_t)u * blockDim.x;
           if (i < n) v[u] = __ldcg(src + i);   // y rows were stored by other SMs: read through L2
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-          const size_t i = i0 + (size_t)u * FFN_THREADS;
+          const size_t i = i0 + (size_t)u * blockDim.x;
           if (i < n) home[i] = v[u];
         }
       }
@@ -1256,7 +1341,7 @@ __device__ void role_return(const FfnArgs& a, SmemCtl* ctl, int nb, int n_items,
     for (int b = b0; b < b1; ++b) {
       const Band bd = w.bands[b];
       uint32_t* arrive = a.ep_home_arrive[w.band_dest[b].x];
-      for (int r = threadIdx.x; r < bd.rows; r += FFN_THREADS)
+      for (int r = threadIdx.x; r < bd.rows; r += (int)blockDim.x)
         red_release_sys_add(&arrive[a.ep_slot[bd.row0 + r] / k], 1u);
     }
     if (threadIdx.x == 0 && (a.flags & MOE_DBG_TIMESTAMPS) && blockIdx.x < STAMP_CTAS)
@@ -1266,11 +1351,14 @@ __device__ void role_return(const FfnArgs& a, SmemCtl* ctl, int nb, int n_items,
 }
 
 // ------------------------------------------------------------------- kernel ---
-template <int V>
-__global__ void __launch_bounds__(FFN_THREADS, 1)
+// GW: extra warps that copy GEMM1's A rows from x (MOE_SCHED_GATHER_LSU), 0 otherwise.
+template <int V, int GW>
+__global__ void __launch_bounds__(FFN_THREADS + 32 * GW, 1)
 ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_w1,
            const __grid_constant__ CUtensorMap tm_w3, const __grid_constant__ CUtensorMap tm_a2,
            const __grid_constant__ CUtensorMap tm_w2, const FfnArgs a) {
+  constexpr int NTHREADS = FFN_THREADS + 32 * GW;
+  constexpr int GW0 = FFN_THREADS / 32;         // first gather warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + (size_t)STAGE_AREA);
@@ -1281,18 +1369,21 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
 
   // prologue (touches nothing the previous kernel writes): barriers, TMEM, descriptors
   if (threadIdx.x == 0) {
-    for (int i = 0; i < MAX_NST; ++i) { mbar_init(&ctl->full[i], 1); mbar_init(&ctl->empty[i], 1); }
+    // a stage is full after the TMA thread's expected bytes and, with gather warps, one
+    // arrival per gather thread
+    for (int i = 0; i < MAX_NST; ++i) { mbar_init(&ctl->full[i], 1 + 32 * GW); mbar_init(&ctl->empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&ctl->tfull[i], 1); mbar_init(&ctl->tempty[i], EPI_WARPS * CTAS); }
     for (int i = 0; i < SCHED_DEPTH; ++i) {
       mbar_init(&ctl->sfull[i], 1);
-      mbar_init(&ctl->sempty[i], (1 + EPI_WARPS) * CTAS);   // MMA + epilogue; a pair adds the peer's TMA + epilogue
+      // MMA + epilogue (+ gather warps); a pair adds the peer's TMA + epilogue
+      mbar_init(&ctl->sempty[i], (1 + EPI_WARPS + GW) * CTAS);
     }
     mbar_init(&ctl->epi_done[0], EPI_WARPS);
     mbar_init(&ctl->epi_done[1], EPI_WARPS);
     mbar_init(&ctl->mma_done, 1);
     mbar_init(&ctl->gbar[0], 1);
     mbar_init(&ctl->gbar[1], 1);
-    for (int i = 0; i < CONS_SLOTS; ++i) { mbar_init(&ctl->cfull[i], 1); mbar_init(&ctl->cempty[i], FFN_THREADS / 32 - 1); }
+    for (int i = 0; i < CONS_SLOTS; ++i) { mbar_init(&ctl->cfull[i], 1); mbar_init(&ctl->cempty[i], NTHREADS / 32 - 1); }
     mbar_fence_init();
     fence_proxy_async_shared();
   }
@@ -1337,7 +1428,7 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
     if (warp == 0) {
       bool warp_wide = false;
       if constexpr (V != 2) {
-        if (a.gather) {
+        if (a.gather == 1) {
           role_tma_gathered<V>(&tm_a1, &tm_w1, &tm_w3, &tm_a2, &tm_w2, a, ctl, smem, run_g1, run_g2, n1,
                                n2, abort);
           warp_wide = true;
@@ -1348,8 +1439,10 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
                     abort);
     } else if (warp == 1) {
       if (lane == 0 && rank == 0) role_mma<V>(a, ctl, smem, tmem_base, abort);
-    } else {
+    } else if (warp < GW0) {
       role_epilogue<V>(a, ctl, tmem_base, rank, warp, lane, abort);
+    } else {
+      if constexpr (GW > 0 && V != 2) role_gather_lsu<V, GW>(a, ctl, smem, warp - GW0, lane, abort);
     }
     __syncwarp();
   }
@@ -1417,14 +1510,19 @@ static bool encode4(CUtensorMap* m, const void* base, const cuuint64_t* dims,
 
 namespace {
 constexpr int MAX_DEV = 64;
-int g_configured[3][MAX_DEV] = {{0}};
-int g_grid[3][MAX_DEV] = {{0}};
+constexpr int LSU_GW = 2;   // gather warps of the MOE_SCHED_GATHER_LSU kernels
+// index of (V, with gather warps): 0-2 plain V = 1..3, 3 V = 1 + GW, 4 V = 3 + GW
+int g_configured[5][MAX_DEV] = {{0}};
+int g_grid[5][MAX_DEV] = {{0}};
 
-template <int V>
+inline int kernel_slot(int V, int gw) { return gw ? (V == 1 ? 3 : 4) : V - 1; }
+
+template <int V, int GW>
 cudaError_t configure(int dev) {
   if (dev < 0 || dev >= MAX_DEV) return cudaErrorInvalidDevice;
-  if (g_configured[V - 1][dev]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(ffn_kernel<V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const int ks = kernel_slot(V, GW);
+  if (g_configured[ks][dev]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(ffn_kernel<V, GW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)ffn_smem_bytes());
   if (e != cudaSuccess) return e;
   int nsm = 0;
@@ -1445,21 +1543,26 @@ cudaError_t configure(int dev) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, ffn_kernel<2>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&clusters, ffn_kernel<2, 0>, &cfg);
     if (e != cudaSuccess) return e;
     if (clusters < 1) return cudaErrorInvalidConfiguration;
     grid = 2 * min(clusters, nsm / 2);
   }
-  g_grid[V - 1][dev] = grid;
-  g_configured[V - 1][dev] = 1;
+  g_grid[ks][dev] = grid;
+  g_configured[ks][dev] = 1;
   return cudaSuccess;
 }
 
-cudaError_t configure_variant(int V, int dev) {
+cudaError_t configure_variant(int V, int gw, int dev) {
+  if (gw) {
+    if (V == 1) return configure<1, LSU_GW>(dev);
+    if (V == 3) return configure<3, LSU_GW>(dev);
+    return cudaErrorInvalidValue;   // CTA pairs have no gather-warp kernel
+  }
   switch (V) {
-    case 1: return configure<1>(dev);
-    case 2: return configure<2>(dev);
-    case 3: return configure<3>(dev);
+    case 1: return configure<1, 0>(dev);
+    case 2: return configure<2, 0>(dev);
+    case 3: return configure<3, 0>(dev);
   }
   return cudaErrorInvalidValue;
 }
@@ -1470,9 +1573,9 @@ cudaError_t ffn_grid(int V, int* grid) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  e = configure_variant(V, dev);
+  e = configure_variant(V, 0, dev);
   if (e != cudaSuccess) return e;
-  *grid = g_grid[V - 1][dev];
+  *grid = g_grid[kernel_slot(V, 0)][dev];
   return cudaSuccess;
 }
 
@@ -1480,11 +1583,12 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  e = configure_variant(a.V, dev);
+  const int gw = a.gather == 2 ? LSU_GW : 0;
+  e = configure_variant(a.V, gw, dev);
   if (e != cudaSuccess) return e;
   CUtensorMap tm_a1, tm_w1, tm_w3, tm_a2, tm_w2;
   const cuuint64_t R = (cuuint64_t)a.R, d = (cuuint64_t)a.d, f = (cuuint64_t)a.f, E = (cuuint64_t)a.E;
-  if (a.gather) {
+  if (a.gather == 1) {
     // token rows of x, boxes one row high for gather4
     const cuuint64_t dims[2] = {d, (cuuint64_t)a.T}, st[1] = {d * 2};
     if (!encode(&tm_a1, a.x, 2, dims, st, 1)) return cudaErrorInvalidValue;
@@ -1519,7 +1623,7 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(FFN_THREADS);
+  cfg.blockDim = dim3(FFN_THREADS + 32 * gw);
   cfg.dynamicSmemBytes = ffn_smem_bytes();
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -1538,9 +1642,13 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
     cfg.numAttrs = 1;
   }
   cfg.attrs = attr;
-  if (a.V == 2) return cudaLaunchKernelEx(&cfg, ffn_kernel<2>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
-  if (a.V == 3) return cudaLaunchKernelEx(&cfg, ffn_kernel<3>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
-  return cudaLaunchKernelEx(&cfg, ffn_kernel<1>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+  if (gw) {
+    if (a.V == 3) return cudaLaunchKernelEx(&cfg, ffn_kernel<3, LSU_GW>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+    return cudaLaunchKernelEx(&cfg, ffn_kernel<1, LSU_GW>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+  }
+  if (a.V == 2) return cudaLaunchKernelEx(&cfg, ffn_kernel<2, 0>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+  if (a.V == 3) return cudaLaunchKernelEx(&cfg, ffn_kernel<3, 0>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+  return cudaLaunchKernelEx(&cfg, ffn_kernel<1, 0>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
 }
 
 }  // namespace moe

@@ -83,7 +83,8 @@ struct FfnArgs {
   const __nv_bfloat16* x_perm;   // A operand of GEMM1 (tiled path)
   const __nv_bfloat16* x;        // token rows for GEMM1's gathered A path
   const int32_t* tok_band;       // [bands][BM] token of each band row (gathered path)
-  int gather;                    // 1: GEMM1 gathers its A rows from x with TMA gather4
+  int gather;                    // GEMM1's A rows from x instead of x_perm: 1 TMA gather4,
+                                 // 2 cp.async by extra gather warps (single CTAs)
   __nv_bfloat16* h;              // GEMM1 output / GEMM2 A operand
   __nv_bfloat16* y;              // GEMM2 output
   const void* W1; const void* W3; const void* W2;

@@ -38,6 +38,7 @@ DBG_IDENTITY_EXPERTS = 0x200
 SCHED_INTERLEAVE = 0x400
 SCHED_EVICT_FIRST = 0x800
 SCHED_EXP_SILU = 0x4000
+SCHED_GATHER_LSU = 0x8000
 
 
 class MoEError(RuntimeError):

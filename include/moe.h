@@ -112,6 +112,11 @@ typedef enum {
                                         instead of the default a/2 (1 + tanh(a/2)) with the
                                         hardware tanh approximation (one op; other bits in
                                         h, within the same bound of the oracle) */
+#define MOE_SCHED_GATHER_LSU   0x8000u /* single-CTA tiles: two extra warps copy GEMM1's
+                                        A rows from x with 16-byte cp.async into the
+                                        swizzled operand layout (x_perm is not written);
+                                        the TMA loads the weights only.  Same bits.  With
+                                        CTA pairs: MOE_ERR_UNSUPPORTED */
 #define MOE_SCHED_EVICT_FIRST  0x800u /* the epilogue stores h and y with an L2
                                         evict-first policy (they compete with the weights
                                         for L2).  Same bits */

@@ -103,14 +103,17 @@ def test_layer_small(orc, wl):
     dflt, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED)
     assert moe.tile_variant(wl.T, wl.f, wl.E, wl.k) == (3 if wl.T * wl.k >= 256 * wl.E else 1)
     assert np.array_equal(gu.host(dflt), gu.host(seq1))
-    # GEMM1 reading its A rows with TMA gather4 from x instead of x_perm: same
-    # arithmetic on the same rows, so the same bits, in every tile variant;
+    # GEMM1 reading its A rows from x instead of x_perm -- copied by extra warps
+    # with cp.async, or by TMA gather4: same arithmetic on the same rows, so the
+    # same bits, in every tile variant;
     # and single CTAs loading the weight tiles one 64-column atom per copy (3-D
     # maps) instead of one 4-D copy per operand: the same bytes in the same places
     # and CTA pairs running an expert's odd last band as a full 256-row tile
     # and the schedule and store-policy variants: GEMM2 tiles interleaved with
     # GEMM1 tiles (instead of all GEMM1 tiles first), evict-first h/y stores
-    for fl in (moe.SCHED_GATHER_A | pair, moe.SCHED_GATHER_A | one, moe.SCHED_GATHER_A | wide,
+    for fl in (moe.SCHED_GATHER_LSU | one, moe.SCHED_GATHER_LSU | wide,
+               moe.SCHED_GATHER_LSU | wide | moe.SCHED_INTERLEAVE,
+               moe.SCHED_GATHER_A | pair, moe.SCHED_GATHER_A | one, moe.SCHED_GATHER_A | wide,
                moe.SCHED_GATHER_A | wide | moe.SCHED_B_PER_ATOM, moe.SCHED_B_PER_ATOM | one,
                moe.SCHED_FULL_TILES | pair, moe.SCHED_INTERLEAVE | one, moe.SCHED_INTERLEAVE | pair,
                moe.SCHED_INTERLEAVE | wide, moe.SCHED_EVICT_FIRST | wide,
@@ -234,6 +237,16 @@ def test_layer_every_token_one_expert(orc, k):
     inp = gu.inputs(wl)
     inp["logits"][:, 3] += 50.0
     _check_variants(orc, wl, inp)
+
+
+def test_gather_lsu_refuses_cta_pairs():
+    # the cp.async gather warps exist for single-CTA tiles only
+    wl = synth.WORKLOADS["tiny"]
+    inp = gu.inputs(wl)
+    ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
+    with pytest.raises(moe.MoEError) as e:
+        _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=moe.SCHED_GATHER_LSU | moe.SCHED_CTA_PAIR)
+    assert e.value.code == moe.MOE_ERR_UNSUPPORTED
 
 
 def test_binding_rejects_mismatched_shapes():
