@@ -444,6 +444,10 @@ def run_ours(args):
     code, _, _ = moe.get_status(ws)
     if code != moe.MOE_OK:
         raise RuntimeError(f"timed runs: {moe.status_string(code)}")
+    # one more overlapped call, untimed: how many tokens the persistent kernel
+    # combined itself (the combine pass after it did the rest)
+    step(moe.MODE_OVERLAPPED)
+    in_kernel = moe.debug_tokens_combined(ws, wl.T, wl.d, wl.f, wl.E, wl.k, stream)
 
     (t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med, ffn_ovl_med, post_seq, post_ovl,
      t_graph, t_ovl_hooked) = max_over_ranks([t_ovl, t_seq, ffn_ovl, ffn_seq, t_e2e, t_ovl_med,
@@ -511,7 +515,9 @@ def run_ours(args):
             "overlap": {"producer_only_ms": ffn_seq, "combine_only_ms": post_seq,
                         "overlapped_ms": ffn_ovl_med + post_ovl, "remainder_combine_ms": post_ovl,
                         "ratio": 1.0 - (ffn_ovl_med + post_ovl - ffn_seq) / post_seq,
-                        "op_speedup": (ffn_seq + post_seq) / (ffn_ovl_med + post_ovl)},
+                        "op_speedup": (ffn_seq + post_seq) / (ffn_ovl_med + post_ovl),
+                        "tokens_combined_in_kernel": in_kernel,
+                        "tokens": wl.T},
             "graph": {"ms_per_step": t_graph, "eager_ms_per_step": t_ovl,
                       "method": "the overlapped call captured once in a CUDA graph, K replays"},
             "consumer_sms": consumer_sms,
@@ -744,6 +750,13 @@ def run_sweep(args):
         code, _, _ = moe.get_status(ws)
         if code != moe.MOE_OK:
             raise RuntimeError(f"{name}: {moe.status_string(code)}")
+        # per overlapped cell, one more untimed call: tokens the persistent kernel
+        # combined itself
+        in_kernel = {}
+        for cell in cells:
+            if cell[1] is not None:
+                step(cell)
+                in_kernel[cell[0]] = moe.debug_tokens_combined(ws, wl.T, wl.d, wl.f, wl.E, wl.k)
         ms = {c: sorted(a.elapsed_time(b) for a, b in v) for c, v in evs.items()}
         med = {c: statistics.median(v) for c, v in ms.items()}
         q = {c: (v[len(v) // 4], v[(3 * len(v)) // 4]) for c, v in ms.items()}
@@ -759,6 +772,8 @@ def run_sweep(args):
                     "roofline_frac": t_roof / med[c]}
             if c in used:
                 cell["consumer_sms_used"] = used[c]
+            if c in in_kernel:
+                cell["tokens_combined_in_kernel"] = in_kernel[c]
             if "seq" in med and c != "seq":
                 cell["speedup_vs_sequential"] = med["seq"] / med[c]
             base = cells[0][0]

@@ -6,6 +6,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <vector>
+
 namespace moe {
 namespace {
 // The CUDA error behind the calling thread's latest MOE_ERR_CUDA.
@@ -364,6 +366,12 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
                        : (A.flags & MOE_SCHED_GATHER_A) ? 1 : 0;
   const int V = choose_variant(A.T, A.f, A.E, A.k, A.flags);
   if (gather_a == 2 && V == 2) return MOE_ERR_UNSUPPORTED;
+  // MOE_SCHED_SIDE_COMBINE: side combine warps in every producer CTA (single CTAs;
+  // CTA pairs keep the ticketed consumer protocol); exclusive with the LSU gather,
+  // which uses the same extra warps
+  const bool side_flag = (A.flags & MOE_SCHED_SIDE_COMBINE) != 0;
+  if (side_flag && gather_a == 2) return MOE_ERR_UNSUPPORTED;
+  const int side = (side_flag && V != 2 && mode == MOE_MODE_OVERLAPPED) ? 1 : 0;
   int grid = 0;
   MOE_TRY(ffn_grid(V, &grid));
   if (nsm <= 1 || grid <= ctas_per_tile(V)) return cuda_fail(cudaErrorInvalidConfiguration);
@@ -380,7 +388,9 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   const int nblk = route_blocks(T);
   MOE_TRY(launch_route(A.logits, T, E, k, w.topk_idx, w.topk_gate, w.blk_hist, w.arrive, w.ready_q, st));
   const int join = (A.flags & MOE_SCHED_NO_JOIN) ? 0 : 1;
-  MOE_TRY(launch_plan(w, nblk, nullptr, T, d, f, E, k, grid, A.consumer_sms, mgb, bands_per_tile(V),
+  // with side warps no SM is a dedicated consumer unless the caller asks for some
+  const int consumer_hint = (side && A.consumer_sms == 0) ? -1 : A.consumer_sms;
+  MOE_TRY(launch_plan(w, nblk, nullptr, T, d, f, E, k, grid, consumer_hint, mgb, bands_per_tile(V),
                       ctas_per_tile(V), join,
                       default_cost_model(), st));
   // Default: a gather kernel writes x_perm and GEMM1 reads it with tiled TMA loads.
@@ -417,6 +427,7 @@ moe_status moe_layer_forward(const moe_layer_args* args, moe_mode mode, void* ws
   if (mode == MOE_MODE_OVERLAPPED) {
     a.phase = PH_G1 | PH_G2 | PH_CONS;
     a.join = join;
+    a.side = side;
     MOE_TRY(launch_ffn(a, grid, st));
     if (A.ev_ffn_end) MOE_TRY(cudaEventRecord(static_cast<cudaEvent_t>(A.ev_ffn_end), st));
     // Consumers stop once the GEMM work is done; a full-occupancy combine pass
@@ -570,6 +581,22 @@ moe_status moe_debug_stamps(void* ws, void* stream, uint64_t* host_out, int max_
     for (int i = 0; i < n; ++i) g += host_out[(size_t)i * NSTAMP] != 0;
     *n_ctas = g;
   }
+  return MOE_OK;
+}
+
+moe_status moe_debug_tokens_combined(const void* ws, int T, int d, int f, int E, int k, void* stream,
+                                     int* n_combined) {
+  if (!ws || !aligned16(ws) || !n_combined) return MOE_ERR_INVALID;
+  moe_status s = check_shape(T, d, f, E, k);
+  if (s != MOE_OK) return s;
+  MOE_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  const Layout L = layout(T, d, f, E, k);
+  std::vector<uint32_t> words((size_t)T);
+  MOE_TRY(cudaMemcpy(words.data(), static_cast<const char*>(ws) + L.arrive, (size_t)T * 4,
+                     cudaMemcpyDeviceToHost));
+  int n = 0;
+  for (uint32_t v : words) n += (v & TOKEN_DONE) ? 1 : 0;
+  *n_combined = n;
   return MOE_OK;
 }
 

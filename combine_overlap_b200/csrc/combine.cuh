@@ -26,17 +26,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-// One warp combines token t.  y rows are read through L2 (ld.global.cg): a row
-// may have been written by another SM during this kernel.
-__device__ __forceinline__ void combine_token_warp(const __nv_bfloat16* __restrict__ y,
-                                                   const int32_t* __restrict__ row_of,
-                                                   const float* __restrict__ gate, int t, int d,
-                                                   int k, __nv_bfloat16* __restrict__ out,
-                                                   int lane) {
-  int rows[MAX_K];
-  float g[MAX_K];
+// One warp combines token t (k <= KMAX): each pass, every lane loads U 16-byte
+// vectors of each of the k rows (U*k loads in flight), then reduces them.  y rows
+// are read through L2 (ld.global.cg): a row may have been written by another SM
+// during this kernel.  The arithmetic per element does not depend on KMAX or U.
+template <int KMAX, int U>
+__device__ __forceinline__ void combine_token_warp_u(const __nv_bfloat16* __restrict__ y,
+                                                     const int32_t* __restrict__ row_of,
+                                                     const float* __restrict__ gate, int t, int d,
+                                                     int k, __nv_bfloat16* __restrict__ out,
+                                                     int lane) {
+  int rows[KMAX];
+  float g[KMAX];
 #pragma unroll
-  for (int j = 0; j < MAX_K; ++j) {
+  for (int j = 0; j < KMAX; ++j) {
     if (j < k) {
       rows[j] = row_of[(size_t)t * k + j];
       g[j] = gate[(size_t)t * k + j];
@@ -45,25 +48,24 @@ __device__ __forceinline__ void combine_token_warp(const __nv_bfloat16* __restri
   const int dv = d >> 3;
   const uint4* yv = reinterpret_cast<const uint4*>(y);
   uint4* ov = reinterpret_cast<uint4*>(out) + (size_t)t * dv;
-  // two 16-byte vectors per lane per pass: 2k loads in flight per lane
-  for (int v0 = lane; v0 < dv; v0 += 64) {
-    const bool two = v0 + 32 < dv;
-    uint4 in[2][MAX_K];
+  for (int v0 = lane; v0 < dv; v0 += 32 * U) {
+    uint4 in[U][KMAX];
 #pragma unroll
-    for (int j = 0; j < MAX_K; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
       if (j < k) {
-        in[0][j] = __ldcg(yv + (size_t)rows[j] * dv + v0);
-        if (two) in[1][j] = __ldcg(yv + (size_t)rows[j] * dv + v0 + 32);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (v0 + 32 * u < dv) in[u][j] = __ldcg(yv + (size_t)rows[j] * dv + v0 + 32 * u);
       }
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      if (u == 1 && !two) break;
+    for (int u = 0; u < U; ++u) {
+      if (v0 + 32 * u >= dv) break;
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
 #pragma unroll
-      for (int j = 0; j < MAX_K; ++j) {
+      for (int j = 0; j < KMAX; ++j) {
         if (j < k) {
           float f[8];
           bf16x8_to_f32(in[u][j], f);
@@ -79,6 +81,15 @@ __device__ __forceinline__ void combine_token_warp(const __nv_bfloat16* __restri
       ov[v0 + 32 * u] = o;
     }
   }
+}
+
+// The combine kernels' form: two vectors per lane per pass, any k <= MAX_K.
+__device__ __forceinline__ void combine_token_warp(const __nv_bfloat16* __restrict__ y,
+                                                   const int32_t* __restrict__ row_of,
+                                                   const float* __restrict__ gate, int t, int d,
+                                                   int k, __nv_bfloat16* __restrict__ out,
+                                                   int lane) {
+  combine_token_warp_u<MAX_K, 2>(y, row_of, gate, t, d, k, out, lane);
 }
 
 }  // namespace moe

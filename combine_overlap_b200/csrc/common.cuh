@@ -42,7 +42,8 @@ enum : uint32_t { ST_OK = 0, ST_INVALID = 1, ST_TIMEOUT = 4 };
 enum : uint32_t {
   W_NONE = 0, W_SCHED_EMPTY = 1, W_SCHED_FULL = 2, W_STAGE_EMPTY = 3, W_STAGE_FULL = 4,
   W_TMEM_EMPTY = 5, W_TMEM_FULL = 6, W_BAND1 = 7, W_BAND2 = 8, W_DRAIN = 9,
-  W_CONS_EMPTY = 10, W_CONS_FULL = 11, W_CONS_QUEUE = 12, W_CONS_IDLE = 13
+  W_CONS_EMPTY = 10, W_CONS_FULL = 11, W_CONS_QUEUE = 12, W_CONS_IDLE = 13,
+  W_SIDE_QUEUE = 14, W_SIDE_IDLE = 15
 };
 
 struct Status {

@@ -89,6 +89,9 @@ struct __align__(16) Item {
 constexpr int EPI_WARPS = FFN_THREADS / 32 - 2;   // warps 2.. : two per TMEM lane quadrant
 constexpr int OSTAGE_ROW = 80;                    // staged bytes per row: 64 of data + 16 of pad
 
+constexpr int SIDE_RING = 64;   // completed bands a CTA's side warps may have pending
+constexpr int SIDE_TOK = 2;     // ready tokens a side warp claims at a time
+
 struct SmemCtl {
   uint64_t full[MAX_NST];        // operands of a stage landed (pair: counted on the leader)
   uint64_t empty[MAX_NST];       // the MMAs reading a stage finished
@@ -110,6 +113,11 @@ struct SmemCtl {
   int ctok[BM];                  // ... and which,
   int crow[BM][MAX_K];           // ... their k expert rows
   float cgate[BM][MAX_K];        // ... and their k gates (staged once, read by every warp)
+  // side combine warps: bands this CTA completed, waiting for their arrivals (one
+  // writer, the publishing thread; the side warps claim entries with a CAS on bhead)
+  int bring[SIDE_RING];
+  int bhead, btail;
+  int prod_left;                 // producer warps (TMA, MMA, epilogue) still in their roles
   // epilogue: per warp, 32 rows x 32 bf16 columns on their way to global memory
   alignas(16) uint8_t ostage[EPI_WARPS][32 * OSTAGE_ROW];
 };
@@ -947,6 +955,44 @@ __device__ __forceinline__ void publish_band(const FfnArgs& a, int kind, int ban
   red_release_add(kind == K_G1 ? &a.w.band_done1[band] : &a.w.band_done2[band], units);
 }
 
+// The arrivals of a completed band: every row's token gets one more of its k rows
+// (acq_rel, so the rows' stores are seen by whoever sees the count); the row that
+// brings a token to k appends it to the ready queue (st.release of t + 1 into an
+// allocated entry).  Threads lane, lane + nl, ... take the band's rows.
+__device__ void band_arrivals(const FfnArgs& a, int band, int lane, int nl) {
+  const Work& w = a.w;
+  const Band bd = w.bands[band];
+  const int k = a.k;
+  for (int r = lane; r < bd.rows; r += nl) {
+    const int t = w.perm[bd.row0 + r] / k;
+    if (atom_acq_rel_add(&w.arrive[t], 1u) == (uint32_t)(k - 1)) {
+      const uint32_t e = atomicAdd(&w.sync->rq_alloc, 1u);
+      __threadfence();
+      st_release(&w.ready_q[e], (uint32_t)t + 1u);
+    }
+  }
+}
+
+// Publish a stored GEMM2 tile with side combine warps: the counter is bumped with a
+// returning acq_rel atomic, so the CTA whose tile completes the band knows it (and
+// has acquired every other tile's stores); it hands the band to its side warps
+// through the shared-memory ring, or, with the ring full, does the arrivals itself.
+__device__ __forceinline__ void publish_g2_side(const FfnArgs& a, SmemCtl* ctl, int band, uint32_t units) {
+  __threadfence();
+  const uint32_t full = BAND_UNIT * (uint32_t)(a.d / BN2);
+  if (atom_acq_rel_add(&a.w.band_done2[band], units) + units != full) return;
+  volatile int* vt = &ctl->btail;
+  volatile int* vh = &ctl->bhead;
+  const int tl = *vt;
+  if (tl - *vh < SIDE_RING) {
+    ctl->bring[tl % SIDE_RING] = band;
+    __threadfence_block();   // the entry before the tail that exposes it
+    *vt = tl + 1;
+  } else {
+    band_arrivals(a, band, 0, 1);
+  }
+}
+
 // Eight warps per CTA; warp w reads TMEM lanes [32q, 32q+32) with q = w mod 4,
 // i.e. rows 32q.. of each accumulator's 128 rows, and half of the accumulator's
 // columns, hc = (w - 2) / 4.  Stores are masked to the band's valid rows; then
@@ -999,7 +1045,9 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
         for (int b = 0; b < 2; ++b) {
           const bool stored = wait_bar(&ctl->epi_done[b], (eph >> b) & 1u, tmo, abort);
           if (!stored) { set_error(w.status, W_DRAIN); break; }
-          if (it.rows > b * BM) publish_band(a, it.kind, it.band0 + b, BAND_UNIT);
+          if (it.rows <= b * BM) continue;
+          if (a.side && it.kind == K_G2) publish_g2_side(a, ctl, it.band0 + b, BAND_UNIT);
+          else publish_band(a, it.kind, it.band0 + b, BAND_UNIT);
         }
       }
       eph ^= 3u;
@@ -1039,6 +1087,7 @@ __device__ void role_epilogue(const FfnArgs& a, SmemCtl* ctl, uint32_t tmem_base
     if (warp == 2 && lane == 0) {
       const bool stored = wait_bar(&ctl->epi_done[my_acc], (eph >> my_acc) & 1u, tmo, abort);
       if (!stored) set_error(w.status, W_DRAIN);
+      else if (a.side && it.kind == K_G2 && m.rows > 0) publish_g2_side(a, ctl, m.band, BAND_UNIT);
       else if (half || m.rows > 0) publish_band(a, it.kind, m.band, half ? BAND_UNIT / 2 : BAND_UNIT);
     }
     eph ^= 1u << my_acc;
@@ -1089,7 +1138,9 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
   const bool stamp_on = (a.flags & MOE_DBG_TIMESTAMPS) != 0;
   uint64_t idle_since = 0;
   int my_item = -1;                                       // thread 0: band ticket held, not yet processed
-  bool items_left = true;                                 // thread 0: band tickets may remain
+  // thread 0: band tickets may remain (none with side warps: the producers' CTAs
+  // do every band's arrivals)
+  bool items_left = !a.side;
   while (true) {
     // ---- thread 0 decides what to do next.  Band items and queue entries are
     // taken with fetch-and-add tickets (no CAS contention at the tail).  A CTA
@@ -1273,6 +1324,114 @@ __device__ void role_consumer(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, int
     w.stamps[(size_t)blockIdx.x * NSTAMP + 6] = n_bands_done;
 }
 
+// ------------------------------------------------------------ side warps ---
+// MOE_SCHED_SIDE_COMBINE: the consumer work of [TLS] Section 3.3.3 spread over two
+// extra warps in every producer CTA instead of a partition of whole SMs, so that no
+// SM gives up tensor-core time for it.  A side warp repeatedly takes, in this order:
+//  * a band its CTA completed (the ring filled by publish_g2_side): the band's
+//    arrivals, 32 rows at a time;
+//  * up to SIDE_TOK tokens of the ready queue, claimed only where entries are
+//    already allocated (never waiting for future bands): each token is combined
+//    straight from global memory by the warp (the combine kernel's routine, so the
+//    same bits) and flagged TOKEN_DONE;
+// and leaves as soon as its CTA's producer warps have all left their roles.  The CTA then joins the consumer role (without band tickets) if joining
+// is on; the combine pass after the kernel finishes any token left.
+enum : int { S_IDLE = 0, S_BAND = 1, S_COMBINE = 2, S_EXIT = 3, S_RETRY = 4 };
+
+__device__ void role_side(const FfnArgs& a, SmemCtl* ctl, int lane, const volatile uint32_t* abort) {
+  const Work& w = a.w;
+  volatile int* vh = &ctl->bhead;
+  volatile int* vt = &ctl->btail;
+  volatile int* vl = &ctl->prod_left;
+  uint64_t idle_since = 0;
+  uint32_t nap = 64;
+  while (true) {
+    int act = S_IDLE, arg = 0, n = 0;
+    if (lane == 0) {
+      if (*abort) {
+        act = S_EXIT;
+      } else {
+        const int hd = *vh, tl = *vt;
+        if (*vl == 0) {
+          // The CTA's producers are done: leave at once, so that the CTA's exit (and
+          // with the last CTA, the kernel's end) waits for nothing here.  Bands
+          // still in the ring and tokens not combined go to the combine pass.
+          act = S_EXIT;
+        } else if (hd < tl) {
+          __threadfence_block();   // the entry after the tail that exposed it
+          const int b = ctl->bring[hd % SIDE_RING];   // read before the claim frees the slot
+          if (atomicCAS(&ctl->bhead, hd, hd + 1) == hd) { act = S_BAND; arg = b; }
+          else act = S_RETRY;
+        } else {
+          const uint32_t h = ld_relaxed(&w.sync->rq_head);
+          const uint32_t al = ld_relaxed(&w.sync->rq_alloc);
+          if (h < al) {
+            const uint32_t m = min(al - h, (uint32_t)SIDE_TOK);
+            if (atomicCAS(&w.sync->rq_head, h, h + m) == h) { act = S_COMBINE; arg = (int)h; n = (int)m; }
+            else act = S_RETRY;
+          }
+        }
+      }
+      // Idle for long stretches is normal (no band completes during GEMM1); the
+      // producers' own waits are bounded, so their exit ends this loop.  The limit
+      // here is a backstop only.
+      if (act == S_IDLE) {
+        const uint64_t now = globaltimer();
+        if (idle_since == 0) idle_since = now;
+        else if (now - idle_since > 4 * a.timeout_ns) { set_error(w.status, W_SIDE_IDLE); act = S_EXIT; }
+      } else if (act != S_RETRY) {
+        idle_since = 0;
+        nap = 64;
+      }
+    }
+    act = __shfl_sync(0xffffffffu, act, 0);
+    arg = __shfl_sync(0xffffffffu, arg, 0);
+    n = __shfl_sync(0xffffffffu, n, 0);
+    if (act == S_EXIT) break;
+    if (act == S_RETRY) continue;
+    if (act == S_IDLE) {
+      if (lane == 0) {
+        __nanosleep(nap);
+        if (nap < 2048) nap <<= 1;
+      }
+      __syncwarp();
+      continue;
+    }
+    if (act == S_BAND) {
+      __threadfence();   // the publishing thread's acquire of the band's tiles comes first
+      band_arrivals(a, arg, lane, 32);
+      __syncwarp();
+      continue;
+    }
+    // S_COMBINE: queue entries [arg, arg + n), allocated, so written soon if not yet;
+    // a token not reached before the producers are done is left to the combine pass
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      if (i > 0 && *vl == 0) break;
+      uint32_t* q = &w.ready_q[arg + i];
+      int got = 1;
+      if (lane == 0) {
+        uint32_t v = ld_acquire(q);
+        const uint64_t deadline = globaltimer() + a.timeout_ns;
+        while (v == 0u) {
+          if (*abort) { got = 0; break; }
+          if (globaltimer() > deadline) { set_error(w.status, W_SIDE_QUEUE); got = 0; break; }
+          __nanosleep(32);
+          v = ld_acquire(q);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+      if (!ok) break;
+      const int t = (int)ld_acquire(q) - 1;   // every lane: the token's rows are stored before
+      if (a.k <= 4) combine_token_warp_u<4, 3>(a.y, w.row_of, a.gate, t, a.d, a.k, a.out, lane);
+      else combine_token_warp_u<MAX_K, 2>(a.y, w.row_of, a.gate, t, a.d, a.k, a.out, lane);
+      __syncwarp();
+      if (lane == 0) atomicOr(&w.arrive[t], TOKEN_DONE);
+    }
+    if (!ok) break;
+  }
+}
+
 // ------------------------------------------------------------- EP return ---
 // The consumer role of an expert-parallel owner: the return all-to-all of "Fine-
 // grained Computation-Communication Overlap via Tile-level Signaling and
@@ -1351,14 +1510,16 @@ __device__ void role_return(const FfnArgs& a, SmemCtl* ctl, int nb, int n_items,
 }
 
 // ------------------------------------------------------------------- kernel ---
-// GW: extra warps that copy GEMM1's A rows from x (MOE_SCHED_GATHER_LSU), 0 otherwise.
-template <int V, int GW>
-__global__ void __launch_bounds__(FFN_THREADS + 32 * GW, 1)
+// XW: extra warps, 0 or 2: they copy GEMM1's A rows from x (a.gather == 2,
+// MOE_SCHED_GATHER_LSU) or are side combine warps (a.side).
+template <int V, int XW>
+__global__ void __launch_bounds__(FFN_THREADS + 32 * XW, 1)
 ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_w1,
            const __grid_constant__ CUtensorMap tm_w3, const __grid_constant__ CUtensorMap tm_a2,
            const __grid_constant__ CUtensorMap tm_w2, const FfnArgs a) {
-  constexpr int NTHREADS = FFN_THREADS + 32 * GW;
-  constexpr int GW0 = FFN_THREADS / 32;         // first gather warp
+  constexpr int GW0 = FFN_THREADS / 32;         // first extra warp
+  const int GW = (XW > 0 && a.gather == 2) ? XW : 0;   // gather warps
+  const bool side = XW > 0 && a.side != 0 && a.gather != 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + (size_t)STAGE_AREA);
@@ -1383,7 +1544,10 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
     mbar_init(&ctl->mma_done, 1);
     mbar_init(&ctl->gbar[0], 1);
     mbar_init(&ctl->gbar[1], 1);
-    for (int i = 0; i < CONS_SLOTS; ++i) { mbar_init(&ctl->cfull[i], 1); mbar_init(&ctl->cempty[i], NTHREADS / 32 - 1); }
+    for (int i = 0; i < CONS_SLOTS; ++i) { mbar_init(&ctl->cfull[i], 1); mbar_init(&ctl->cempty[i], (int)(blockDim.x / 32) - 1); }
+    ctl->bhead = 0;
+    ctl->btail = 0;
+    ctl->prod_left = GW0;
     mbar_fence_init();
     fence_proxy_async_shared();
   }
@@ -1441,10 +1605,15 @@ ffn_kernel(const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CU
       if (lane == 0 && rank == 0) role_mma<V>(a, ctl, smem, tmem_base, abort);
     } else if (warp < GW0) {
       role_epilogue<V>(a, ctl, tmem_base, rank, warp, lane, abort);
-    } else {
-      if constexpr (GW > 0 && V != 2) role_gather_lsu<V, GW>(a, ctl, smem, warp - GW0, lane, abort);
+    } else if constexpr (XW > 0 && V != 2) {
+      if (GW > 0) role_gather_lsu<V, XW>(a, ctl, smem, warp - GW0, lane, abort);
+      else if (side) role_side(a, ctl, lane, abort);
     }
     __syncwarp();
+    if (side && warp < GW0 && lane == 0) {
+      __threadfence_block();   // this warp's ring entries before its exit
+      atomicSub(&ctl->prod_left, 1);
+    }
   }
   __syncthreads();
   if (stamp && threadIdx.x == 0) my_stamps[2] = globaltimer();
@@ -1510,8 +1679,8 @@ static bool encode4(CUtensorMap* m, const void* base, const cuuint64_t* dims,
 
 namespace {
 constexpr int MAX_DEV = 64;
-constexpr int LSU_GW = 2;   // gather warps of the MOE_SCHED_GATHER_LSU kernels
-// index of (V, with gather warps): 0-2 plain V = 1..3, 3 V = 1 + GW, 4 V = 3 + GW
+constexpr int XW_WARPS = 2;   // extra warps: gather (MOE_SCHED_GATHER_LSU) or side combine
+// index of (V, with extra warps): 0-2 plain V = 1..3, 3 V = 1 + XW, 4 V = 3 + XW
 int g_configured[5][MAX_DEV] = {{0}};
 int g_grid[5][MAX_DEV] = {{0}};
 
@@ -1555,9 +1724,9 @@ cudaError_t configure(int dev) {
 
 cudaError_t configure_variant(int V, int gw, int dev) {
   if (gw) {
-    if (V == 1) return configure<1, LSU_GW>(dev);
-    if (V == 3) return configure<3, LSU_GW>(dev);
-    return cudaErrorInvalidValue;   // CTA pairs have no gather-warp kernel
+    if (V == 1) return configure<1, XW_WARPS>(dev);
+    if (V == 3) return configure<3, XW_WARPS>(dev);
+    return cudaErrorInvalidValue;   // CTA pairs have no extra-warp kernel
   }
   switch (V) {
     case 1: return configure<1, 0>(dev);
@@ -1583,7 +1752,8 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const int gw = a.gather == 2 ? LSU_GW : 0;
+  const int gw = (a.gather == 2 || a.side) ? XW_WARPS : 0;
+  if (gw && a.V == 2) return cudaErrorInvalidValue;   // CTA pairs have no extra-warp kernel
   e = configure_variant(a.V, gw, dev);
   if (e != cudaSuccess) return e;
   CUtensorMap tm_a1, tm_w1, tm_w3, tm_a2, tm_w2;
@@ -1643,8 +1813,8 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   }
   cfg.attrs = attr;
   if (gw) {
-    if (a.V == 3) return cudaLaunchKernelEx(&cfg, ffn_kernel<3, LSU_GW>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
-    return cudaLaunchKernelEx(&cfg, ffn_kernel<1, LSU_GW>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+    if (a.V == 3) return cudaLaunchKernelEx(&cfg, ffn_kernel<3, XW_WARPS>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
+    return cudaLaunchKernelEx(&cfg, ffn_kernel<1, XW_WARPS>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
   }
   if (a.V == 2) return cudaLaunchKernelEx(&cfg, ffn_kernel<2, 0>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);
   if (a.V == 3) return cudaLaunchKernelEx(&cfg, ffn_kernel<3, 0>, tm_a1, tm_w1, tm_w3, tm_a2, tm_w2, args);

@@ -95,6 +95,10 @@ struct FfnArgs {
                                  // 256-row tile (cta_group::2), 3 one CTA per 256-row tile
   int phase;                     // PH_* bits
   int join;                      // producers join the combine when the tile queue drains
+  int side;                      // side combine warps (MOE_SCHED_SIDE_COMBINE, single CTAs):
+                                 // the CTA whose GEMM2 tile completes a band hands the band's
+                                 // arrivals to two extra warps, which also combine ready
+                                 // tokens while the tiles run; consumers take no band tickets
   int mgb;
   int b_atoms;                   // single CTA: weight maps are 4-D, one box carries all 64-column atoms
   uint32_t flags;

@@ -295,7 +295,7 @@ __device__ void plan_tables(const Work& w, int U, const int* cnt, const int* row
   __shared__ int c_pick;
   if (warp == 0) {
     const int cmin = cg;   // at least one dedicated consumer group (measured: see choose_consumers)
-    const int C = consumer_hint > 0 ? consumer_hint : choose_consumers(num_sms, cg, cmin, R, T, d, f, cm, lane);
+    const int C = consumer_hint != 0 ? consumer_hint : choose_consumers(num_sms, cg, cmin, R, T, d, f, cm, lane);
     if (lane == 0) c_pick = C;
   }
   for (int i = tid; i < (int)(sizeof(Sync) / 4); i += blockDim.x) reinterpret_cast<uint32_t*>(w.sync)[i] = 0u;
@@ -303,8 +303,12 @@ __device__ void plan_tables(const Work& w, int U, const int* cnt, const int* row
   if (tid == 0) {
     const int cmin = cg;
     int C = c_pick;
-    C = cg * cdiv(C, cg);                       // consumers come in whole CTA groups
-    C = max(cmin, min(C, num_sms - cg));        // and leave at least one producer group
+    if (C < 0) {
+      C = 0;                                    // no dedicated consumers (side combine warps)
+    } else {
+      C = cg * cdiv(C, cg);                     // consumers come in whole CTA groups
+      C = max(cmin, min(C, num_sms - cg));      // and leave at least one producer group
+    }
     Status st;
     st.code = code;
     st.consumer_sms = C;

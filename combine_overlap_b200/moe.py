@@ -37,6 +37,7 @@ SCHED_WIDE_CTA = 0x100
 DBG_IDENTITY_EXPERTS = 0x200
 SCHED_INTERLEAVE = 0x400
 SCHED_EVICT_FIRST = 0x800
+SCHED_SIDE_COMBINE = 0x1000
 SCHED_EXP_SILU = 0x4000
 SCHED_GATHER_LSU = 0x8000
 
@@ -104,6 +105,8 @@ _lib.moe_debug_stamps.argtypes = [_P, _P, _P, _I, ctypes.POINTER(_I)]
 _lib.moe_debug_stamps.restype = _I
 _lib.moe_debug_band_stamps.argtypes = [_P, _P, _P, _I]
 _lib.moe_debug_band_stamps.restype = _I
+_lib.moe_debug_tokens_combined.argtypes = [_P, _I, _I, _I, _I, _I, _P, ctypes.POINTER(_I)]
+_lib.moe_debug_tokens_combined.restype = _I
 _lib.moe_permute_noalloc.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
 _lib.moe_permute_noalloc.restype = _I
 _lib.moe_permute_noalloc_scratch_bytes.restype = _S
@@ -379,6 +382,15 @@ def debug_band_stamps(ws: torch.Tensor, n_bands: int, stream=None):
     _check(_lib.moe_debug_band_stamps(_ptr(ws), _stream(stream), out.ctypes.data_as(ctypes.c_void_p), n),
            "moe_debug_band_stamps")
     return out
+
+
+def debug_tokens_combined(ws: torch.Tensor, T: int, d: int, f: int, E: int, k: int, stream=None) -> int:
+    """Tokens of the last overlapped call on ws (this shape) that the persistent
+    kernel combined itself; the combine pass after it did the rest."""
+    n = ctypes.c_int(0)
+    _check(_lib.moe_debug_tokens_combined(_ptr(ws), T, d, f, E, k, _stream(stream), ctypes.byref(n)),
+           "moe_debug_tokens_combined")
+    return int(n.value)
 
 
 class MoELayer:

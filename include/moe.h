@@ -117,6 +117,15 @@ typedef enum {
                                         swizzled operand layout (x_perm is not written);
                                         the TMA loads the weights only.  Same bits.  With
                                         CTA pairs: MOE_ERR_UNSUPPORTED */
+#define MOE_SCHED_SIDE_COMBINE 0x1000u /* overlapped mode, single-CTA tiles: two extra
+                                        warps in every producer CTA do the combine while
+                                        the tiles run -- the CTA whose GEMM2 tile
+                                        completes a row band hands them its arrivals,
+                                        and they combine ready tokens from global
+                                        memory -- and no SM is a dedicated consumer
+                                        unless consumer_sms asks for some.  Same bits.
+                                        With CTA pairs: no effect.  With
+                                        MOE_SCHED_GATHER_LSU: MOE_ERR_UNSUPPORTED */
 #define MOE_SCHED_EVICT_FIRST  0x800u /* the epilogue stores h and y with an L2
                                         evict-first policy (they compete with the weights
                                         for L2).  Same bits */
@@ -338,6 +347,13 @@ moe_status moe_debug_stamps(void* ws, void* stream, uint64_t* host_out, int max_
  * [0] band ready (globaltimer ns), [1] band combined, [2] tokens it completed,
  * [3] consuming CTA.  host_out must hold max_bands x 4 values. */
 moe_status moe_debug_band_stamps(void* ws, void* stream, uint64_t* host_out, int max_bands);
+
+/* Debug aid: synchronises `stream` and sets *n_combined to the number of tokens of
+ * the last overlapped layer call on `ws` (shape T, d, f, E, k as in that call) that
+ * the persistent kernel combined itself -- the rest were left to the combine pass
+ * after it.  Reads T arrival words from the workspace. */
+moe_status moe_debug_tokens_combined(const void* ws, int T, int d, int f, int E, int k, void* stream,
+                                     int* n_combined);
 
 /* Static English description of a status code. */
 const char* moe_status_string(moe_status s);

@@ -71,6 +71,8 @@ def test_layer_small(orc, wl):
             outI, _, _ = _forward(inp, wl, ws, mode, flags=moe.DBG_IDENTITY_EXPERTS)
             gu.assert_combine_close(gu.host(outI), refI["out"], what=f"tiny identity experts {mode}")
     seq, extra, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL, flags=pair)
+    # the sequential mode combines after the FFN only: no token combined in-kernel
+    assert moe.debug_tokens_combined(ws, wl.T, wl.d, wl.f, wl.E, wl.k) == 0
     assert np.array_equal(gu.host(extra["topk_idx"]), ref["topk_idx"])
     gu.assert_gates(gu.host(extra["topk_gate"]), ref["topk_gate"])
     assert np.array_equal(gu.host(extra["counts"]), ref["counts"])
@@ -121,6 +123,21 @@ def test_layer_small(orc, wl):
         gat, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=fl)
         base = seq_bits if fl & pair else gu.host(seq1)
         assert np.array_equal(gu.host(gat), base), f"flags {fl:#x} differ"
+    # side combine warps: the producers' CTAs do the arrivals and combine ready
+    # tokens while the tiles run (no dedicated consumer unless asked for), with
+    # or without joining, interleaved or not; CTA pairs ignore the flag.  Same bits.
+    side = moe.SCHED_SIDE_COMBINE
+    for fl, kw in ((side | one, dict()), (side | wide, dict()), (side, dict()),
+                   (side | wide | moe.SCHED_INTERLEAVE, dict()), (side | one | moe.SCHED_INTERLEAVE, dict()),
+                   (side | wide, dict(consumer_sms=2)), (side | one | moe.SCHED_NO_JOIN, dict()),
+                   (side | wide | moe.SCHED_NO_JOIN | moe.SCHED_INTERLEAVE, dict(consumer_sms=3)),
+                   (side | wide, dict(mgb=2)), (side | pair, dict())):
+        sd, _, c = _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=fl, **kw)
+        assert 0 <= moe.debug_tokens_combined(ws, wl.T, wl.d, wl.f, wl.E, wl.k) <= wl.T
+        base = seq_bits if fl & pair else gu.host(seq1)
+        assert np.array_equal(gu.host(sd), base), f"side combine flags {fl:#x} {kw} differ"
+        if not fl & pair:
+            assert c == kw.get("consumer_sms", 0)
     # SiLU in its exp form (the default uses the hardware tanh): other bits in h,
     # the same bound against the oracle, and the same bits in every mode and tile
     # variant
@@ -151,14 +168,15 @@ FULL = ["mixtral", "fine_grained", "imbalanced"] + \
 # tiles from 256 rows per expert up, 128-row tiles below), and the other variants
 # on a few
 FULL_CASES = [(n, 0) for n in FULL] + [("mixtral", 0x4), ("mixtral", 0x20), ("fine_grained", 0x20),
-                                        ("sweep_T512_hot", 0x100)]
+                                        ("sweep_T512_hot", 0x100)] + \
+    [(n, 0x1000) for n in ("mixtral", "fine_grained", "imbalanced", "sweep_T2048_uniform",
+                           "sweep_T32768_uniform", "sweep_T512_zipf")]
+_FLAG_IDS = {0: "default", 0x4: "one", 0x20: "pair", 0x100: "wide", 0x1000: "side"}
 
 
-@pytest.mark.parametrize("name,flags", FULL_CASES,
-                         ids=[f"{n}-{ {0: 'default', 0x4: 'one', 0x20: 'pair', 0x100: 'wide'}[f]}"
-                              for n, f in FULL_CASES])
+@pytest.mark.parametrize("name,flags", FULL_CASES, ids=[f"{n}-{_FLAG_IDS[f]}" for n, f in FULL_CASES])
 def test_layer_full_size_sampled(orc, name, flags):
-    assert flags in (0, moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR, moe.SCHED_WIDE_CTA)
+    assert flags in (0, moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR, moe.SCHED_WIDE_CTA, moe.SCHED_SIDE_COMBINE)
     wl = synth.WORKLOADS[name]
     orc.set_threads(os.cpu_count() or 1)
     inp = gu.inputs(wl)
@@ -246,6 +264,10 @@ def test_gather_lsu_refuses_cta_pairs():
     ws = moe.alloc_workspace(wl.T, wl.d, wl.f, wl.E, wl.k)
     with pytest.raises(moe.MoEError) as e:
         _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=moe.SCHED_GATHER_LSU | moe.SCHED_CTA_PAIR)
+    assert e.value.code == moe.MOE_ERR_UNSUPPORTED
+    # ... and the side combine warps are the same extra warps: not both
+    with pytest.raises(moe.MoEError) as e:
+        _forward(inp, wl, ws, moe.MODE_OVERLAPPED, flags=moe.SCHED_GATHER_LSU | moe.SCHED_SIDE_COMBINE)
     assert e.value.code == moe.MOE_ERR_UNSUPPORTED
 
 
