@@ -12,7 +12,8 @@ namespace moe {
 
 // ---------------------------------------------------------------- tiling ---
 constexpr int BM = 128;         // rows per row band (= MMA M, = TMEM lanes)
-constexpr int BK = 64;          // K elements per pipeline stage (128 B of bf16)
+constexpr int BK = 64;          // K elements per pipeline stage (128 B of bf16; 256-row
+                                // single-CTA tiles use 32, see Cfg in ffn.cu)
 constexpr int BN1 = 128;        // h columns per GEMM1 tile (accumulates W1 and W3: 256 TMEM cols)
 constexpr int BN2 = 256;        // y columns per GEMM2 tile
 constexpr int NSTAGE = 4;       // smem pipeline depth
@@ -460,6 +461,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;                 // descriptor version for tcgen05
   d |= (uint64_t)2 << 61;                 // SWIZZLE_128B
+  return d;
+}
+
+// The same with 64-byte swizzle: a K-major tile of 64-byte rows (32 bf16 of K),
+// 8-row atoms `sbo` = 512 bytes apart; lbo unused.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;                 // descriptor version for tcgen05
+  d |= (uint64_t)4 << 61;                 // SWIZZLE_64B
   return d;
 }
 

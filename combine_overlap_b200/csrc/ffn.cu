@@ -68,6 +68,11 @@ constexpr int STAGE_AREA = 196608;  // shared memory of the operand ring (and th
 //   V = 3  one CTA per 256x256 tile, as two 128-row MMAs (two A boxes, one B
 //          stage) into its two accumulators.
 // V = 2 and V = 3 stream 32 KB of operands per 128x256x64 of MMA work, V = 1 48 KB.
+// A stage holds BK = 64 elements of K: A rows of 128 bytes in the 128-byte swizzle.
+// (The roles also take BK = 32 -- 64-byte A rows in the 64-byte swizzle -- which
+// gives V = 3 six stages of 32 KB instead of three of 64 KB.  Measured on B200 it
+// was 10-12 % slower on every V = 3 layer, and a V = 3 ring of two 64 KB stages
+// 16-22 % slower than three, so three stages of 64 KB it is.)
 template <int V>
 struct Cfg {
   static_assert(V >= 1 && V <= 3, "tile variant");
@@ -75,9 +80,14 @@ struct Cfg {
   static constexpr int BANDS = V == 1 ? 1 : 2;                     // row bands per tile
   static constexpr int ABOX = V == 3 ? 2 : 1;                      // 128-row A boxes per CTA
   static constexpr int NBOX = V == 2 ? 2 : 4;                      // 64-column B boxes per CTA
-  static constexpr int STAGE = ABOX * A_STAGE_BYTES + NBOX * B_BOX_BYTES;
+  static constexpr int BK = 64;                                    // K elements per stage
+  static constexpr int A_ROW = BK * 2;                             // bytes of an A row (swizzle span)
+  static constexpr int A_BYTES = BM * A_ROW;                       // one 128-row A box
+  static constexpr int B_BOX = BK * 64 * 2;                        // one 64-column B atom
+  static constexpr int STAGE = ABOX * A_BYTES + NBOX * B_BOX;
   static constexpr int NST = STAGE_AREA / STAGE;
   static_assert(NST <= MAX_NST && NST * STAGE == STAGE_AREA, "stage ring must fill the area");
+  static_assert(BK % 16 == 0 && (A_ROW == 64 || A_ROW == 128), "A rows of one swizzle span");
 };
 
 // 16-byte aligned: the pair leader copies items into its peer's ring with 16-byte
@@ -130,7 +140,7 @@ static_assert(1024 + STAGE_AREA + sizeof(SmemCtl) <= 227 * 1024, "over the 227 K
 
 // Weight-tile bytes of one stage of variant V (the whole B share of a CTA).
 template <int V>
-__device__ __forceinline__ constexpr int NBOX_BYTES() { return Cfg<V>::NBOX * B_BOX_BYTES; }
+__device__ __forceinline__ constexpr int NBOX_BYTES() { return Cfg<V>::NBOX * Cfg<V>::B_BOX; }
 
 __device__ __forceinline__ void set_error(Status* st, uint32_t where) {
   if (atomicCAS(&st->code, (uint32_t)ST_OK, (uint32_t)ST_TIMEOUT) == (uint32_t)ST_OK) {
@@ -446,11 +456,11 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
       }
       fence_proxy_async_global();  // generic-proxy stores -> async-proxy (TMA) loads
     }
-    const int nk = (is1 ? a.d : a.f) / BK;
+    const int nk = (is1 ? a.d : a.f) / C::BK;
     for (int kb = 0; kb < nk; ++kb) {
       if (!wait_bar<V == 2>(&ctl->empty[stage], ph ^ 1u, tmo, abort)) { set_error(w.status, W_STAGE_EMPTY); ok = false; break; }
       uint8_t* sa = smem + (size_t)stage * C::STAGE;
-      uint8_t* sb = sa + C::ABOX * A_STAGE_BYTES;
+      uint8_t* sb = sa + C::ABOX * C::A_BYTES;
       uint64_t* fb = &ctl->full[stage];
       const uint32_t fbl = V == 2 ? mapa_shared(smem_u32(fb), 0) : 0u;
       // a pair's leader expects both CTAs' bytes; V = 3 without a second band
@@ -458,7 +468,7 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
       const bool lsu = is1 && a.gather == 2;
       if (leader)
         mbar_arrive_expect_tx(fb, lsu ? NBOX_BYTES<V>() :
-                                  C::CTAS * C::STAGE - (V == 3 && !two ? A_STAGE_BYTES : 0));
+                                  C::CTAS * C::STAGE - (V == 3 && !two ? C::A_BYTES : 0));
       // A: 128 rows x 64 columns of x_perm (tiled) or of x (gathered); h for GEMM2
       if (lsu) {
         // (the gather warps copy these A rows)
@@ -466,36 +476,36 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
 #pragma unroll 8
         for (int q = 0; q < BM / 4; ++q) {
           const int4 tk = m.rows > 0 ? ctl->gidx[buf][q] : make_int4(0, 0, 0, 0);
-          if (V != 2) tma_gather4(sa + q * 512, tm_a1, fb, kb * BK, tk.x, tk.y, tk.z, tk.w);
-          else tma_gather4_pair(sa + q * 512, tm_a1, fbl, kb * BK, tk.x, tk.y, tk.z, tk.w);
+          if (V != 2) tma_gather4(sa + q * 4 * C::A_ROW, tm_a1, fb, kb * C::BK, tk.x, tk.y, tk.z, tk.w);
+          else tma_gather4_pair(sa + q * 4 * C::A_ROW, tm_a1, fbl, kb * C::BK, tk.x, tk.y, tk.z, tk.w);
         }
       } else if (V != 2) {
-        tma_load_2d(sa, is1 ? tm_a1 : tm_a2, fb, kb * BK, m.row0);
-        if (two) tma_load_2d(sa + A_STAGE_BYTES, is1 ? tm_a1 : tm_a2, fb, kb * BK, m.row0 + BM);
+        tma_load_2d(sa, is1 ? tm_a1 : tm_a2, fb, kb * C::BK, m.row0);
+        if (two) tma_load_2d(sa + C::A_BYTES, is1 ? tm_a1 : tm_a2, fb, kb * C::BK, m.row0 + BM);
       } else {
-        tma_load_2d_pair(sa, is1 ? tm_a1 : tm_a2, fbl, kb * BK, m.row0);
+        tma_load_2d_pair(sa, is1 ? tm_a1 : tm_a2, fbl, kb * C::BK, m.row0);
       }
-      // B: 64-column atoms of W1/W3 (GEMM1) or W2 (GEMM2), K-rows kb*BK.., each
-      // atom 64 K rows x 128 B, atom after atom (the MMA's leading-byte offset)
+      // B: 64-column atoms of W1/W3 (GEMM1) or W2 (GEMM2), K-rows kb*C::BK.., each
+      // atom BK K rows x 128 B, atom after atom (the MMA's leading-byte offset)
       if (V != 2 && a.b_atoms) {
         // 4-D maps {64 columns, K, atom, expert}: one copy per operand
-        const int k0 = kb * BK;
+        const int k0 = kb * C::BK;
         if (is1) {
           tma_load_4d(sb, tm_w1, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
-          tma_load_4d(sb + 2 * B_BOX_BYTES, tm_w3, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
+          tma_load_4d(sb + 2 * C::B_BOX, tm_w3, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
         } else {
           tma_load_4d(sb, tm_w2, fb, 0, k0, cur.nt * (BN2 / 64), cur.expert);
         }
       } else if (V != 2) {
         if (is1) {
-          tma_load_3d(sb, tm_w1, fb, cur.nt * BN1, kb * BK, cur.expert);
-          tma_load_3d(sb + B_BOX_BYTES, tm_w1, fb, cur.nt * BN1 + 64, kb * BK, cur.expert);
-          tma_load_3d(sb + 2 * B_BOX_BYTES, tm_w3, fb, cur.nt * BN1, kb * BK, cur.expert);
-          tma_load_3d(sb + 3 * B_BOX_BYTES, tm_w3, fb, cur.nt * BN1 + 64, kb * BK, cur.expert);
+          tma_load_3d(sb, tm_w1, fb, cur.nt * BN1, kb * C::BK, cur.expert);
+          tma_load_3d(sb + C::B_BOX, tm_w1, fb, cur.nt * BN1 + 64, kb * C::BK, cur.expert);
+          tma_load_3d(sb + 2 * C::B_BOX, tm_w3, fb, cur.nt * BN1, kb * C::BK, cur.expert);
+          tma_load_3d(sb + 3 * C::B_BOX, tm_w3, fb, cur.nt * BN1 + 64, kb * C::BK, cur.expert);
         } else {
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            tma_load_3d(sb + q * B_BOX_BYTES, tm_w2, fb, cur.nt * BN2 + q * 64, kb * BK, cur.expert);
+            tma_load_3d(sb + q * C::B_BOX, tm_w2, fb, cur.nt * BN2 + q * 64, kb * C::BK, cur.expert);
         }
       } else {
         if (is1 && half) {
@@ -503,17 +513,17 @@ __device__ void role_tma(const CUtensorMap* tm_a1, const CUtensorMap* tm_w1,
           // leader's the first, the peer's the second), so every accumulator
           // lane holds matching W1 and W3 columns
           const int n0 = cur.nt * BN1 + (int)rank * 64;
-          tma_load_3d_pair(sb, tm_w1, fbl, n0, kb * BK, cur.expert);
-          tma_load_3d_pair(sb + B_BOX_BYTES, tm_w3, fbl, n0, kb * BK, cur.expert);
+          tma_load_3d_pair(sb, tm_w1, fbl, n0, kb * C::BK, cur.expert);
+          tma_load_3d_pair(sb + C::B_BOX, tm_w3, fbl, n0, kb * C::BK, cur.expert);
         } else if (is1) {
           // B columns [0,128) of the N=256 MMA come from the leader (W1), [128,256) from the peer (W3)
           const CUtensorMap* tw = rank == 0 ? tm_w1 : tm_w3;
-          tma_load_3d_pair(sb, tw, fbl, cur.nt * BN1, kb * BK, cur.expert);
-          tma_load_3d_pair(sb + B_BOX_BYTES, tw, fbl, cur.nt * BN1 + 64, kb * BK, cur.expert);
+          tma_load_3d_pair(sb, tw, fbl, cur.nt * BN1, kb * C::BK, cur.expert);
+          tma_load_3d_pair(sb + C::B_BOX, tw, fbl, cur.nt * BN1 + 64, kb * C::BK, cur.expert);
         } else {
           const int n0 = cur.nt * BN2 + (int)rank * 128;
-          tma_load_3d_pair(sb, tm_w2, fbl, n0, kb * BK, cur.expert);
-          tma_load_3d_pair(sb + B_BOX_BYTES, tm_w2, fbl, n0 + 64, kb * BK, cur.expert);
+          tma_load_3d_pair(sb, tm_w2, fbl, n0, kb * C::BK, cur.expert);
+          tma_load_3d_pair(sb + C::B_BOX, tm_w2, fbl, n0 + 64, kb * C::BK, cur.expert);
         }
       }
       pending |= 1u << stage;
@@ -628,46 +638,46 @@ __device__ void role_tma_gathered(const CUtensorMap* tm_a1, const CUtensorMap* t
     int4 tk[2] = {make_int4(0, 0, 0, 0), make_int4(0, 0, 0, 0)};
     if (is1)
       for (int b = 0; b < nb; ++b) tk[b] = ctl->gidx[buf][b * (BM / 4) + lane];
-    const int nk = (is1 ? a.d : a.f) / BK;
+    const int nk = (is1 ? a.d : a.f) / C::BK;
     for (int kb = 0; kb < nk; ++kb) {
       int oks = 1;
       if (lane == 0) {
         oks = wait_bar(&ctl->empty[stage], ph ^ 1u, tmo, abort) ? 1 : 0;
-        if (oks) mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE - (nb < 2 ? (C::ABOX - 1) * A_STAGE_BYTES : 0));
+        if (oks) mbar_arrive_expect_tx(&ctl->full[stage], C::STAGE - (nb < 2 ? (C::ABOX - 1) * C::A_BYTES : 0));
         else set_error(w.status, W_STAGE_EMPTY);
       }
       oks = __shfl_sync(0xffffffffu, oks, 0);   // (a warp shuffle orders lane 0's expect first)
       if (!oks) { ok = false; break; }
       uint8_t* sa = smem + (size_t)stage * C::STAGE;
-      uint8_t* sb = sa + C::ABOX * A_STAGE_BYTES;
+      uint8_t* sb = sa + C::ABOX * C::A_BYTES;
       uint64_t* fb = &ctl->full[stage];
       if (is1) {
         for (int b = 0; b < nb; ++b)
-          tma_gather4(sa + b * A_STAGE_BYTES + lane * 512, tm_a1, fb, kb * BK, tk[b].x, tk[b].y,
+          tma_gather4(sa + b * C::A_BYTES + lane * 4 * C::A_ROW, tm_a1, fb, kb * C::BK, tk[b].x, tk[b].y,
                       tk[b].z, tk[b].w);
       }
       if (lane == 0) {
         if (!is1) {
-          tma_load_2d(sa, tm_a2, fb, kb * BK, cur.row0);
-          if (nb == 2) tma_load_2d(sa + A_STAGE_BYTES, tm_a2, fb, kb * BK, cur.row0 + BM);
+          tma_load_2d(sa, tm_a2, fb, kb * C::BK, cur.row0);
+          if (nb == 2) tma_load_2d(sa + C::A_BYTES, tm_a2, fb, kb * C::BK, cur.row0 + BM);
         }
-        const int k0 = kb * BK;
+        const int k0 = kb * C::BK;
         if (a.b_atoms) {
           if (is1) {
             tma_load_4d(sb, tm_w1, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
-            tma_load_4d(sb + 2 * B_BOX_BYTES, tm_w3, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
+            tma_load_4d(sb + 2 * C::B_BOX, tm_w3, fb, 0, k0, cur.nt * (BN1 / 64), cur.expert);
           } else {
             tma_load_4d(sb, tm_w2, fb, 0, k0, cur.nt * (BN2 / 64), cur.expert);
           }
         } else if (is1) {
           tma_load_3d(sb, tm_w1, fb, cur.nt * BN1, k0, cur.expert);
-          tma_load_3d(sb + B_BOX_BYTES, tm_w1, fb, cur.nt * BN1 + 64, k0, cur.expert);
-          tma_load_3d(sb + 2 * B_BOX_BYTES, tm_w3, fb, cur.nt * BN1, k0, cur.expert);
-          tma_load_3d(sb + 3 * B_BOX_BYTES, tm_w3, fb, cur.nt * BN1 + 64, k0, cur.expert);
+          tma_load_3d(sb + C::B_BOX, tm_w1, fb, cur.nt * BN1 + 64, k0, cur.expert);
+          tma_load_3d(sb + 2 * C::B_BOX, tm_w3, fb, cur.nt * BN1, k0, cur.expert);
+          tma_load_3d(sb + 3 * C::B_BOX, tm_w3, fb, cur.nt * BN1 + 64, k0, cur.expert);
         } else {
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            tma_load_3d(sb + q * B_BOX_BYTES, tm_w2, fb, cur.nt * BN2 + q * 64, k0, cur.expert);
+            tma_load_3d(sb + q * C::B_BOX, tm_w2, fb, cur.nt * BN2 + q * 64, k0, cur.expert);
         }
         pending |= 1u << stage;
         pend_par = (pend_par & ~(1u << stage)) | (ph << stage);
@@ -697,11 +707,12 @@ __device__ void role_tma_gathered(const CUtensorMap* tm_a1, const CUtensorMap* t
 
 // ------------------------------------------- GEMM1 A rows, load/store path ---
 // MOE_SCHED_GATHER_LSU (single CTAs): GW extra warps copy every GEMM1 k-block's
-// A rows straight from x into the stage with 16-byte cp.async, in the 128-byte-
-// swizzled layout a tiled TMA load gives -- chunk c of row r at r*128 +
-// ((c ^ (r & 7)) << 4) -- so x_perm is never written and the TMA thread loads the
-// weights only.  Thread t copies chunk t % 8 of rows t / 8, t / 8 + NT / 8, ...
-// (each warp instruction: 4 rows of 128 contiguous bytes on both sides).  The
+// A rows straight from x into the stage with 16-byte cp.async, in the swizzled
+// layout a tiled TMA load gives -- rows of A_ROW bytes (CPR 16-byte chunks), chunk
+// c of row r at r*A_ROW + ((c ^ ((r*A_ROW >> 7) & (CPR-1))) << 4), the 128- or
+// 64-byte swizzle -- so x_perm is never written and the TMA thread loads the
+// weights only.  Thread t copies chunk t % CPR of rows t / CPR, t / CPR + NT / CPR,
+// ... (each warp instruction: 32 / CPR rows of A_ROW contiguous bytes).  The
 // warps walk the item ring like the MMA and epilogue warps; for every k-block of
 // every item each thread waits (through lane 0) for the stage to be free, issues
 // its copies (GEMM1 only: GEMM2's A rows come by TMA) and arrives on the stage's
@@ -716,10 +727,11 @@ __device__ void role_gather_lsu(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, i
   const Work& w = a.w;
   const uint64_t tmo = a.timeout_ns;
   constexpr int NT = GW * 32;                  // copying threads
-  constexpr int RSTEP = NT / 8;                // rows per pass of all threads
+  constexpr int CPR = C::A_ROW / 16;           // 16-byte chunks per A row
+  constexpr int RSTEP = NT / CPR;              // rows per pass of all threads
   constexpr int ROWS = C::ABOX * BM;           // A rows of a k-block
   const int gt = gw * 32 + lane;
-  const int c = gt & 7;
+  const int c = gt % CPR;
   const size_t row_bytes = (size_t)a.d * 2;
   const char* x = reinterpret_cast<const char*>(a.x);
   int slot = 0, stage = 0;
@@ -736,7 +748,7 @@ __device__ void role_gather_lsu(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, i
     if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
     if (it.kind == K_END) break;
     const bool is1 = it.kind == K_G1;
-    const int nk = (is1 ? a.d : a.f) / BK;
+    const int nk = (is1 ? a.d : a.f) / C::BK;
     // rows to copy: the group's bands (V = 3 without a second band: the first 128)
     const int nrows = (V == 3 && it.rows > BM) ? 2 * BM : BM;
     const int32_t* tok = a.tok_band + (size_t)it.band0 * BM;   // 0 past the bands' rows
@@ -751,12 +763,13 @@ __device__ void role_gather_lsu(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, i
       }
       if (is1) {
         uint8_t* sa = smem + (size_t)stage * C::STAGE;
-        const size_t col = (size_t)kb * BK * 2 + (size_t)c * 16;
+        const size_t col = (size_t)kb * C::BK * 2 + (size_t)c * 16;
 #pragma unroll 4
-        for (int r = gt >> 3; r < ROWS; r += RSTEP) {
+        for (int r = gt / CPR; r < ROWS; r += RSTEP) {
           if (r >= nrows) break;
           const int t = __ldg(tok + r);
-          cp_async16(sa + r * 128 + ((c ^ (r & 7)) << 4), x + (size_t)t * row_bytes + col);
+          const int sw = ((r * C::A_ROW) >> 7) & (CPR - 1);
+          cp_async16(sa + r * C::A_ROW + ((c ^ sw) << 4), x + (size_t)t * row_bytes + col);
         }
         cp_async_arrive_noinc(&ctl->full[stage]);   // arrives when these copies landed
       } else {
@@ -769,6 +782,15 @@ __device__ void role_gather_lsu(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, i
 }
 
 // --------------------------------------------------------------- MMA issuer ---
+// MMA descriptor of an A box at `saddr` (plus the K offset of the MMA step): K-major
+// rows of A_ROW bytes in the matching swizzle, 8-row atoms 8 * A_ROW bytes apart.
+// B (MN-major) is always 128-byte K rows, 64-column atoms B_BOX bytes apart.
+template <int V>
+__device__ __forceinline__ uint64_t a_desc(uint32_t saddr) {
+  if constexpr (Cfg<V>::A_ROW == 64) return smem_desc_sw64(saddr, 16, 8 * 64);
+  else return smem_desc_sw128(saddr, 16, 8 * 128);
+}
+
 // One thread (a single CTA's, or the pair leader's) issues every MMA.
 // V = 1, 2: one accumulator per tile, alternating, so the epilogue of tile i
 // overlaps the main loop of tile i+1.  V = 3: both accumulators per tile, acc b
@@ -790,19 +812,19 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
     mbar_arrive(&ctl->sempty[slot]);
     if (++slot == SCHED_DEPTH) { slot = 0; sph ^= 1u; }
     if (it.kind == K_END) break;
-    const int nk = (it.kind == K_G1 ? a.d : a.f) / BK;
+    const int nk = (it.kind == K_G1 ? a.d : a.f) / C::BK;
     bool ok = true;
     if (V == 3) {
       const bool two = it.rows > BM;
       // acc b's 4 MMAs of one k-block from stage `st`
       auto issue = [&](int b, int st, int kb) {
         const uint32_t sa = smem_u32(smem + (size_t)st * C::STAGE);
-        const uint32_t sb = sa + C::ABOX * A_STAGE_BYTES;
+        const uint32_t sb = sa + C::ABOX * C::A_BYTES;
         const uint32_t dt = tmem_base + (uint32_t)(b * ACC_COLS);
 #pragma unroll
-        for (int ks = 0; ks < BK / 16; ++ks) {
-          const uint64_t ad = smem_desc_sw128(sa + b * A_STAGE_BYTES + ks * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sb + ks * 2048, B_BOX_BYTES, 1024);
+        for (int ks = 0; ks < C::BK / 16; ++ks) {
+          const uint64_t ad = a_desc<V>(sa + b * C::A_BYTES + ks * 32);
+          const uint64_t bd = smem_desc_sw128(sb + ks * 2048, C::B_BOX, 1024);
           tc_mma_f16(dt, ad, bd, idesc_full, (kb | ks) != 0 ? 1u : 0u);
         }
       };
@@ -840,11 +862,11 @@ __device__ void role_mma(const FfnArgs& a, SmemCtl* ctl, uint8_t* smem, uint32_t
       if (lsu) fence_proxy_async_shared();   // the gather warps' generic-proxy writes
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + (size_t)stage * C::STAGE);
-      const uint32_t sb = sa + A_STAGE_BYTES;
+      const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
-      for (int ks = 0; ks < BK / 16; ++ks) {
-        const uint64_t ad = smem_desc_sw128(sa + ks * 32, 16, 1024);
-        const uint64_t bd = smem_desc_sw128(sb + ks * 2048, B_BOX_BYTES, 1024);
+      for (int ks = 0; ks < C::BK / 16; ++ks) {
+        const uint64_t ad = a_desc<V>(sa + ks * 32);
+        const uint64_t bd = smem_desc_sw128(sb + ks * 2048, C::B_BOX, 1024);
         if (V != 2) tc_mma_f16(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
         else tc_mma_f16_pair(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
       }
@@ -1654,23 +1676,26 @@ static EncodeTiledFn get_encode() {
 }
 
 // bf16 tensor of `rank` dims (innermost first), box of 64 x rows (x 1), 128-B swizzle.
+// bf16, rank 2 or 3: box `inner` x `box_rows` (x 1); the swizzle spans the box's
+// inner bytes (128 or 64).
 static bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-                   const cuuint64_t* strides_bytes, cuuint32_t box_rows) {
+                   const cuuint64_t* strides_bytes, cuuint32_t inner, cuuint32_t box_rows) {
   EncodeTiledFn fn = get_encode();
   if (!fn) return false;
-  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t box[3] = {inner, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = inner * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
-            strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 weights as 4-D {64, K, atoms, E}: box 64 x 64 x `atoms` x 1, 128-B swizzle.
+// bf16 weights as 4-D {64, K, atoms, E}: box 64 x `bk` x `atoms` x 1, 128-B swizzle.
 static bool encode4(CUtensorMap* m, const void* base, const cuuint64_t* dims,
-                    const cuuint64_t* strides_bytes, cuuint32_t atoms) {
+                    const cuuint64_t* strides_bytes, cuuint32_t bk, cuuint32_t atoms) {
   EncodeTiledFn fn = get_encode();
   if (!fn) return false;
-  cuuint32_t box[4] = {64, 64, atoms, 1};
+  cuuint32_t box[4] = {64, bk, atoms, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides_bytes,
             box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1758,17 +1783,20 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   CUtensorMap tm_a1, tm_w1, tm_w3, tm_a2, tm_w2;
   const cuuint64_t R = (cuuint64_t)a.R, d = (cuuint64_t)a.d, f = (cuuint64_t)a.f, E = (cuuint64_t)a.E;
+  // K elements per stage of this variant: the A boxes' inner extent (and swizzle
+  // span) and the weight boxes' K rows
+  const cuuint32_t bk = a.V == 3 ? Cfg<3>::BK : a.V == 2 ? Cfg<2>::BK : Cfg<1>::BK;
   if (a.gather == 1) {
     // token rows of x, boxes one row high for gather4
     const cuuint64_t dims[2] = {d, (cuuint64_t)a.T}, st[1] = {d * 2};
-    if (!encode(&tm_a1, a.x, 2, dims, st, 1)) return cudaErrorInvalidValue;
+    if (!encode(&tm_a1, a.x, 2, dims, st, bk, 1)) return cudaErrorInvalidValue;
   } else {
     const cuuint64_t dims[2] = {d, R}, st[1] = {d * 2};
-    if (!encode(&tm_a1, a.x_perm, 2, dims, st, BM)) return cudaErrorInvalidValue;
+    if (!encode(&tm_a1, a.x_perm, 2, dims, st, bk, BM)) return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[2] = {f, R}, st[1] = {f * 2};
-    if (!encode(&tm_a2, a.h, 2, dims, st, BM)) return cudaErrorInvalidValue;
+    if (!encode(&tm_a2, a.h, 2, dims, st, bk, BM)) return cudaErrorInvalidValue;
   }
   // Single CTAs (V = 1, 3) read the weights through 4-D maps {64 columns, K,
   // 64-column atom, expert} with the atom stride 128 B, so that one box holds
@@ -1781,15 +1809,15 @@ cudaError_t launch_ffn(const FfnArgs& a, int grid, cudaStream_t s) {
   if (a.V != 2 && !(a.flags & MOE_SCHED_B_PER_ATOM)) {
     const cuuint64_t d1[4] = {64, d, f / 64, E}, s1[3] = {f * 2, 128, d * f * 2};
     const cuuint64_t d2[4] = {64, f, d / 64, E}, s2[3] = {d * 2, 128, f * d * 2};
-    args.b_atoms = encode4(&tm_w1, a.W1, d1, s1, 2) && encode4(&tm_w3, a.W3, d1, s1, 2) &&
-                   encode4(&tm_w2, a.W2, d2, s2, 4);
+    args.b_atoms = encode4(&tm_w1, a.W1, d1, s1, bk, 2) && encode4(&tm_w3, a.W3, d1, s1, bk, 2) &&
+                   encode4(&tm_w2, a.W2, d2, s2, bk, 4);
   }
   if (!args.b_atoms) {
     const cuuint64_t dims[3] = {f, d, E}, st[2] = {f * 2, d * f * 2};
-    if (!encode(&tm_w1, a.W1, 3, dims, st, 64)) return cudaErrorInvalidValue;
-    if (!encode(&tm_w3, a.W3, 3, dims, st, 64)) return cudaErrorInvalidValue;
+    if (!encode(&tm_w1, a.W1, 3, dims, st, 64, bk)) return cudaErrorInvalidValue;
+    if (!encode(&tm_w3, a.W3, 3, dims, st, 64, bk)) return cudaErrorInvalidValue;
     const cuuint64_t dims2[3] = {d, f, E}, st2[2] = {d * 2, f * d * 2};
-    if (!encode(&tm_w2, a.W2, 3, dims2, st2, 64)) return cudaErrorInvalidValue;
+    if (!encode(&tm_w2, a.W2, 3, dims2, st2, 64, bk)) return cudaErrorInvalidValue;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);

@@ -117,6 +117,7 @@ def test_layer_small(orc, wl):
                moe.SCHED_GATHER_LSU | wide | moe.SCHED_INTERLEAVE,
                moe.SCHED_GATHER_A | pair, moe.SCHED_GATHER_A | one, moe.SCHED_GATHER_A | wide,
                moe.SCHED_GATHER_A | wide | moe.SCHED_B_PER_ATOM, moe.SCHED_B_PER_ATOM | one,
+               moe.SCHED_B_PER_ATOM | wide,
                moe.SCHED_FULL_TILES | pair, moe.SCHED_INTERLEAVE | one, moe.SCHED_INTERLEAVE | pair,
                moe.SCHED_INTERLEAVE | wide, moe.SCHED_EVICT_FIRST | wide,
                moe.SCHED_EVICT_FIRST | moe.SCHED_INTERLEAVE | one):
@@ -257,7 +258,7 @@ def test_layer_every_token_one_expert(orc, k):
     _check_variants(orc, wl, inp)
 
 
-def test_gather_lsu_refuses_cta_pairs():
+def test_gather_variants_refused():
     # the cp.async gather warps exist for single-CTA tiles only
     wl = synth.WORKLOADS["tiny"]
     inp = gu.inputs(wl)
