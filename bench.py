@@ -43,7 +43,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the persistent FFN kernel, keyed by workload, valid only for the kernel sources
 # whose hash is recorded with it (see profiles/).
-TRAFFIC = {"mixtral": {"bytes": 4165375000 + 311689728, "kernel_hash": "550528ecfe84"}}
+TRAFFIC = {"mixtral": {"bytes": 4202588000 + 312804096, "kernel_hash": "dd7fc0020a58"}}
 
 
 def kernel_source_hash() -> str:
