@@ -149,3 +149,15 @@ def test_ep_owner_host_side_argument_errors():
               None) == moe.MOE_ERR_UNSUPPORTED
     assert hc(P(0x1000), P(0x2000), P(0x3000), P(0x4000), 16, 512, 2, P(0x5000), None, 0,
               None) == moe.MOE_ERR_INVALID
+
+
+def test_debug_tokens_combined_rejects_bad_arguments_on_the_host():
+    # argument checks come before any device call, so they hold without a GPU
+    n = ctypes.c_int(-1)
+    f = moe._lib.moe_debug_tokens_combined
+    assert f(None, 256, 512, 1024, 8, 2, None, ctypes.byref(n)) == moe.MOE_ERR_INVALID          # no ws
+    assert f(ctypes.c_void_p(0x1001), 256, 512, 1024, 8, 2, None, ctypes.byref(n)) == moe.MOE_ERR_INVALID  # misaligned
+    assert f(ctypes.c_void_p(0x1000), 256, 512, 1024, 8, 2, None, None) == moe.MOE_ERR_INVALID   # no output
+    assert f(ctypes.c_void_p(0x1000), 256, 500, 1024, 8, 2, None, ctypes.byref(n)) == moe.MOE_ERR_UNSUPPORTED  # d % 256
+    assert f(ctypes.c_void_p(0x1000), 256, 512, 1024, 8, 9, None, ctypes.byref(n)) == moe.MOE_ERR_INVALID  # k > E
+    assert n.value == -1
