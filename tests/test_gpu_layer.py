@@ -12,7 +12,10 @@
   tokens through the oracle's token-by-token definition path that holds at least
   one routed row of every 128-row band (so every producer tile row group and
   every consumer band is checked), plus the first and last tokens and a seeded
-  random set; overlapped == sequential in full.
+  random set; overlapped == sequential in full.  The same at full size for the
+  other tile variants and the schedule options (side combine warps, the two
+  GEMM1 gathers, the interleaved queue, evict-first stores) on a few layers each,
+  the schedule options also bit-identical to the default in full.
 * The same layers with identity experts (MOE_DBG_IDENTITY_EXPERTS): route,
   permute and combine, checked element by element over the whole output.
 * The oracle's fp32-intermediate variant (h kept in fp32): the GPU output is
@@ -171,13 +174,19 @@ FULL = ["mixtral", "fine_grained", "imbalanced"] + \
 FULL_CASES = [(n, 0) for n in FULL] + [("mixtral", 0x4), ("mixtral", 0x20), ("fine_grained", 0x20),
                                         ("sweep_T512_hot", 0x100)] + \
     [(n, 0x1000) for n in ("mixtral", "fine_grained", "imbalanced", "sweep_T2048_uniform",
-                           "sweep_T32768_uniform", "sweep_T512_zipf")]
-_FLAG_IDS = {0: "default", 0x4: "one", 0x20: "pair", 0x100: "wide", 0x1000: "side"}
+                           "sweep_T32768_uniform", "sweep_T512_zipf")] + \
+    [(n, 0x8000) for n in ("fine_grained", "sweep_T8192_zipf")] + \
+    [(n, 0x10) for n in ("sweep_T2048_hot", "sweep_T512_uniform")] + \
+    [(n, 0x400) for n in ("mixtral", "imbalanced")] + \
+    [(n, 0x800) for n in ("fine_grained", "sweep_T32768_hot")]
+_FLAG_IDS = {0: "default", 0x4: "one", 0x20: "pair", 0x100: "wide", 0x1000: "side", 0x8000: "lsu_gather",
+             0x10: "tma_gather", 0x400: "interleave", 0x800: "evict_first"}
 
 
 @pytest.mark.parametrize("name,flags", FULL_CASES, ids=[f"{n}-{_FLAG_IDS[f]}" for n, f in FULL_CASES])
 def test_layer_full_size_sampled(orc, name, flags):
-    assert flags in (0, moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR, moe.SCHED_WIDE_CTA, moe.SCHED_SIDE_COMBINE)
+    assert flags in (0, moe.SCHED_ONE_CTA, moe.SCHED_CTA_PAIR, moe.SCHED_WIDE_CTA, moe.SCHED_SIDE_COMBINE,
+                     moe.SCHED_GATHER_LSU, moe.SCHED_GATHER_A, moe.SCHED_INTERLEAVE, moe.SCHED_EVICT_FIRST)
     wl = synth.WORKLOADS[name]
     orc.set_threads(os.cpu_count() or 1)
     inp = gu.inputs(wl)
@@ -186,6 +195,11 @@ def test_layer_full_size_sampled(orc, name, flags):
     ovl_bits = gu.host(ovl)
     seq, _, _ = _forward(inp, wl, ws, moe.MODE_SEQUENTIAL, flags=flags)
     assert np.array_equal(gu.host(seq), ovl_bits), "overlapped differs from sequential"
+    if flags in (moe.SCHED_SIDE_COMBINE, moe.SCHED_GATHER_LSU, moe.SCHED_GATHER_A, moe.SCHED_INTERLEAVE,
+                 moe.SCHED_EVICT_FIRST):
+        # a schedule option changes where and when, not what: the default's bits
+        dflt, _, _ = _forward(inp, wl, ws, moe.MODE_OVERLAPPED)
+        assert np.array_equal(gu.host(dflt), ovl_bits), f"flags {flags:#x} differ from the default"
     # routing in full
     oidx, ogate = orc.route(gu.host(inp["logits"]), wl.k)
     assert np.array_equal(gu.host(extra["topk_idx"]), oidx)
