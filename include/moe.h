@@ -47,7 +47,7 @@ extern "C" {
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID = 1,      /* bad argument (null pointer, bad size, misaligned)    */
-  MOE_ERR_UNSUPPORTED = 2,  /* valid MoE shape this build does not handle          */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid MoE shape the library does not handle        */
   MOE_ERR_CUDA = 3,         /* a CUDA call failed                                  */
   MOE_ERR_TIMEOUT = 4,      /* a bounded device wait ran out (see moe_get_status)  */
   MOE_ERR_WORKSPACE = 5     /* workspace missing or smaller than moe_workspace_size */
